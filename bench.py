@@ -1,0 +1,355 @@
+#!/usr/bin/env python
+"""Benchmark of the B200 MoBA causal prefill forward pass.
+
+`python bench.py --gpus N --steps K --warmup W [--config 32k]` prints one JSON
+line. A step is one whole forward pass (pool, gate, router, attention, merge)
+over one synthetic sequence resident in HBM. With N > 1 (launched by
+torch.distributed.run) every rank runs its own independent sequence: weak
+scaling, no collective on the data path (a MAX all-reduce of the timings
+only).
+
+`--impl reference` times the fp64 CPU oracle instead (on rank 0), on a bounded
+sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import synth_inputs as si  # noqa: E402
+
+METRIC = "MoBA prefill tokens/s and effective TFLOP/s (selected blocks) vs bf16 TC roofline"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+FLUSH_BYTES = 256 << 20  # twice the 126 MB L2
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    except (OSError, ValueError):
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def routed_rows(w) -> int:
+    """Past-block partials per step: sum over rows of min(k-1, t//B)."""
+    nb = w.nblocks
+    k_eff = min(w.topk, nb)
+    tot = 0
+    for b in range(nb):
+        n = min(w.seqlen, (b + 1) * w.block_size) - b * w.block_size
+        tot += n * min(k_eff - 1, b)
+    return tot * w.heads_q
+
+
+def stage_bytes(w) -> dict:
+    """Algorithmic HBM bytes per step of the memory-bound stages."""
+    d = w.head_dim
+    k_eff = min(w.topk, w.nblocks)
+    nbp = max(w.nblocks - 1, 0)
+    r = routed_rows(w)
+    return {
+        # read every key that can be pooled once, write the means
+        "pool": nbp * w.block_size * w.heads_kv * d * 2 + nbp * w.heads_kv * d * 4,
+        # read Q once and the means, write the selection table
+        "gate": w.seqlen * w.heads_q * d * 2 + nbp * w.heads_kv * d * 4 + w.seqlen * w.heads_q * k_eff * 4,
+        # read the table and every partial (O fp32 + lse), write out bf16 + lse
+        "merge": w.seqlen * w.heads_q * k_eff * 4 + (r + w.seqlen * w.heads_q) * (d * 4 + 4)
+        + w.seqlen * w.heads_q * (d * 2 + 4),
+    }
+
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_uuid: str | None):
+        self.proc = None
+        self.lines = []
+        cmd = ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "200"]
+        if device_uuid:
+            cmd += ["-i", device_uuid]
+        try:
+            self.proc = subprocess.Popen(cmd, stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.splitlines():
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax.append(float(parts[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def dist_env():
+    return int(os.environ.get("RANK", 0)), int(os.environ.get("WORLD_SIZE", 1)), int(os.environ.get("LOCAL_RANK", 0))
+
+
+# ------------------------------------------------------------------ oracle
+
+def oracle_sample(w, seconds: float, seed: int):
+    """Time the fp64 oracle on a seeded sample of rows of workload w.
+
+    Returns (tokens/s, threads, description). Per-token cost = pool cost / S +
+    (gate + attention cost of one row) * heads_q.
+    """
+    import oracle
+    threads = oracle.threads()
+    rng = np.random.default_rng(seed)
+    q = np.empty((w.seqlen, w.heads_q, w.head_dim), dtype=np.uint16)
+    k = np.empty((w.seqlen, w.heads_kv, w.head_dim), dtype=np.uint16)
+    v = np.empty((w.seqlen, w.heads_kv, w.head_dim), dtype=np.uint16)
+    si.fill_q(q.ctypes.data, w)
+    si.fill_k(k.ctypes.data, w)
+    si.fill_v(v.ctypes.data, w)
+    t0 = time.perf_counter()
+    m = oracle.kmean(k, w.block_size)
+    t_pool = time.perf_counter() - t0
+
+    def run(n):
+        rt = rng.integers(0, w.seqlen, size=n).astype(np.int64)
+        rh = rng.integers(0, w.heads_q, size=n).astype(np.int32)
+        s = time.perf_counter()
+        oracle.attend(q, k, v, w.block_size, w.topk, rt, rh, m=m, nthreads=threads)
+        return time.perf_counter() - s
+
+    n = max(threads, 8)
+    dt = run(n)
+    while dt < 0.5 and n < (1 << 22):
+        n *= 4
+        dt = run(n)
+    n_final = max(n, int(n * max(seconds - t_pool, 0.5) / max(dt, 1e-9)))
+    steps = []
+    return q, k, v, m, t_pool, run, n_final, threads
+
+
+def run_reference(args, w):
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return 0
+    per_step = 3.0
+    q, k, v, m, t_pool, run, n, threads = oracle_sample(w, per_step, w.seed + 4242)
+    for _ in range(args.warmup):
+        run(max(n // 8, 1))
+    times = [run(n) for _ in range(args.steps)]
+    t_row = statistics.mean(times) / n
+    tok_s = 1.0 / (t_pool / w.seqlen + t_row * w.heads_q)
+    line = {
+        "impl": "reference", "metric": METRIC, "value": tok_s, "unit": "tokens/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * w.seqlen / tok_s,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": workload_config(w, args.gpus),
+        "cpu_baseline": {"value": tok_s, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+                         "sample": f"{n} uniformly drawn (token, head) rows per step, gate + masked softmax in fp64; "
+                                   f"full-sequence key mean-pool timed once ({t_pool:.2f} s) and amortised over "
+                                   f"{w.seqlen} tokens"},
+        "e2e": {"value": tok_s, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def workload_config(w, n):
+    return {"workload": w.name, "seqlen": w.seqlen, "heads_q": w.heads_q, "heads_kv": w.heads_kv,
+            "head_dim": w.head_dim, "block_size": w.block_size, "topk": w.topk, "batch_per_gpu": 1,
+            "global_batch": n, "parallelism": f"replicas{n}" if n > 1 else "single",
+            "l2": f"flushed between timed steps ({FLUSH_BYTES >> 20} MiB write)"}
+
+
+# --------------------------------------------------------------------- ours
+
+def run_ours(args, w):
+    import torch
+    import torch.distributed as dist
+
+    import block_sparse_long_fwd_b200 as moba
+
+    rank, world, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=dev)
+    # every rank: its own sequence (independent seed), same shape
+    wr = si.Workload(w.name, w.seqlen, w.heads_q, w.heads_kv, w.head_dim, w.block_size, w.topk,
+                     w.seed + 7919 * rank)
+    S, Hq, Hkv, d = wr.seqlen, wr.heads_q, wr.heads_kv, wr.head_dim
+    q_h = torch.empty((S, Hq, d), dtype=torch.bfloat16, pin_memory=True)
+    k_h = torch.empty((S, Hkv, d), dtype=torch.bfloat16, pin_memory=True)
+    v_h = torch.empty((S, Hkv, d), dtype=torch.bfloat16, pin_memory=True)
+    si.fill_q(q_h.data_ptr(), wr)
+    si.fill_k(k_h.data_ptr(), wr)
+    si.fill_v(v_h.data_ptr(), wr)
+    q, k, v = q_h.to(dev), k_h.to(dev), v_h.to(dev)
+    out = torch.empty_like(q)
+    lse = torch.empty((Hq, S), dtype=torch.float32, device=dev)
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        moba.fwd(q, k, v, wr.block_size, wr.topk, out=out, lse=lse)
+    if moba.device_status() != 0:
+        raise RuntimeError("device status set during warm-up: " + moba.last_error())
+
+    uuid = None
+    try:
+        uuid = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
+    except Exception:  # noqa: BLE001
+        uuid = None
+    sampler = ClockSampler(uuid)
+    time.sleep(0.3)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    moba.profile_begin()
+    for i in range(args.steps):
+        flush.zero_()
+        starts[i].record(stream)
+        moba.fwd(q, k, v, wr.block_size, wr.topk, out=out, lse=lse)
+        ends[i].record(stream)
+    stages, launches, calls = moba.profile_end()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
+    total_ms = sum(step_ms)
+    # keep the GPU busy for >= 1 s so the clock samples see the load
+    t_pad = time.perf_counter()
+    while time.perf_counter() - t_pad < max(0.0, 1.0 - total_ms / 1e3):
+        moba.fwd(q, k, v, wr.block_size, wr.topk, out=out, lse=lse)
+        torch.cuda.synchronize()
+    clocks = sampler.stop()
+    status = moba.device_status()
+    if status != 0:
+        raise RuntimeError("device status set during timing: " + moba.last_error())
+
+    # end to end through the public API: host buffers in, host buffers out
+    out_h = torch.empty((S, Hq, d), dtype=torch.bfloat16, pin_memory=True)
+    lse_h = torch.empty((Hq, S), dtype=torch.float32, pin_memory=True)
+    e2e_steps = max(1, min(args.steps, 10))
+    moba.fwd_host(q_h, k_h, v_h, wr.block_size, wr.topk, out=out_h, lse=lse_h)
+    if world > 1:
+        dist.barrier()
+    e2e_ms = []
+    for _ in range(e2e_steps):
+        t0 = time.perf_counter()
+        moba.fwd_host(q_h, k_h, v_h, wr.block_size, wr.topk, out=out_h, lse=lse_h)
+        e2e_ms.append(1e3 * (time.perf_counter() - t0))
+    e2e_total = sum(e2e_ms)
+
+    # max over ranks of the device time
+    tm = torch.tensor([total_ms, e2e_total, stages["attention"]], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(tm, op=dist.ReduceOp.MAX)
+    total_ms, e2e_total, attn_ms_max = tm.tolist()
+
+    line = None
+    if rank == 0:
+        peaks, peaks_src = load_peaks()
+        flops = moba.effective_flops(S, Hq, wr.block_size, wr.topk, d)
+        value = world * S * args.steps / (total_ms / 1e3)
+        ms_per_step = total_ms / args.steps
+        attn_ms = stages["attention"] / max(calls, 1)
+        long_step = ms_per_step > 200.0
+        peak = peaks["bf16_tflops_sustained"] if long_step else peaks["bf16_tflops"]
+        achieved = flops / (attn_ms / 1e3) / 1e12
+        sb = stage_bytes(wr)
+        stage_roof = {}
+        for st in ("pool", "gate", "merge"):
+            ms = stages[st] / max(calls, 1)
+            if ms > 0:
+                gbs = sb[st] / (ms / 1e3) / 1e9
+                stage_roof[st] = {"ms": ms, "bytes": sb[st], "gbs": gbs, "frac_of_hbm": gbs / peaks["hbm_gbs"]}
+        line = {
+            "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": workload_config(wr, world),
+            "eff_tflops": world * flops * args.steps / (total_ms / 1e3) / 1e12,
+            "stage_ms_per_step": {kk: vv / max(calls, 1) for kk, vv in stages.items()},
+            "roofline": {"bound": "tensor", "kernel": "attn_kernel", "achieved": achieved, "peak": peak,
+                         "unit": "TFLOP/s", "frac": achieved / peak, "traffic": None,
+                         "peak_source": f"{peaks_src} bf16 {'sustained' if long_step else 'burst'}",
+                         "algorithmic": f"{flops:.4e} selected-block FLOPs per step / attention ms per step"},
+            "stage_roofline_hbm": stage_roof,
+            "e2e": {"value": world * S * e2e_steps / (e2e_total / 1e3), "unit": "tokens/s",
+                    "h2d_bytes_per_step": int(q_h.nbytes + k_h.nbytes + v_h.nbytes),
+                    "d2h_bytes_per_step": int(out_h.nbytes + lse_h.nbytes)},
+            "gpu_launches": launches,
+            "gpu_launches_per_step": launches / max(calls, 1),
+            "clocks": clocks,
+            "clocks_window": "timed region, padded with untimed steps to >= 1 s",
+        }
+        if world == 1 and not args.no_cpu_baseline:
+            q_, k_, v_, m_, t_pool, run, n, threads = oracle_sample(wr, args.cpu_seconds, wr.seed + 4242)
+            dt = run(n)
+            tok_s = 1.0 / (t_pool / S + dt / n * Hq)
+            line["cpu_baseline"] = {
+                "value": tok_s, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+                "sample": f"{n} uniformly drawn (token, head) rows, gate + masked softmax in fp64 ({dt:.1f} s); "
+                          f"full-sequence key mean-pool timed once ({t_pool:.2f} s) and amortised over {S} tokens"}
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--config", choices=sorted(si.WORKLOADS), default="32k")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    w = si.WORKLOADS[args.config]
+    if args.impl == "reference":
+        return run_reference(args, w)
+    return run_ours(args, w)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,116 @@
+// Stage 5: log-sum-exp merge of the partial outputs of one query row.
+//
+// A row attends its own block (own-tile partial) and up to k-1 past blocks
+// (routed partials). Each partial i holds the normalised output O_i and
+// lse_i = ln sum exp(scaled logits) over its keys, so the softmax over the
+// union of the selected keys is
+//   L = ln sum_i exp(lse_i),   O = sum_i exp(lse_i - L) O_i,
+// added in a fixed order (ascending block index, own block last). A routed
+// partial of past block j is found through the router's flag words: its
+// list slot is wordbase[g][j][w] + popcount of the bits below the row.
+#pragma once
+
+#include "route.cuh"
+
+namespace moba {
+
+struct MergeParams {
+  const int32_t* sel;
+  const uint32_t* flags;
+  const int32_t* wordbase;
+  const float* part_o;
+  const float* part_lse;
+  const float* own_o;
+  const float* own_lse;
+  __nv_bfloat16* out;  // [S][Hq][128]
+  float* lse;          // [Hq][S]
+  WindowGeom w;
+};
+
+__device__ __forceinline__ float warp_max(float v) {
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+
+__device__ __forceinline__ float warp_sum(float v) {
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+// grid ceil(wlen * Hq / 8), 256 threads: one warp per (token, q head) row,
+// lane c owns channels 4c..4c+3.
+__global__ void __launch_bounds__(256) merge_kernel(MergeParams m) {
+  const WindowGeom& w = m.w;
+  const int lane = threadIdx.x & 31;
+  const int64_t row = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
+  if (row >= w.wlen * w.Hq) return;
+  const int64_t tl = row / w.Hq;
+  const int h = (int)(row % w.Hq);
+  const int64_t t = w.w0 + tl;
+  const int g = h / w.G, hl = h % w.G;
+  const int bt = (int)(t / w.B);
+  const int64_t rr = tl * w.G + hl;
+  const int64_t word = rr >> 5;
+  const uint32_t below = (1u << (rr & 31)) - 1u;
+  const int32_t* srow = m.sel + ((int64_t)h * w.S + t) * w.k_eff;
+  const int P = w.k_eff - 1;
+
+  auto slot = [&](int i, float& li) -> int64_t {
+    li = -INFINITY;
+    if (i >= P) return -1;
+    const int j = __ldg(srow + i);
+    if (j < 0 || j >= bt) return -1;
+    const int64_t f = ((int64_t)g * w.nbp + j) * w.wwords + word;
+    const int64_t pos = (int64_t)__ldg(m.wordbase + f) + __popc(__ldg(m.flags + f) & below);
+    li = __ldg(m.part_lse + pos);
+    return pos;
+  };
+
+  const float own_l = m.own_lse[tl * w.Hq + h];
+  float mx = own_l;
+  for (int i0 = 0; i0 < P; i0 += 32) {
+    float li;
+    slot(i0 + lane, li);
+    mx = fmaxf(mx, warp_max(li));
+  }
+  float sum = 0.f;
+  for (int i0 = 0; i0 < P; i0 += 32) {
+    float li;
+    slot(i0 + lane, li);
+    sum += warp_sum(li == -INFINITY ? 0.f : expf(li - mx));
+  }
+  sum += expf(own_l - mx);
+  const float L = mx + logf(sum);
+
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int i0 = 0; i0 < P; i0 += 32) {
+    float li;
+    const int64_t pos = slot(i0 + lane, li);
+    const int n = min(32, P - i0);
+    for (int k = 0; k < n; ++k) {
+      const int64_t pk = __shfl_sync(0xffffffffu, pos, k);
+      const float lk = __shfl_sync(0xffffffffu, li, k);
+      if (pk >= 0) {
+        const float wk = expf(lk - L);
+        const float4 o = __ldg(reinterpret_cast<const float4*>(m.part_o + pk * kHeadDim) + lane);
+        acc.x += wk * o.x;
+        acc.y += wk * o.y;
+        acc.z += wk * o.z;
+        acc.w += wk * o.w;
+      }
+    }
+  }
+  {
+    const float wk = expf(own_l - L);
+    const float4 o = __ldg(reinterpret_cast<const float4*>(m.own_o + (tl * w.Hq + h) * kHeadDim) + lane);
+    acc.x += wk * o.x;
+    acc.y += wk * o.y;
+    acc.z += wk * o.z;
+    acc.w += wk * o.w;
+  }
+  uint2 packed = make_uint2(pack_bf16x2(acc.x, acc.y), pack_bf16x2(acc.z, acc.w));
+  *reinterpret_cast<uint2*>(m.out + (t * w.Hq + h) * kHeadDim + lane * 4) = packed;
+  if (lane == 0) m.lse[(int64_t)h * w.S + t] = L;
+}
+
+}  // namespace moba

@@ -1,0 +1,565 @@
+// Host side of the C ABI declared in include/moba.h: argument checks,
+// scratch layout, query windows and the launch sequence
+//   pool -> gate -> for each window: route (flags, count, scan, fill)
+//                                    -> attention -> merge.
+#include <cudaTypedefs.h>
+
+#include <algorithm>
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstdlib>
+#include <cstring>
+#include <mutex>
+#include <string>
+#include <vector>
+
+#include "attn.cuh"
+#include "common.cuh"
+#include "merge.cuh"
+#include "pool_gate.cuh"
+#include "route.cuh"
+
+namespace {
+
+thread_local std::string g_err;
+
+int fail(int code, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_err = buf;
+  return code;
+}
+
+#define MOBA_CUDA(call)                                                                                  \
+  do {                                                                                                   \
+    cudaError_t e_ = (call);                                                                             \
+    if (e_ != cudaSuccess) return fail(MOBA_ERR_CUDA, "%s failed: %s", #call, cudaGetErrorString(e_)); \
+  } while (0)
+
+struct DeviceInfo {
+  bool ready = false;
+  bool sm100 = false;
+  int sms = 0;
+};
+
+std::mutex g_dev_mu;
+DeviceInfo g_dev[64];
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+
+int device_info(DeviceInfo* out) {
+  int dev = 0;
+  MOBA_CUDA(cudaGetDevice(&dev));
+  if (dev < 0 || dev >= 64) return fail(MOBA_ERR_UNSUPPORTED, "device index %d out of range", dev);
+  std::lock_guard<std::mutex> lk(g_dev_mu);
+  DeviceInfo& d = g_dev[dev];
+  if (!d.ready) {
+    int major = 0, minor = 0;
+    MOBA_CUDA(cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev));
+    MOBA_CUDA(cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev));
+    MOBA_CUDA(cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev));
+    d.sm100 = (major == 10 && minor == 0);
+    if (d.sm100) {
+      MOBA_CUDA(cudaFuncSetAttribute(moba::attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     moba::kAttnSmemBytes));
+      // keep freed scratch in the stream-ordered pool between calls
+      cudaMemPool_t pool;
+      MOBA_CUDA(cudaDeviceGetDefaultMemPool(&pool, dev));
+      uint64_t thr = UINT64_MAX;
+      MOBA_CUDA(cudaMemPoolSetAttribute(pool, cudaMemPoolAttrReleaseThreshold, &thr));
+    }
+    if (!g_encode) {
+      cudaDriverEntryPointQueryResult q;
+      void* fn = nullptr;
+      MOBA_CUDA(cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &fn, 12000, cudaEnableDefault, &q));
+      if (q != cudaDriverEntryPointSuccess || !fn)
+        return fail(MOBA_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+      g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+    }
+    d.ready = true;
+  }
+  *out = d;
+  if (!d.sm100) return fail(MOBA_ERR_UNSUPPORTED, "device %d is not sm_100 (B200); this library is sm_100a only", dev);
+  return MOBA_OK;
+}
+
+// [S][H][128] bf16 viewed as 3-D (channel, head, token); box 64 x 1 x 128,
+// 128-byte swizzle (one 64-channel half of a 128-token tile per load).
+int make_kv_map(CUtensorMap* map, const void* base, int64_t S, int H) {
+  cuuint64_t dims[3] = {(cuuint64_t)moba::kHeadDim, (cuuint64_t)H, (cuuint64_t)S};
+  cuuint64_t strides[2] = {(cuuint64_t)moba::kHeadDim * 2, (cuuint64_t)H * moba::kHeadDim * 2};
+  cuuint32_t box[3] = {64, 1, (cuuint32_t)moba::kTile};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(MOBA_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+  return MOBA_OK;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
+
+int check_shape(int64_t S, int Hq, int Hkv, int d, int B, int topk) {
+  if (S < 1) return fail(MOBA_ERR_INVALID_ARG, "seqlen must be >= 1 (got %lld)", (long long)S);
+  if (Hkv < 1 || Hq < 1) return fail(MOBA_ERR_INVALID_ARG, "heads must be >= 1 (q %d, kv %d)", Hq, Hkv);
+  if (Hq % Hkv) return fail(MOBA_ERR_INVALID_ARG, "heads_q (%d) must be a multiple of heads_kv (%d)", Hq, Hkv);
+  if (d != MOBA_HEAD_DIM) return fail(MOBA_ERR_INVALID_ARG, "head_dim must be %d (got %d)", MOBA_HEAD_DIM, d);
+  if (B < 128 || B % 128) return fail(MOBA_ERR_INVALID_ARG, "block_size must be a positive multiple of 128 (got %d)", B);
+  if (B > 128 * 1024) return fail(MOBA_ERR_UNSUPPORTED, "block_size above %d is not supported", 128 * 1024);
+  if (topk < 1) return fail(MOBA_ERR_INVALID_ARG, "topk must be >= 1 (got %d)", topk);
+  if (S > (int64_t)INT32_MAX - 2 * B) return fail(MOBA_ERR_UNSUPPORTED, "seqlen too large");
+  const int64_t nb = (S + B - 1) / B;
+  const int64_t k_eff = std::min<int64_t>(topk, nb);
+  if (k_eff < nb && k_eff > MOBA_MAX_TOPK)
+    return fail(MOBA_ERR_UNSUPPORTED, "topk %d above %d with fewer than all blocks is not supported", topk, MOBA_MAX_TOPK);
+  if ((int64_t)Hq * S * k_eff > ((int64_t)1 << 40)) return fail(MOBA_ERR_UNSUPPORTED, "selection table too large");
+  return MOBA_OK;
+}
+
+struct Carve {
+  size_t off = 0;
+  size_t take(size_t bytes) {
+    size_t o = off;
+    off += (bytes + 255) & ~size_t(255);
+    return o;
+  }
+};
+
+struct Plan {
+  int64_t S;
+  int Hq, Hkv, G, B, topk, k_eff, P, nb, nbp;
+  int64_t W;       // window tokens (multiple of 128)
+  int64_t wwords;  // flag words per bucket for a full window
+  int64_t list_cap, tile_cap;
+  size_t o_kmean, o_sel, o_flags, o_wordbase, o_cnt, o_loff, o_toff, o_list, o_tiles, o_hdr, o_part_o, o_part_lse,
+      o_own_o, o_own_lse, total;
+};
+
+size_t window_bytes(const Plan& p, int64_t W) {
+  const int64_t nbk = (int64_t)p.Hkv * p.nbp;
+  const int64_t wwords = (W * p.G + 31) / 32;
+  const int64_t list = W * p.Hq * p.P;
+  const int64_t tiles = list / moba::kTile + nbk + (W / moba::kTile + 1) * p.Hq;
+  return (size_t)(nbk * wwords * 8 + list * (4 + 4 + 4 * moba::kHeadDim) + tiles * 16 +
+                  W * p.Hq * (4 + 4 * moba::kHeadDim));
+}
+
+int make_plan(Plan* pl, int64_t S, int Hq, int Hkv, int B, int topk) {
+  Plan& p = *pl;
+  p.S = S;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.G = Hq / Hkv;
+  p.B = B;
+  p.topk = topk;
+  p.nb = (int)((S + B - 1) / B);
+  p.nbp = p.nb - 1;
+  p.k_eff = std::min(topk, p.nb);
+  p.P = p.k_eff - 1;
+  const int64_t S128 = (S + 127) / 128 * 128;
+  int64_t W = 0;
+  if (const char* env = getenv("MOBA_WINDOW")) {
+    W = atoll(env);
+    W = std::max<int64_t>(128, (W + 127) / 128 * 128);
+  } else {
+    size_t free_b = 0, total_b = 0;
+    if (cudaMemGetInfo(&free_b, &total_b) != cudaSuccess) free_b = (size_t)16 << 30;
+    const size_t budget = std::min<size_t>((size_t)8 << 30, free_b / 3);
+    const size_t per = window_bytes(p, 128);
+    W = std::max<int64_t>(1, (int64_t)(budget / std::max<size_t>(per, 1))) * 128;
+    if (W > 1024 && W % 1024) W = W / 1024 * 1024;
+  }
+  W = std::min(W, S128);
+  // list slots and positions are 32-bit
+  while (W > 128 && W * Hq * (int64_t)p.P >= ((int64_t)1 << 31) - 1) W = std::max<int64_t>(128, W / 2 / 128 * 128);
+  if (W * Hq * (int64_t)p.P >= ((int64_t)1 << 31) - 1) return fail(MOBA_ERR_UNSUPPORTED, "window too large");
+  p.W = W;
+  p.wwords = (W * p.G + 31) / 32;
+  const int64_t nbk = (int64_t)Hkv * p.nbp;
+  p.list_cap = W * Hq * p.P;
+  p.tile_cap = p.list_cap / moba::kTile + nbk + (W / moba::kTile + 1) * Hq;
+  Carve c;
+  p.o_kmean = c.take((size_t)nbk * moba::kHeadDim * 4);
+  p.o_sel = c.take((size_t)Hq * S * p.k_eff * 4);
+  p.o_flags = c.take((size_t)nbk * p.wwords * 4);
+  p.o_wordbase = c.take((size_t)nbk * p.wwords * 4);
+  p.o_cnt = c.take((size_t)(nbk + 1) * 4);
+  p.o_loff = c.take((size_t)(nbk + 1) * 4);
+  p.o_toff = c.take((size_t)(nbk + 1) * 4);
+  p.o_list = c.take((size_t)std::max<int64_t>(p.list_cap, 1) * 4);
+  p.o_tiles = c.take((size_t)p.tile_cap * 16);
+  p.o_hdr = c.take(16);
+  p.o_part_o = c.take((size_t)std::max<int64_t>(p.list_cap, 1) * moba::kHeadDim * 4);
+  p.o_part_lse = c.take((size_t)std::max<int64_t>(p.list_cap, 1) * 4);
+  p.o_own_o = c.take((size_t)W * Hq * moba::kHeadDim * 4);
+  p.o_own_lse = c.take((size_t)W * Hq * 4);
+  p.total = c.off;
+  return MOBA_OK;
+}
+
+template <int KP>
+void launch_gate_kp(const Plan& p, const void* q, const float* kmean, int32_t* sel, cudaStream_t st) {
+  dim3 grid((unsigned)((p.S * p.G + moba::kGateThreads - 1) / moba::kGateThreads), p.Hkv);
+  moba::gate_kernel<KP><<<grid, moba::kGateThreads, 0, st>>>(static_cast<const __nv_bfloat16*>(q), kmean, p.S, p.Hq,
+                                                             p.G, p.B, p.nbp, p.k_eff, sel);
+}
+
+void launch_gate(const Plan& p, const void* q, const float* kmean, int32_t* sel, cudaStream_t st) {
+  const bool full = p.k_eff == p.nb;
+  const int need = full ? 1 : std::max(1, p.P);
+  if (need <= 1) launch_gate_kp<1>(p, q, kmean, sel, st);
+  else if (need <= 2) launch_gate_kp<2>(p, q, kmean, sel, st);
+  else if (need <= 4) launch_gate_kp<4>(p, q, kmean, sel, st);
+  else if (need <= 8) launch_gate_kp<8>(p, q, kmean, sel, st);
+  else if (need <= 16) launch_gate_kp<16>(p, q, kmean, sel, st);
+  else if (need <= 32) launch_gate_kp<32>(p, q, kmean, sel, st);
+  else launch_gate_kp<64>(p, q, kmean, sel, st);
+}
+
+void launch_pool(const Plan& p, const void* k, float* kmean, cudaStream_t st) {
+  if (p.nbp <= 0) return;
+  dim3 grid(p.nbp, p.Hkv);
+  moba::pool_kernel<<<grid, moba::kPoolThreads, 0, st>>>(static_cast<const __nv_bfloat16*>(k), p.Hkv, p.B, p.nbp,
+                                                         kmean);
+}
+
+// Optional per-stage device timing: an event after every stage, tagged with
+// the stage it closes (-1 opens a call); elapsed times between consecutive
+// events are summed per stage when the profile ends.
+enum Stage { kPool = 0, kGate = 1, kRoute = 2, kAttn = 3, kMerge = 4, kNumStages = 5 };
+
+struct StageTimer {
+  bool on = false;
+  cudaStream_t st = nullptr;
+  int launches = 0;
+  int calls = 0;
+  struct Mark {
+    int stage;
+    cudaEvent_t ev;
+  };
+  std::vector<Mark> marks;
+  void mark(int stage) {
+    if (!on) return;
+    cudaEvent_t e;
+    if (cudaEventCreate(&e) != cudaSuccess) return;
+    cudaEventRecord(e, st);
+    marks.push_back({stage, e});
+  }
+  void count(int n) {
+    if (on) launches += n;
+  }
+  int finish(float* ms) {
+    for (int i = 0; i < kNumStages; ++i) ms[i] = 0.f;
+    cudaError_t err = cudaSuccess;
+    if (!marks.empty()) err = cudaEventSynchronize(marks.back().ev);
+    for (size_t i = 1; i < marks.size() && err == cudaSuccess; ++i) {
+      float d = 0.f;
+      if (marks[i].stage >= 0 && cudaEventElapsedTime(&d, marks[i - 1].ev, marks[i].ev) == cudaSuccess)
+        ms[marks[i].stage] += d;
+    }
+    for (auto& m : marks) cudaEventDestroy(m.ev);
+    marks.clear();
+    on = false;
+    if (err != cudaSuccess) return fail(MOBA_ERR_CUDA, "event synchronise failed: %s", cudaGetErrorString(err));
+    return MOBA_OK;
+  }
+};
+
+thread_local StageTimer g_timer;
+
+int run_forward(const Plan& p, const DeviceInfo& dev, const void* q, const void* k, const void* v, void* out,
+                float* lse, uint8_t* ws, cudaStream_t st) {
+  StageTimer* tm = &g_timer;
+  tm->st = st;
+  if (tm->on) tm->calls++;
+  float* kmean = reinterpret_cast<float*>(ws + p.o_kmean);
+  int32_t* sel = reinterpret_cast<int32_t*>(ws + p.o_sel);
+  uint32_t* flags = reinterpret_cast<uint32_t*>(ws + p.o_flags);
+  int32_t* wordbase = reinterpret_cast<int32_t*>(ws + p.o_wordbase);
+  int32_t* cnt = reinterpret_cast<int32_t*>(ws + p.o_cnt);
+  int32_t* loff = reinterpret_cast<int32_t*>(ws + p.o_loff);
+  int32_t* toff = reinterpret_cast<int32_t*>(ws + p.o_toff);
+  int32_t* list = reinterpret_cast<int32_t*>(ws + p.o_list);
+  int4* tiles = reinterpret_cast<int4*>(ws + p.o_tiles);
+  int32_t* hdr = reinterpret_cast<int32_t*>(ws + p.o_hdr);
+  float* part_o = reinterpret_cast<float*>(ws + p.o_part_o);
+  float* part_lse = reinterpret_cast<float*>(ws + p.o_part_lse);
+  float* own_o = reinterpret_cast<float*>(ws + p.o_own_o);
+  float* own_lse = reinterpret_cast<float*>(ws + p.o_own_lse);
+
+  CUtensorMap tmk, tmv;
+  int rc = make_kv_map(&tmk, k, p.S, p.Hkv);
+  if (rc) return rc;
+  rc = make_kv_map(&tmv, v, p.S, p.Hkv);
+  if (rc) return rc;
+
+  tm->mark(-1);
+  if (p.P > 0 && p.k_eff < p.nb && p.nbp > 0) {
+    launch_pool(p, k, kmean, st);
+    tm->count(1);
+    tm->mark(kPool);
+  }
+  launch_gate(p, q, kmean, sel, st);
+  tm->count(1);
+  tm->mark(kGate);
+
+  const int nbk = p.Hkv * p.nbp;
+  moba::AttnParams ap;
+  ap.q = static_cast<const __nv_bfloat16*>(q);
+  ap.list = list;
+  ap.tiles = tiles;
+  ap.hdr = hdr;
+  ap.part_o = part_o;
+  ap.part_lse = part_lse;
+  ap.own_o = own_o;
+  ap.own_lse = own_lse;
+  ap.S = p.S;
+  ap.Hq = p.Hq;
+  ap.G = p.G;
+  ap.B = p.B;
+  ap.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)moba::kHeadDim));
+
+  for (int64_t w0 = 0; w0 < p.S; w0 += p.W) {
+    moba::WindowGeom wg;
+    wg.S = p.S;
+    wg.Hq = p.Hq;
+    wg.Hkv = p.Hkv;
+    wg.G = p.G;
+    wg.B = p.B;
+    wg.k_eff = p.k_eff;
+    wg.nbp = p.nbp;
+    wg.w0 = w0;
+    wg.wlen = std::min(p.W, p.S - w0);
+    wg.wwords = (wg.wlen * p.G + 31) / 32;
+    const bool routed = p.P > 0 && p.nbp > 0 && (w0 + wg.wlen) > p.B;
+    if (routed) {
+      dim3 gf((unsigned)((wg.wwords + 7) / 8), p.Hkv);
+      moba::route_flags_kernel<<<gf, 256, 0, st>>>(sel, wg, flags);
+      dim3 gb(p.nbp, p.Hkv);
+      moba::route_count_kernel<<<gb, 256, 0, st>>>(flags, wg, cnt);
+      tm->count(2);
+    }
+    moba::route_scan_kernel<<<1, 1024, 0, st>>>(cnt, routed ? nbk : 0, wg, loff, toff, tiles, hdr);
+    tm->count(1);
+    if (routed) {
+      dim3 gb(p.nbp, p.Hkv);
+      moba::route_fill_kernel<<<gb, 256, 0, st>>>(flags, cnt, loff, toff, wg, wordbase, list, tiles);
+      tm->count(1);
+    }
+    tm->mark(kRoute);
+    ap.w0 = w0;
+    moba::attn_kernel<<<dev.sms, moba::kAttnThreads, moba::kAttnSmemBytes, st>>>(tmk, tmv, ap);
+    tm->count(1);
+    tm->mark(kAttn);
+    moba::MergeParams mp;
+    mp.sel = sel;
+    mp.flags = flags;
+    mp.wordbase = wordbase;
+    mp.part_o = part_o;
+    mp.part_lse = part_lse;
+    mp.own_o = own_o;
+    mp.own_lse = own_lse;
+    mp.out = static_cast<__nv_bfloat16*>(out);
+    mp.lse = lse;
+    mp.w = wg;
+    const int64_t rows = wg.wlen * p.Hq;
+    moba::merge_kernel<<<(unsigned)((rows + 7) / 8), 256, 0, st>>>(mp);
+    tm->count(1);
+    tm->mark(kMerge);
+  }
+  MOBA_CUDA(cudaGetLastError());
+  return MOBA_OK;
+}
+
+}  // namespace
+
+extern "C" const char* moba_last_error(void) { return g_err.c_str(); }
+
+namespace {
+
+int fwd_impl(const void* q, const void* k, const void* v, int64_t seqlen, int heads_q, int heads_kv, int head_dim,
+             int block_size, int topk, void* out, float* lse, cudaStream_t stream) {
+  g_err.clear();
+  if (!q || !k || !v || !out || !lse) return fail(MOBA_ERR_INVALID_ARG, "null pointer argument");
+  int rc = check_shape(seqlen, heads_q, heads_kv, head_dim, block_size, topk);
+  if (rc) return rc;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(lse))
+    return fail(MOBA_ERR_INVALID_ARG, "device buffers must be 16-byte aligned");
+  DeviceInfo dev;
+  rc = device_info(&dev);
+  if (rc) return rc;
+  Plan p;
+  rc = make_plan(&p, seqlen, heads_q, heads_kv, block_size, topk);
+  if (rc) return rc;
+  void* ws = nullptr;
+  cudaError_t e = cudaMallocAsync(&ws, p.total, stream);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return fail(MOBA_ERR_OOM, "scratch allocation of %zu bytes failed: %s", p.total, cudaGetErrorString(e));
+  }
+  rc = run_forward(p, dev, q, k, v, out, lse, static_cast<uint8_t*>(ws), stream);
+  cudaError_t ef = cudaFreeAsync(ws, stream);
+  if (rc) return rc;
+  if (ef != cudaSuccess) return fail(MOBA_ERR_CUDA, "cudaFreeAsync failed: %s", cudaGetErrorString(ef));
+  return MOBA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int moba_fwd(const void* q, const void* k, const void* v, int64_t seqlen, int heads_q, int heads_kv, int head_dim,
+             int block_size, int topk, void* out, float* lse, cudaStream_t stream) {
+  return fwd_impl(q, k, v, seqlen, heads_q, heads_kv, head_dim, block_size, topk, out, lse, stream);
+}
+
+int moba_profile_begin(void) {
+  g_err.clear();
+  for (auto& m : g_timer.marks) cudaEventDestroy(m.ev);
+  g_timer.marks.clear();
+  g_timer.launches = 0;
+  g_timer.calls = 0;
+  g_timer.on = true;
+  return MOBA_OK;
+}
+
+int moba_profile_end(float* stage_ms, int* launches, int* calls) {
+  g_err.clear();
+  if (!stage_ms || !launches || !calls) return fail(MOBA_ERR_INVALID_ARG, "null pointer argument");
+  int rc = g_timer.finish(stage_ms);
+  *launches = g_timer.launches;
+  *calls = g_timer.calls;
+  return rc;
+}
+
+int moba_fwd_host(const void* q_host, const void* k_host, const void* v_host, int64_t seqlen, int heads_q,
+                  int heads_kv, int head_dim, int block_size, int topk, void* out_host, float* lse_host,
+                  cudaStream_t stream) {
+  g_err.clear();
+  if (!q_host || !k_host || !v_host || !out_host || !lse_host) return fail(MOBA_ERR_INVALID_ARG, "null pointer argument");
+  int rc = check_shape(seqlen, heads_q, heads_kv, head_dim, block_size, topk);
+  if (rc) return rc;
+  DeviceInfo dev;
+  rc = device_info(&dev);
+  if (rc) return rc;
+  const size_t qb = (size_t)seqlen * heads_q * head_dim * 2, kb = (size_t)seqlen * heads_kv * head_dim * 2;
+  const size_t lb = (size_t)seqlen * heads_q * 4;
+  Carve c;
+  const size_t oq = c.take(qb), ok = c.take(kb), ov = c.take(kb), oo = c.take(qb), ol = c.take(lb);
+  void* buf = nullptr;
+  cudaError_t e = cudaMallocAsync(&buf, c.off, stream);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return fail(MOBA_ERR_OOM, "device buffers of %zu bytes: %s", c.off, cudaGetErrorString(e));
+  }
+  uint8_t* b = static_cast<uint8_t*>(buf);
+  rc = MOBA_OK;
+  if (cudaMemcpyAsync(b + oq, q_host, qb, cudaMemcpyHostToDevice, stream) != cudaSuccess ||
+      cudaMemcpyAsync(b + ok, k_host, kb, cudaMemcpyHostToDevice, stream) != cudaSuccess ||
+      cudaMemcpyAsync(b + ov, v_host, kb, cudaMemcpyHostToDevice, stream) != cudaSuccess)
+    rc = fail(MOBA_ERR_CUDA, "host to device copy failed: %s", cudaGetErrorString(cudaGetLastError()));
+  if (!rc)
+    rc = moba_fwd(b + oq, b + ok, b + ov, seqlen, heads_q, heads_kv, head_dim, block_size, topk, b + oo,
+                  reinterpret_cast<float*>(b + ol), stream);
+  if (!rc && (cudaMemcpyAsync(out_host, b + oo, qb, cudaMemcpyDeviceToHost, stream) != cudaSuccess ||
+              cudaMemcpyAsync(lse_host, b + ol, lb, cudaMemcpyDeviceToHost, stream) != cudaSuccess))
+    rc = fail(MOBA_ERR_CUDA, "device to host copy failed: %s", cudaGetErrorString(cudaGetLastError()));
+  cudaFreeAsync(buf, stream);
+  cudaError_t es = cudaStreamSynchronize(stream);
+  if (!rc && es != cudaSuccess) rc = fail(MOBA_ERR_CUDA, "stream synchronise failed: %s", cudaGetErrorString(es));
+  return rc;
+}
+
+int moba_pool(const void* k, int64_t seqlen, int heads_kv, int head_dim, int block_size, float* kmean,
+              cudaStream_t stream) {
+  g_err.clear();
+  if (!k || !kmean) return fail(MOBA_ERR_INVALID_ARG, "null pointer argument");
+  int rc = check_shape(seqlen, heads_kv, heads_kv, head_dim, block_size, 1);
+  if (rc) return rc;
+  if (!aligned16(k) || !aligned16(kmean)) return fail(MOBA_ERR_INVALID_ARG, "device buffers must be 16-byte aligned");
+  DeviceInfo dev;
+  rc = device_info(&dev);
+  if (rc) return rc;
+  Plan p;
+  p.S = seqlen;
+  p.Hkv = heads_kv;
+  p.B = block_size;
+  p.nb = (int)((seqlen + block_size - 1) / block_size);
+  p.nbp = p.nb - 1;
+  launch_pool(p, k, kmean, stream);
+  MOBA_CUDA(cudaGetLastError());
+  return MOBA_OK;
+}
+
+int moba_gate(const void* q, const float* kmean, int64_t seqlen, int heads_q, int heads_kv, int head_dim,
+              int block_size, int topk, int32_t* sel, cudaStream_t stream) {
+  g_err.clear();
+  if (!q || !sel) return fail(MOBA_ERR_INVALID_ARG, "null pointer argument");
+  int rc = check_shape(seqlen, heads_q, heads_kv, head_dim, block_size, topk);
+  if (rc) return rc;
+  const int nb = (int)((seqlen + block_size - 1) / block_size);
+  if (std::min(topk, nb) > 1 && std::min(topk, nb) < nb && !kmean)
+    return fail(MOBA_ERR_INVALID_ARG, "kmean is required when the gate chooses");
+  if (!aligned16(q)) return fail(MOBA_ERR_INVALID_ARG, "device buffers must be 16-byte aligned");
+  DeviceInfo dev;
+  rc = device_info(&dev);
+  if (rc) return rc;
+  Plan p;
+  p.S = seqlen;
+  p.Hq = heads_q;
+  p.Hkv = heads_kv;
+  p.G = heads_q / heads_kv;
+  p.B = block_size;
+  p.nb = nb;
+  p.nbp = nb - 1;
+  p.k_eff = std::min(topk, nb);
+  p.P = p.k_eff - 1;
+  launch_gate(p, q, kmean, sel, stream);
+  MOBA_CUDA(cudaGetLastError());
+  return MOBA_OK;
+}
+
+int moba_device_status(cudaStream_t stream) {
+  g_err.clear();
+  MOBA_CUDA(cudaStreamSynchronize(stream));
+  int s = 0;
+  MOBA_CUDA(cudaMemcpyFromSymbol(&s, moba::g_status, sizeof(int)));
+  const int zero = 0;
+  MOBA_CUDA(cudaMemcpyToSymbol(moba::g_status, &zero, sizeof(int)));
+  if (s) fail(s, "a kernel reported device status %d", s);
+  return s;
+}
+
+}  // extern "C"
+
+namespace moba {
+
+// One thread waits on an mbarrier that nothing ever arrives on.
+__global__ void selftest_wait_kernel(uint64_t timeout_ns) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    abort_flag = 0;
+    fence_barrier_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) mbar_wait(&bar, 0, &abort_flag, timeout_ns);
+}
+
+}  // namespace moba
+
+extern "C" int moba_selftest_bounded_wait(int timeout_us, cudaStream_t stream) {
+  g_err.clear();
+  if (timeout_us < 1 || timeout_us > 2000000) return fail(MOBA_ERR_INVALID_ARG, "timeout_us must be in [1, 2e6]");
+  DeviceInfo dev;
+  int rc = device_info(&dev);
+  if (rc) return rc;
+  rc = moba_device_status(stream);  // clear earlier state
+  moba::selftest_wait_kernel<<<1, 32, 0, stream>>>((uint64_t)timeout_us * 1000ull);
+  MOBA_CUDA(cudaGetLastError());
+  return moba_device_status(stream);
+}

@@ -1,0 +1,160 @@
+/*
+ * moba.h - C ABI of the B200 (sm_100a) MoBA causal prefill forward pass.
+ *
+ * MoBA (Mixture of Block Attention; "MoBA: Mixture of Block Attention for
+ * Long-Context LLMs", abstract) cuts the context into blocks of block_size
+ * tokens, lets a parameter-less top-k gate pick for every query token the
+ * key/value blocks most relevant to it, and runs attention over the picked
+ * blocks only ("MoBA (Mixture of Block Attention)" project summary, section
+ * "How It Works"). Causality: a query never picks a future block, its own
+ * block is always picked, and a causal mask applies inside the own block
+ * ("MoBA - Moonshot AIが提案した新しいアテンションメカニズム", section
+ * "MoBAの技術的原則").
+ *
+ * Conventions of this library (the pages leave them open):
+ *   - gate score of block j for query row (t, h): q[t][h] . mean_{u in blk j}
+ *     k[u][g(h)], unscaled; ties go to the lower block index;
+ *   - the own block counts toward topk: a row attends min(topk, t/B + 1)
+ *     blocks; topk >= number of blocks gives full causal attention;
+ *   - GQA: q head h reads kv head h / (heads_q / heads_kv);
+ *   - softmax scale 1/sqrt(head_dim); lse is the natural log of the sum of
+ *     exp(scaled logits) over the attended keys.
+ *
+ * All tensors are batch 1, dense, row-major:
+ *   q, out : [seqlen][heads_q][head_dim]   bf16
+ *   k, v   : [seqlen][heads_kv][head_dim]  bf16
+ *   lse    : [heads_q][seqlen]             fp32
+ *   kmean  : [heads_kv][nblocks - 1][head_dim] fp32 (only blocks that can be
+ *            a past block are pooled; nblocks = ceil(seqlen / block_size))
+ *   sel    : [heads_q][seqlen][min(topk, nblocks)] int32, ascending block
+ *            indices (the own block is last), padded with -1
+ *
+ * Ownership and ordering: the caller owns every buffer. Device pointers must
+ * be 16-byte aligned. Outputs must not alias inputs. Calls are asynchronous
+ * on `stream`; the library keeps no pointer after a call returns. Scratch
+ * memory is taken from the stream-ordered allocator (cudaMallocAsync) and
+ * returned (cudaFreeAsync) on the same stream inside each call.
+ *
+ * Errors: argument checks run before any launch and return a nonzero
+ * moba_status; moba_last_error() then gives a message (thread-local). Device
+ * side faults that the kernels detect (a bounded wait that ran out, an index
+ * check) are recorded in a per-device status word that moba_device_status()
+ * reads after synchronising the stream.
+ */
+#ifndef MOBA_B200_H
+#define MOBA_B200_H
+
+#include <stdint.h>
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    MOBA_OK = 0,
+    MOBA_ERR_INVALID_ARG = 1,    /* null pointer, bad shape, misaligned    */
+    MOBA_ERR_UNSUPPORTED = 2,    /* device is not sm_100, or a shape limit */
+    MOBA_ERR_OOM = 3,            /* scratch allocation failed              */
+    MOBA_ERR_CUDA = 4,           /* a CUDA runtime call failed             */
+    MOBA_ERR_DEVICE_TIMEOUT = 5, /* a kernel's bounded wait ran out        */
+    MOBA_ERR_DEVICE_CHECK = 6    /* a kernel's index check failed          */
+} moba_status;
+
+/* Limits checked before launch. */
+#define MOBA_HEAD_DIM 128      /* head_dim must equal this                  */
+#define MOBA_MAX_TOPK 64       /* topk - 1 past blocks at most, unless topk >= nblocks */
+
+/*
+ * moba_fwd - the whole forward pass: key mean-pool, gate + top-k, router,
+ * block attention and log-sum-exp merge, all on the GPU.
+ *
+ * q, k, v    device bf16 inputs (layouts above).
+ * seqlen     number of tokens, >= 1.
+ * heads_q    query heads, a positive multiple of heads_kv.
+ * heads_kv   key/value heads, >= 1.
+ * head_dim   must be 128.
+ * block_size tokens per block: a positive multiple of 128. seqlen need not
+ *            be a multiple of it (the last block is then partial).
+ * topk       blocks per query including its own block, >= 1. Values above
+ *            the number of blocks are clamped (full causal attention). When
+ *            topk < nblocks, topk - 1 must not exceed MOBA_MAX_TOPK.
+ * out        device bf16 output [seqlen][heads_q][head_dim].
+ * lse        device fp32 output [heads_q][seqlen].
+ * stream     CUDA stream for every launch and the scratch memory.
+ *
+ * Returns MOBA_OK once all work is queued. Scratch size grows with seqlen;
+ * long sequences are processed in query windows whose size the library
+ * picks (environment MOBA_WINDOW=<tokens> overrides it, rounded to 128).
+ */
+int moba_fwd(const void* q, const void* k, const void* v, int64_t seqlen,
+             int heads_q, int heads_kv, int head_dim, int block_size, int topk,
+             void* out, float* lse, cudaStream_t stream);
+
+/*
+ * moba_fwd_host - moba_fwd on HOST buffers (same layouts): copies q, k, v to
+ * the device, runs the forward pass and copies out and lse back, all on
+ * `stream`, and synchronises the stream before returning. Host buffers that
+ * are page-locked (cudaHostAlloc / pinned) copy fastest. Device buffers come
+ * from the stream-ordered allocator and are released before returning.
+ */
+int moba_fwd_host(const void* q_host, const void* k_host, const void* v_host,
+                  int64_t seqlen, int heads_q, int heads_kv, int head_dim,
+                  int block_size, int topk, void* out_host, float* lse_host,
+                  cudaStream_t stream);
+
+/*
+ * moba_pool - the first stage alone: kmean[g][j][:] = mean of k[t][g][:]
+ * over the tokens t of block j, for j < nblocks - 1 (fp32 accumulation, fixed
+ * order). kmean is a device fp32 buffer [heads_kv][nblocks-1][head_dim].
+ * Does nothing when nblocks == 1.
+ */
+int moba_pool(const void* k, int64_t seqlen, int heads_kv, int head_dim,
+              int block_size, float* kmean, cudaStream_t stream);
+
+/*
+ * moba_gate - the second stage alone: gate scores q . kmean over past blocks
+ * and the per-row top-(k-1) with the own block forced, written as `sel`
+ * (layout above). kmean as produced by moba_pool.
+ */
+int moba_gate(const void* q, const float* kmean, int64_t seqlen, int heads_q,
+              int heads_kv, int head_dim, int block_size, int topk,
+              int32_t* sel, cudaStream_t stream);
+
+/*
+ * Per-stage device timing of the forward passes issued from this host
+ * thread. After moba_profile_begin(), every moba_fwd call also records CUDA
+ * events on its stream between its stages (no extra synchronisation).
+ * moba_profile_end() waits for the last recorded event, writes the summed
+ * milliseconds per stage to stage_ms[0..4] = {pool, gate, route, attention,
+ * merge}, the number of kernels launched to *launches and the number of
+ * forward calls to *calls, then turns the timing off. Returns a moba_status.
+ */
+int moba_profile_begin(void);
+int moba_profile_end(float* stage_ms, int* launches, int* calls);
+
+/* Message of the last failed call on this host thread ("" if none). */
+const char* moba_last_error(void);
+
+/*
+ * Synchronises `stream`, then returns and clears the status word that the
+ * kernels on the current device write when a bounded wait runs out
+ * (MOBA_ERR_DEVICE_TIMEOUT) or an index check fails (MOBA_ERR_DEVICE_CHECK);
+ * MOBA_OK when neither happened. The word is shared by every call on the
+ * device since the last read.
+ */
+int moba_device_status(cudaStream_t stream);
+
+/*
+ * Launches one tiny kernel whose single wait can never be satisfied, bounded
+ * at `timeout_us` microseconds, and returns the status it leaves
+ * (MOBA_ERR_DEVICE_TIMEOUT when the bound works). It exercises the same
+ * bounded-wait helper the attention kernel uses, without faulting the GPU.
+ */
+int moba_selftest_bounded_wait(int timeout_us, cudaStream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOBA_B200_H */

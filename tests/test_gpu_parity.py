@@ -1,0 +1,105 @@
+"""GPU parity: the CUDA path through the C ABI against the fp64 oracle.
+
+Small cases check every row; the large workloads (128K, 1M, 10M tokens) run
+in the configuration the benchmark times and are checked on sampled rows
+(edge rows plus a seeded uniform sample), which the oracle computes one by
+one. Tolerances live in parity_helpers.
+"""
+import os
+
+import numpy as np
+import pytest
+
+import oracle
+import synth_inputs as si
+from parity_helpers import full_check, make_inputs, run_gpu
+
+pytestmark = pytest.mark.gpu
+
+torch = pytest.importorskip("torch")
+if not torch.cuda.is_available():  # pragma: no cover
+    pytest.skip("no CUDA device", allow_module_level=True)
+
+
+SMALL = [
+    # S,    Hq, Hkv, B,   topk, seed
+    (1,     1,  1,   128, 3,    1),     # one token
+    (100,   2,  1,   128, 3,    2),     # shorter than a block
+    (1000,  4,  2,   128, 3,    3),     # ragged tail, GQA
+    (1536,  3,  1,   128, 4,    4),     # group size 3
+    (2048,  8,  8,   256, 2,    5),     # MHA
+    (4096,  2,  1,   128, 1,    6),     # topk 1: own block only
+    (1536,  2,  1,   128, 20,   7),     # topk >= blocks: full causal attention
+    (2125,  2,  1,   256, 5,    8),     # ragged, several routed blocks
+    (8192,  4,  1,   512, 9,    9),     # many past blocks per row
+]
+
+
+@pytest.mark.parametrize("S,Hq,Hkv,B,topk,seed", SMALL)
+def test_small_all_rows(S, Hq, Hkv, B, topk, seed):
+    w, q, k, v = make_inputs(S, Hq, Hkv, B, topk, seed)
+    stats = full_check(q, k, v, B, topk)
+    print(stats)
+
+
+@pytest.mark.parametrize("window", [128, 384, 1024])
+def test_query_windows(monkeypatch, window):
+    S, Hq, Hkv, B, topk = 2125, 4, 2, 256, 4
+    w, q, k, v = make_inputs(S, Hq, Hkv, B, topk, 40 + window)
+    monkeypatch.setenv("MOBA_WINDOW", str(window))
+    stats = full_check(q, k, v, B, topk)
+    print(window, stats)
+
+
+@pytest.mark.parametrize("name", ["4k", "32k"])
+def test_workload_all_rows(name):
+    w = si.WORKLOADS[name]
+    q, k, v = si.make_qkv(w)
+    stats = full_check(q, k, v, w.block_size, w.topk)
+    print(name, stats)
+
+
+def test_deterministic_bits():
+    w = si.WORKLOADS["32k"]
+    q, k, v = si.make_qkv(w)
+    a = run_gpu(q, k, v, w.block_size, w.topk)
+    b = run_gpu(q, k, v, w.block_size, w.topk)
+    assert torch.equal(a[0], b[0])
+    for x, y in zip(a[1:], b[1:]):
+        assert np.array_equal(x, y)
+
+
+def sample_rows(w, n, seed):
+    rng = np.random.default_rng(seed)
+    S, Hq, B = w.seqlen, w.heads_q, w.block_size
+    t = rng.choice(S, size=n, replace=False).astype(np.int64)
+    edge = np.array([0, B - 1, B, 2 * B - 1, S - 1, S // 2], dtype=np.int64)
+    t = np.concatenate([edge, t])
+    h = rng.integers(0, Hq, size=t.size).astype(np.int32)
+    return t, h
+
+
+@pytest.mark.parametrize("name,nrows", [("128k", 256), ("1m", 128), ("10m", 128)])
+def test_large_workload_sampled_rows(name, nrows):
+    w = si.WORKLOADS[name]
+    q, k, v = si.make_qkv(w)
+    rows = sample_rows(w, nrows, w.seed + 1000)
+    stats = full_check(q, k, v, w.block_size, w.topk, rows=rows)
+    print(name, stats)
+
+
+def test_bounded_wait_reports_timeout():
+    import block_sparse_long_fwd_b200 as moba
+    assert moba.selftest_bounded_wait(20000) == moba.MOBA_ERR_DEVICE_TIMEOUT
+    assert moba.device_status() == 0  # cleared by the read
+
+
+def test_host_entry_point_matches_device_entry_point():
+    import block_sparse_long_fwd_b200 as moba
+    S, Hq, Hkv, B, topk = 3000, 4, 2, 256, 3
+    w, q, k, v = make_inputs(S, Hq, Hkv, B, topk, 77)
+    to_t = lambda a: torch.from_numpy(a.view(np.int16)).view(torch.bfloat16)
+    out_h, lse_h = moba.fwd_host(to_t(q).pin_memory(), to_t(k).pin_memory(), to_t(v).pin_memory(), B, topk)
+    out_d, lse_d, _, _ = run_gpu(q, k, v, B, topk)
+    assert torch.equal(out_h, out_d)
+    assert np.array_equal(lse_h.numpy(), lse_d)
