@@ -155,7 +155,6 @@ def oracle_sample(w, seconds: float, seed: int):
         n *= 4
         dt = run(n)
     n_final = max(n, int(n * max(seconds - t_pool, 0.5) / max(dt, 1e-9)))
-    steps = []
     return q, k, v, m, t_pool, run, n_final, threads
 
 
@@ -253,7 +252,7 @@ def run_ours(args, w):
     total_ms = sum(step_ms)
     # keep the GPU busy for >= 1 s so the clock samples see the load
     t_pad = time.perf_counter()
-    while time.perf_counter() - t_pad < max(0.0, 1.0 - total_ms / 1e3):
+    while not args.no_pad and time.perf_counter() - t_pad < max(0.0, 1.0 - total_ms / 1e3):
         moba.fwd(q, k, v, wr.block_size, wr.topk, out=out, lse=lse)
         torch.cuda.synchronize()
     clocks = sampler.stop()
@@ -342,10 +341,15 @@ def main():
     ap.add_argument("--config", choices=sorted(si.WORKLOADS), default="32k")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--seqlen", type=int, default=0, help="override the workload's seqlen (profiling cases)")
+    ap.add_argument("--no-pad", action="store_true", help="no untimed load after the timed steps (profiling)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     w = si.WORKLOADS[args.config]
+    if args.seqlen:
+        w = si.Workload(f"{w.name}_s{args.seqlen}", args.seqlen, w.heads_q, w.heads_kv, w.head_dim, w.block_size,
+                        w.topk, w.seed)
     if args.impl == "reference":
         return run_reference(args, w)
     return run_ours(args, w)
