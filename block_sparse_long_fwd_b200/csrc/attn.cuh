@@ -1,30 +1,39 @@
 // Stage 4: block attention on the 5th-generation tensor cores.
 //
-// Each work tile is 128 query rows against the keys of one KV block:
-//   routed tile: up to 128 rows routed to past block j of kv head g (from the
-//     router's list), attending all B keys of block j, no mask (j < t/B);
-//   own tile:    128 consecutive tokens of one q head attending their own
-//     block from its start up to the tile, causal mask on the diagonal step
-//     ("MoBA - Moonshot AIが提案した新しいアテンションメカニズム",
+// A work unit is a pair of 128-row query tiles (A and B) that read the same
+// keys, so one K/V stream feeds M = 256 rows:
+//   routed unit: up to 256 rows routed to past block j of kv head g (rows
+//     [0,128) form tile A, [128,256) tile B), attending all B keys of block
+//     j without a mask (j < t/B);
+//   own unit:    128 consecutive tokens of two q heads of one GQA group
+//     (tile B absent when the group has no second head left), attending
+//     their own block from its start up to the tile, causal mask on the
+//     diagonal step ("MoBA - Moonshot AIが提案した新しいアテンションメカニズム",
 //     "MoBAの技術的原則": a causal mask applies inside the current block).
-// Both write a normalised partial output O_i (fp32) and its natural-log
-// lse_i; the merge stage combines them. The FlashAttention-style online
-// softmax ("MoBA - Moonshot AIが提案した新しいアテンションメカニズム",
-// high-performance implementation: FlashAttention plus MoE techniques) runs
-// per 128-key step:
-//   S = Q K^T             tcgen05.mma, A = Q and B = K from shared memory,
-//                         fp32 accumulator in TMEM (two S buffers)
-//   P = exp2(S*c - m)     softmax warps read S from TMEM, one row per thread
-//   O += P V              tcgen05.mma, A = P from shared memory, B = V
-//                         (MN-major) from shared memory, O in TMEM.
-// The running max is only moved (and O, l rescaled) when it grows by more
-// than 8 in log2 units, so most steps skip the O rescale.
+// Every tile writes a normalised partial output O_i (fp32) and its
+// natural-log lse_i; the merge stage combines them. The online softmax
+// (FlashAttention-style; the same page credits MoBA's speed to FlashAttention
+// plus MoE techniques) runs per 128-key step, per tile X in {A, B}:
+//   S_X = Q_X K^T      tcgen05.mma, Q and K from shared memory (128B
+//                      swizzle), fp32 accumulator in TMEM
+//   P_X = 2^(S_X*c-m)  the tile's softmax warpgroup reads S_X from TMEM
+//                      (thread = row = TMEM lane) and writes bf16 P_X back
+//                      over the first 64 columns of S_X
+//   O_X += P_X V       tcgen05.mma with A = P_X from TMEM, B = V (MN-major)
+//                      from shared memory, O_X in TMEM.
+// The tensor core alternates S_A, S_B, PV_A, PV_B, so each softmax
+// warpgroup works while the other tile's products run. The running max moves
+// (and O, l are rescaled) only when it grows by more than 8 in log2 units.
+// A quarter of the exponentials are evaluated on the FMA pipe (range
+// reduction 2^x = 2^n 2^f, |f| <= 1/2, and a minimax cubic for 2^f) to take
+// load off the MUFU unit.
 //
-// Warp roles (256 threads, one CTA per SM, persistent over the tile list):
-//   warps 0-3  softmax + epilogue (thread = row = TMEM lane)
-//   warp 4     TMA producer for K/V tiles (3-D tensor maps, 128B swizzle)
-//   warp 5     TMEM owner and single-thread MMA issuer
-//   warps 6-7  Q row gather (cp.async, 16 B per copy, swizzled by hand)
+// TMEM (512 columns): S_A 0..127, S_B 128..255, O_A 256..383, O_B 384..511.
+// Warp roles (384 threads, one CTA per SM, persistent over the unit list):
+//   warps 0-3  softmax + epilogue of tile A     warps 4-7  same for tile B
+//   warp 8     TMA producer for K/V (3-D tensor maps, 128B swizzle)
+//   warp 9     TMEM owner and single-thread MMA issuer
+//   warps 10-11 Q row gather (cp.async, 16 B per copy, swizzled by hand)
 // Every mbarrier wait is bounded; a timeout sets an error status and the
 // whole CTA winds down without trapping.
 #pragma once
@@ -33,17 +42,19 @@
 
 namespace moba {
 
-constexpr int kAttnThreads = 256;
+constexpr int kAttnThreads = 384;
 constexpr int kStages = 2;
 constexpr uint32_t kTileBytes = kTile * kHeadDim * 2;  // 32 KB: 128 rows x 128 bf16
 constexpr uint32_t kHalfBytes = kTileBytes / 2;        // one 64-column half
-constexpr int kAttnSmemBytes = (2 + 2 * kStages + 1) * kTileBytes + 1024 + 256;
+constexpr int kUnitRows = 2 * kTile;                   // rows of a routed unit
+constexpr int kAttnSmemBytes = (2 + 2 * kStages) * kTileBytes + 1024 + 512;
+constexpr uint32_t kNoHead = 0xFFFFu;
 
 struct AttnParams {
   const __nv_bfloat16* q;   // [S][Hq][128]
   const int32_t* list;      // group-rows of the window, per bucket
-  const int4* tiles;        // tile descriptors
-  const int32_t* hdr;       // [1] = number of tiles
+  const int4* units;        // unit descriptors
+  const int32_t* hdr;       // [1] = number of units
   float* part_o;            // [list entries][128]
   float* part_lse;          // [list entries]
   float* own_o;             // [wlen][Hq][128]
@@ -55,44 +66,101 @@ struct AttnParams {
 
 struct AttnShared {
   uint64_t q_full[2], q_empty[2];
-  uint64_t kv_full[kStages], kv_empty[kStages];
-  uint64_t s_full[2];
-  uint64_t p_full, o_done, o_free, drain;
+  uint64_t k_full[kStages], k_empty[kStages], v_full[kStages], v_empty[kStages];
+  uint64_t s_full[2], p_full[2], pv_done[2], o_free[2];
+  uint64_t drain;
   uint32_t tmem_base;
   int abort_flag;
 };
 
-struct TileInfo {
-  bool own;
-  int nrows, nsteps;
-  int g, h;        // kv head; q head (own tiles)
+// Unit descriptor: routed {list_start, nrows (1..256), g, j >= 0};
+//                  own    {t0, nrows (1..128), hA | hB << 16, -nsteps}.
+struct UnitInfo {
+  bool own, has_b;
+  int nsteps;
+  int g;
   int64_t key0;    // first key of step 0
-  int list_start;  // routed
-  int64_t t0;      // own
+  int rows[2];     // valid rows of tile A, B
+  int h[2];        // own: q heads of tile A, B
+  int list0[2];    // routed: first list slot of tile A, B
+  int64_t t0;      // own: first token
 };
 
-__device__ __forceinline__ TileInfo decode_tile(const AttnParams& p, int idx) {
-  const int4 d = p.tiles[idx];
-  TileInfo ti;
-  ti.nrows = d.y;
+__device__ __forceinline__ UnitInfo decode_unit(const AttnParams& p, int idx) {
+  const int4 d = p.units[idx];
+  UnitInfo u;
   if (d.w < 0) {
-    ti.own = true;
-    ti.nsteps = -d.w;
-    ti.t0 = d.x;
-    ti.h = d.z;
-    ti.g = d.z / p.G;
-    ti.key0 = ti.t0 - (int64_t)(ti.nsteps - 1) * kTile;
-    ti.list_start = 0;
+    u.own = true;
+    u.nsteps = -d.w;
+    u.t0 = d.x;
+    u.h[0] = d.z & 0xFFFF;
+    u.h[1] = (int)((uint32_t)d.z >> 16);
+    u.has_b = (uint32_t)u.h[1] != kNoHead;
+    u.g = u.h[0] / p.G;
+    u.key0 = u.t0 - (int64_t)(u.nsteps - 1) * kTile;
+    u.rows[0] = d.y;
+    u.rows[1] = u.has_b ? d.y : 0;
+    u.list0[0] = u.list0[1] = 0;
   } else {
-    ti.own = false;
-    ti.list_start = d.x;
-    ti.g = d.z;
-    ti.h = 0;
-    ti.key0 = (int64_t)d.w * p.B;
-    ti.nsteps = p.B / kTile;
-    ti.t0 = 0;
+    u.own = false;
+    u.nsteps = p.B / kTile;
+    u.t0 = 0;
+    u.g = d.z;
+    u.key0 = (int64_t)d.w * p.B;
+    u.rows[0] = min(d.y, kTile);
+    u.rows[1] = max(d.y - kTile, 0);
+    u.has_b = u.rows[1] > 0;
+    u.list0[0] = d.x;
+    u.list0[1] = d.x + kTile;
+    u.h[0] = u.h[1] = 0;
   }
-  return ti;
+  return u;
+}
+
+// Minimax cubic for 2^f on [-1/2, 1/2] (relative error 7.5e-5), fitted for
+// this kernel with the Remez exchange algorithm. 2^x = 2^n * 2^f with
+// n = rint(x) taken from the low mantissa bits of x + 1.5*2^23; 2^n is then
+// added to the exponent field of the cubic's value.
+constexpr float kExp2C0 = 0.9999280571937561f;
+constexpr float kExp2C1 = 0.6932609677314758f;
+constexpr float kExp2C2 = 0.2426111251115799f;
+constexpr float kExp2C3 = 0.0551716685295105f;
+
+// P = 2^(s*c - m) for one 128-column row of S held as raw fp32 bits in r,
+// on column pairs with packed fp32 arithmetic; each 32-column chunk of P (16
+// TMEM columns of bf16 pairs) is stored to TMEM at tS as soon as it is
+// ready. Row sums accumulate into sum2 (four packed pairs). With kPoly, one
+// pair in four is evaluated on the FMA pipe (minimax cubic above) instead of
+// MUFU; columns masked to -inf must use the MUFU path (kPoly false).
+template <bool kPoly>
+__device__ __forceinline__ void exp_row(const uint32_t (&r)[128], uint64_t c2, uint64_t nm2, uint64_t (&sum2)[4],
+                                        uint32_t tS) {
+#pragma unroll
+  for (int ch = 0; ch < 4; ++ch) {
+    uint32_t pk[16];
+#pragma unroll
+    for (int e = ch * 32; e < ch * 32 + 32; e += 2) {
+      const uint64_t x2 = f2_fma((uint64_t)r[e] | ((uint64_t)r[e + 1] << 32), c2, nm2);
+      float a, b;
+      if (kPoly && (e & 6) == 6) {
+        const uint64_t xx = f2_pack(fmaxf(f2_lo(x2), -125.f), fmaxf(f2_hi(x2), -125.f));
+        const uint64_t t2 = f2_add(xx, f2_pack(12582912.f, 12582912.f));    // + 1.5 * 2^23
+        const uint64_t n2 = f2_add(t2, f2_pack(-12582912.f, -12582912.f));  // rint(x)
+        const uint64_t fr = f2_fma(n2, f2_pack(-1.f, -1.f), xx);            // x - rint(x)
+        uint64_t q = f2_fma(f2_pack(kExp2C3, kExp2C3), fr, f2_pack(kExp2C2, kExp2C2));
+        q = f2_fma(q, fr, f2_pack(kExp2C1, kExp2C1));
+        q = f2_fma(q, fr, f2_pack(kExp2C0, kExp2C0));
+        a = __int_as_float(__float_as_int(f2_lo(q)) + (__float_as_int(f2_lo(t2)) << 23));
+        b = __int_as_float(__float_as_int(f2_hi(q)) + (__float_as_int(f2_hi(t2)) << 23));
+      } else {
+        a = ex2_approx(f2_lo(x2));
+        b = ex2_approx(f2_hi(x2));
+      }
+      sum2[(e >> 1) & 3] = f2_add(sum2[(e >> 1) & 3], f2_pack(a, b));
+      pk[(e >> 1) & 15] = pack_bf16x2(a, b);
+    }
+    tmem_st16(tS + ch * 16, pk);
+  }
 }
 
 __global__ void __launch_bounds__(kAttnThreads, 1)
@@ -100,37 +168,38 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                 AttnParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* sQ = smem;                              // 2 buffers
-  uint8_t* sK = sQ + 2 * kTileBytes;               // kStages buffers
-  uint8_t* sV = sK + kStages * kTileBytes;         // kStages buffers
-  uint8_t* sP = sV + kStages * kTileBytes;         // 1 buffer
-  AttnShared* sh = reinterpret_cast<AttnShared*>(sP + kTileBytes);
+  uint8_t* sQ = smem;                         // tile A, tile B
+  uint8_t* sK = sQ + 2 * kTileBytes;          // kStages buffers
+  uint8_t* sV = sK + kStages * kTileBytes;    // kStages buffers
+  AttnShared* sh = reinterpret_cast<AttnShared*>(sV + kStages * kTileBytes);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int n_tiles = p.hdr[1];
+  const int n_units = p.hdr[1];
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(&sh->q_full[i], 64);
-      mbar_init(&sh->q_empty[i], 1);
-      mbar_init(&sh->s_full[i], 1);
+    for (int x = 0; x < 2; ++x) {
+      mbar_init(&sh->q_full[x], 64);
+      mbar_init(&sh->q_empty[x], 1);
+      mbar_init(&sh->s_full[x], 1);
+      mbar_init(&sh->p_full[x], 128);
+      mbar_init(&sh->pv_done[x], 1);
+      mbar_init(&sh->o_free[x], 128);
     }
     for (int i = 0; i < kStages; ++i) {
-      mbar_init(&sh->kv_full[i], 1);
-      mbar_init(&sh->kv_empty[i], 1);
+      mbar_init(&sh->k_full[i], 1);
+      mbar_init(&sh->k_empty[i], 1);
+      mbar_init(&sh->v_full[i], 1);
+      mbar_init(&sh->v_empty[i], 1);
     }
-    mbar_init(&sh->p_full, 128);
-    mbar_init(&sh->o_done, 1);
-    mbar_init(&sh->o_free, 128);
     mbar_init(&sh->drain, 1);
     sh->abort_flag = 0;
     fence_barrier_init();
   }
-  if (warp == 5) {
+  if (warp == 9) {
     tmem_alloc(&sh->tmem_base, 512);
     tmem_relinquish();
   }
-  if (warp == 4 && lane == 0) {
+  if (warp == 8 && lane == 0) {
     prefetch_tmap(&tmap_k);
     prefetch_tmap(&tmap_v);
   }
@@ -138,44 +207,64 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = sh->tmem_base;
-  const uint32_t tS[2] = {tmem, tmem + 128};
-  const uint32_t tO = tmem + 256;
   volatile int* abort_flag = &sh->abort_flag;
 
-  if (warp < 4) {
-    // ------------------------------------------------ softmax + epilogue
-    const int row = threadIdx.x;  // TMEM lane
-    const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
-    uint32_t it = 0;
-    for (int tile = blockIdx.x; tile < n_tiles; tile += gridDim.x) {
-      const TileInfo ti = decode_tile(p, tile);
+  // register split: the two softmax warpgroups take 200 per thread, the
+  // producer/MMA/gather warpgroup 104 (256*200 + 128*104 = 64512, exactly
+  // the 384*168 registers the block is launched with)
+  if (warp < 8) {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 200;\n" ::: "memory");
+  } else {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 104;\n" ::: "memory");
+  }
+
+  if (warp < 8) {
+    // -------------------------------------------- softmax + epilogue of tile X
+    const int X = warp >> 2;
+    const int row = threadIdx.x & 127;  // TMEM lane
+    const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
+    const uint32_t tS = tmem + X * 128 + lane_off;
+    const uint32_t tO = tmem + 256 + X * 128 + lane_off;
+    uint32_t sx = 0;  // steps done by tile X
+    for (int ui = blockIdx.x; ui < n_units; ui += gridDim.x) {
+      const UnitInfo u = decode_unit(p, ui);
+      if (X == 1 && !u.has_b) continue;
       float m_run = -INFINITY, l_run = 0.f;
-      for (int s = 0; s < ti.nsteps; ++s) {
-        const uint32_t cur = it + s;
-        const int sb = cur & 1;
-        if (!mbar_wait(&sh->s_full[sb], (cur >> 1) & 1, abort_flag)) goto done;
+      for (int s = 0; s < u.nsteps; ++s, ++sx) {
+        if (!mbar_wait(&sh->s_full[X], sx & 1, abort_flag)) goto done;
         __syncwarp();
         tc_fence_after();
-        float x[128];
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          uint32_t r[32];
-          tmem_ld32(tS[sb] + lane_off + c * 32, r);
+        uint32_t r[128];
+        {
+          uint32_t (&r0)[32] = *reinterpret_cast<uint32_t(*)[32]>(&r[0]);
+          uint32_t (&r1)[32] = *reinterpret_cast<uint32_t(*)[32]>(&r[32]);
+          uint32_t (&r2)[32] = *reinterpret_cast<uint32_t(*)[32]>(&r[64]);
+          uint32_t (&r3)[32] = *reinterpret_cast<uint32_t(*)[32]>(&r[96]);
+          tmem_ld32(tS, r0);
+          tmem_ld32(tS + 32, r1);
+          tmem_ld32(tS + 64, r2);
+          tmem_ld32(tS + 96, r3);
           tmem_ld_wait();
-#pragma unroll
-          for (int e = 0; e < 32; ++e) x[c * 32 + e] = __uint_as_float(r[e]) * p.scale_log2;
         }
-        // causal mask on the diagonal step of an own tile: key > query
-        const bool diag = ti.own && (s == ti.nsteps - 1);
+        // causal mask on the diagonal step of an own unit: key > query
+        const bool diag = u.own && (s == u.nsteps - 1);
         if (diag) {
 #pragma unroll
           for (int e = 0; e < 128; ++e)
-            if (e > row) x[e] = -INFINITY;
+            if (e > row) r[e] = __float_as_uint(-INFINITY);
         }
-        float mx = x[0];
+        // row max: eight independent chains of 3-input max over columns
+        // c, c+8, ..., c+120
+        float mx8[8];
 #pragma unroll
-        for (int e = 1; e < 128; ++e) mx = fmaxf(mx, x[e]);
-        const float m_new = fmaxf(m_run, mx);
+        for (int c = 0; c < 8; ++c) {
+          float m = fmax3(__uint_as_float(r[c]), __uint_as_float(r[c + 8]), __uint_as_float(r[c + 16]));
+#pragma unroll
+          for (int e = 24; e < 120; e += 16) m = fmax3(m, __uint_as_float(r[e + c]), __uint_as_float(r[e + 8 + c]));
+          mx8[c] = fmaxf(m, __uint_as_float(r[120 + c]));
+        }
+        const float mx = fmax3(fmax3(mx8[0], mx8[1], mx8[2]), fmax3(mx8[3], mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7]));
+        const float m_new = fmaxf(m_run, mx * p.scale_log2);
         float m_ref = m_run, factor = 1.f;
         bool rescale = false;
         if (s == 0) {
@@ -185,212 +274,265 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           factor = ex2_approx(m_run - m_new);
           rescale = true;
         }
-        float sum = 0.f;
-        uint32_t pk[64];
-#pragma unroll
-        for (int e = 0; e < 64; ++e) {
-          const float a = ex2_approx(x[2 * e] - m_ref);
-          const float b = ex2_approx(x[2 * e + 1] - m_ref);
-          sum += a + b;
-          pk[e] = pack_bf16x2(a, b);
+        // p = 2^(s*c - m), stored into TMEM over the first 64 columns of S_X
+        {
+          const uint64_t c2 = f2_pack(p.scale_log2, p.scale_log2);
+          const uint64_t nm2 = f2_pack(-m_ref, -m_ref);
+          uint64_t sum2[4] = {0ull, 0ull, 0ull, 0ull};
+          if (diag) {
+            exp_row<false>(r, c2, nm2, sum2, tS);
+          } else {
+            exp_row<true>(r, c2, nm2, sum2, tS);
+          }
+          const uint64_t s01 = f2_add(f2_add(sum2[0], sum2[1]), f2_add(sum2[2], sum2[3]));
+          l_run = l_run * factor + (f2_lo(s01) + f2_hi(s01));
+          m_run = m_ref;
         }
-        l_run = l_run * factor + sum;
-        m_run = m_ref;
-        // the previous P.V must be done before P is overwritten / O rescaled
-        if (s > 0) {
-          if (!mbar_wait(&sh->o_done, (cur - 1) & 1, abort_flag)) goto done;
-          __syncwarp();
-          tc_fence_after();
-        }
+        // O rescale: S_X(s) was issued after PV_X(s-1) completed, so O_X is
+        // settled here, and PV_X(s) waits for p_full below
         if (rescale) {
 #pragma unroll
           for (int c = 0; c < 4; ++c) {
-            uint32_t r[32];
-            tmem_ld32(tO + lane_off + c * 32, r);
+            uint32_t o[32];
+            tmem_ld32(tO + c * 32, o);
             tmem_ld_wait();
 #pragma unroll
-            for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * factor);
-            tmem_st32(tO + lane_off + c * 32, r);
+            for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * factor);
+            tmem_st32(tO + c * 32, o);
           }
-          tmem_st_wait();
         }
-        // P row -> shared memory, K-major, 128B swizzle (16-byte chunk c of
-        // row r lands at chunk c ^ (r & 7))
-#pragma unroll
-        for (int c16 = 0; c16 < 16; ++c16) {
-          const int half = c16 >> 3, c = c16 & 7;
-          uint8_t* dst = sP + half * kHalfBytes + row * 128 + ((c ^ (row & 7)) << 4);
-          *reinterpret_cast<uint4*>(dst) = make_uint4(pk[c16 * 4], pk[c16 * 4 + 1], pk[c16 * 4 + 2], pk[c16 * 4 + 3]);
-        }
-        fence_proxy_async_smem();
+        tmem_st_wait();
         tc_fence_before();
-        mbar_arrive(&sh->p_full);
+        mbar_arrive(&sh->p_full[X]);
       }
       {
-        // epilogue: O / l and lse
-        const uint32_t last = it + ti.nsteps - 1;
-        if (!mbar_wait(&sh->o_done, last & 1, abort_flag)) goto done;
+        // epilogue: O / l and lse for this tile's rows
+        if (!mbar_wait(&sh->pv_done[X], (sx - 1) & 1, abort_flag)) goto done;
         __syncwarp();
         tc_fence_after();
         const float inv_l = 1.f / l_run;
         const float lse = (m_run + log2f(l_run)) * 0.69314718055994530942f;
+        const bool write = row < (X ? u.rows[1] : u.rows[0]);
         float* dst_o;
         float* dst_lse;
-        if (ti.own) {
-          const int64_t r = (ti.t0 + row - p.w0) * p.Hq + ti.h;
-          dst_o = p.own_o + r * kHeadDim;
-          dst_lse = p.own_lse + r;
+        if (u.own) {
+          const int64_t rr = (u.t0 + row - p.w0) * p.Hq + (X ? u.h[1] : u.h[0]);
+          dst_o = p.own_o + rr * kHeadDim;
+          dst_lse = p.own_lse + rr;
         } else {
-          const int64_t r = (int64_t)ti.list_start + row;
-          dst_o = p.part_o + r * kHeadDim;
-          dst_lse = p.part_lse + r;
+          const int64_t rr = (int64_t)(X ? u.list0[1] : u.list0[0]) + row;
+          dst_o = p.part_o + rr * kHeadDim;
+          dst_lse = p.part_lse + rr;
         }
-        const bool write = row < ti.nrows;
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
-          uint32_t r[32];
-          tmem_ld32(tO + lane_off + c * 32, r);
+          uint32_t o[32];
+          tmem_ld32(tO + c * 32, o);
           tmem_ld_wait();
           if (write) {
 #pragma unroll
             for (int e = 0; e < 32; e += 4)
               *reinterpret_cast<float4*>(dst_o + c * 32 + e) =
-                  make_float4(__uint_as_float(r[e]) * inv_l, __uint_as_float(r[e + 1]) * inv_l,
-                              __uint_as_float(r[e + 2]) * inv_l, __uint_as_float(r[e + 3]) * inv_l);
+                  make_float4(__uint_as_float(o[e]) * inv_l, __uint_as_float(o[e + 1]) * inv_l,
+                              __uint_as_float(o[e + 2]) * inv_l, __uint_as_float(o[e + 3]) * inv_l);
           }
         }
         if (write) *dst_lse = lse;
         tc_fence_before();
-        mbar_arrive(&sh->o_free);
+        mbar_arrive(&sh->o_free[X]);
       }
-      it += ti.nsteps;
     }
-  } else if (warp == 4) {
+  } else if (warp == 8) {
     // ------------------------------------------------ K/V TMA producer
     if (lane == 0) {
       uint32_t it = 0;
-      for (int tile = blockIdx.x; tile < n_tiles; tile += gridDim.x) {
-        const TileInfo ti = decode_tile(p, tile);
-        for (int s = 0; s < ti.nsteps; ++s, ++it) {
+      for (int ui = blockIdx.x; ui < n_units; ui += gridDim.x) {
+        const UnitInfo u = decode_unit(p, ui);
+        for (int s = 0; s < u.nsteps; ++s, ++it) {
           const int st = it % kStages;
-          if (!mbar_wait(&sh->kv_empty[st], ((it / kStages) & 1) ^ 1, abort_flag)) goto drain_kv;
-          mbar_arrive_expect_tx(&sh->kv_full[st], 2 * kTileBytes);
-          const int key = (int)(ti.key0 + (int64_t)s * kTile);
-          uint8_t* k_dst = sK + st * kTileBytes;
-          uint8_t* v_dst = sV + st * kTileBytes;
-          tma_load_3d(k_dst, &tmap_k, &sh->kv_full[st], 0, ti.g, key);
-          tma_load_3d(k_dst + kHalfBytes, &tmap_k, &sh->kv_full[st], 64, ti.g, key);
-          tma_load_3d(v_dst, &tmap_v, &sh->kv_full[st], 0, ti.g, key);
-          tma_load_3d(v_dst + kHalfBytes, &tmap_v, &sh->kv_full[st], 64, ti.g, key);
+          const uint32_t ph = ((it / kStages) & 1) ^ 1;
+          const int key = (int)(u.key0 + (int64_t)s * kTile);
+          if (!mbar_wait(&sh->k_empty[st], ph, abort_flag)) goto drain_kv;
+          mbar_arrive_expect_tx(&sh->k_full[st], kTileBytes);
+          tma_load_3d(sK + st * kTileBytes, &tmap_k, &sh->k_full[st], 0, u.g, key);
+          tma_load_3d(sK + st * kTileBytes + kHalfBytes, &tmap_k, &sh->k_full[st], 64, u.g, key);
+          if (!mbar_wait(&sh->v_empty[st], ph, abort_flag)) goto drain_kv;
+          mbar_arrive_expect_tx(&sh->v_full[st], kTileBytes);
+          tma_load_3d(sV + st * kTileBytes, &tmap_v, &sh->v_full[st], 0, u.g, key);
+          tma_load_3d(sV + st * kTileBytes + kHalfBytes, &tmap_v, &sh->v_full[st], 64, u.g, key);
         }
       }
     drain_kv:
-      // make sure no TMA write is still in flight when the CTA ends: the
-      // last kStages loads are waited for (bounded) on their full barriers
+      // no TMA write may still be in flight when the CTA ends
       if (*abort_flag) {
         volatile int keep_waiting = 0;
-        for (uint32_t k = (it > (uint32_t)kStages ? it - kStages : 0); k < it; ++k)
-          mbar_wait(&sh->kv_full[k % kStages], (k / kStages) & 1, &keep_waiting, 100000000ull);
+        for (uint32_t k = (it > (uint32_t)kStages ? it - kStages : 0); k <= it; ++k) {
+          mbar_wait(&sh->k_full[k % kStages], (k / kStages) & 1, &keep_waiting, (1ull << 28));
+          mbar_wait(&sh->v_full[k % kStages], (k / kStages) & 1, &keep_waiting, (1ull << 28));
+        }
       }
     }
-  } else if (warp == 5) {
+  } else if (warp == 9) {
     // ------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      const uint32_t idesc_s = idesc_bf16_f32(128, 128, false);
-      const uint32_t idesc_o = idesc_bf16_f32(128, 128, true);
-      const uint32_t aQ0 = smem_u32(sQ), aK0 = smem_u32(sK), aV0 = smem_u32(sV), aP = smem_u32(sP);
-      uint32_t it = 0, n = 0;
-      for (int tile = blockIdx.x; tile < n_tiles; tile += gridDim.x, ++n) {
-        const TileInfo ti = decode_tile(p, tile);
-        const int qb = n & 1;
-        if (!mbar_wait(&sh->q_full[qb], (n >> 1) & 1, abort_flag)) goto mma_done;
-        tc_fence_after();
-        const uint32_t aQ = aQ0 + qb * kTileBytes;
-        // S_{step} = Q K_step^T into S buffer (step & 1)
-        auto issue_s = [&](uint32_t step) -> bool {
-          const int st = step % kStages;
-          if (!mbar_wait(&sh->kv_full[st], (step / kStages) & 1, abort_flag)) return false;
-          tc_fence_after();
-          const uint32_t aK = aK0 + st * kTileBytes;
+    // Per step s the tensor core runs, for each tile X in turn,
+    //   PV_X(s), then S_X(s+1) as two N = 64 halves: columns 64..127 first
+    //   (they do not hold P_X(s)), then, once PV_X(s) has completed,
+    //   columns 0..63.
+    // So tile A's softmax of step s+1 overlaps PV_B(s) and S_B(s+1), and
+    // tile B's overlaps PV_A(s+1) and S_A(s+2). The whole warp runs the loop
+    // (descriptors stay warp-uniform); lane 0 issues every MMA and commit.
+    // lane 0 (the lane elect.sync picks in a converged warp) issues every
+    // MMA and commit
+    const uint32_t idesc_s = idesc_bf16_f32(128, 64, false);
+    const uint32_t idesc_o = idesc_bf16_f32(128, 128, true);
+    // Descriptors are built once; moving the start address by b bytes adds
+    // b >> 4 to the descriptor (the 14-bit start field cannot carry inside
+    // the 228 KB of shared memory).
+    const uint64_t dQ = sdesc_sw128(smem_u32(sQ), 16, 1024);
+    const uint64_t dK = sdesc_sw128(smem_u32(sK), 16, 1024);
+    const uint64_t dV = sdesc_sw128(smem_u32(sV), kHalfBytes, 1024);
+    uint32_t it = 0;          // K/V steps
+    uint32_t sx[2] = {0, 0};  // steps per tile
+    uint32_t ux[2] = {0, 0};  // units per tile
+    // S_X = Q_X K^T for keys [64*half, 64*half + 64) of K stage st
+    auto issue_s_half = [&](int x, int half, int st) {
+      const uint64_t q0 = dQ + ((x * kTileBytes) >> 4);
+      const uint64_t k0 = dK + ((st * kTileBytes + half * 64 * 128) >> 4);
+      const uint32_t d = tmem + x * 128 + half * 64;
+      if (elect_one()) {
 #pragma unroll
-          for (int kk = 0; kk < 8; ++kk) {
-            const uint32_t off = (kk >> 2) * kHalfBytes + (kk & 3) * 32;
-            mma_bf16_ss(tS[step & 1], sdesc_sw128(aQ + off, 16, 1024), sdesc_sw128(aK + off, 16, 1024), idesc_s,
-                        kk > 0);
-          }
-          mma_commit(&sh->s_full[step & 1]);
-          return true;
-        };
-        if (!issue_s(it)) goto mma_done;
-        for (int s = 0; s < ti.nsteps; ++s) {
-          const uint32_t cur = it + s;
-          if (s + 1 < ti.nsteps && !issue_s(cur + 1)) goto mma_done;
-          if (!mbar_wait(&sh->p_full, cur & 1, abort_flag)) goto mma_done;
-          if (s == 0 && n > 0 && !mbar_wait(&sh->o_free, (n - 1) & 1, abort_flag)) goto mma_done;
-          tc_fence_after();
-          const int st = cur % kStages;
-          const uint32_t aV = aV0 + st * kTileBytes;
-#pragma unroll
-          for (int kk = 0; kk < 8; ++kk) {
-            const uint32_t offp = (kk >> 2) * kHalfBytes + (kk & 3) * 32;
-            mma_bf16_ss(tO, sdesc_sw128(aP + offp, 16, 1024), sdesc_sw128(aV + kk * 2048, kHalfBytes, 1024),
-                        idesc_o, (s > 0 || kk > 0) ? 1u : 0u);
-          }
-          mma_commit(&sh->kv_empty[st]);
-          mma_commit(&sh->o_done);
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint32_t off = ((kk >> 2) * kHalfBytes + (kk & 3) * 32) >> 4;
+          mma_bf16_ss(d, q0 + off, k0 + off, idesc_s, kk > 0);
         }
-        mma_commit(&sh->q_empty[qb]);
-        it += ti.nsteps;
       }
-    mma_done:
-      // all issued MMAs must finish before TMEM is released
-      mma_commit(&sh->drain);
+      __syncwarp();
+    };
+    auto commit = [&](uint64_t* bar) {
+      if (elect_one()) mma_commit(bar);
+      __syncwarp();
+    };
+    for (int ui = blockIdx.x; ui < n_units; ui += gridDim.x) {
+      const UnitInfo u = decode_unit(p, ui);
+      const int nx = u.has_b ? 2 : 1;
+#pragma unroll
+      for (int x = 0; x < 2; ++x)
+        if (x < nx && !mbar_wait(&sh->q_full[x], ux[x] & 1, abort_flag)) goto mma_done;
+      {
+        // prologue: S_X(0)
+        const int st0 = it % kStages;
+        if (!mbar_wait(&sh->k_full[st0], (it / kStages) & 1, abort_flag)) goto mma_done;
+        tc_fence_after();
+#pragma unroll
+        for (int x = 0; x < 2; ++x) {
+          if (x >= nx) break;
+          issue_s_half(x, 1, st0);
+          // columns 0..63 held P_X of this tile's previous step
+          if (sx[x] > 0 && !mbar_wait(&sh->pv_done[x], (sx[x] - 1) & 1, abort_flag)) goto mma_done;
+          tc_fence_after();
+          issue_s_half(x, 0, st0);
+          commit(&sh->s_full[x]);
+          if (u.nsteps == 1) commit(&sh->q_empty[x]);
+        }
+        commit(&sh->k_empty[st0]);
+      }
+      for (int s = 0; s < u.nsteps; ++s) {
+        const uint32_t cur = it + s;
+        const int st = cur % kStages, nst = (cur + 1) % kStages;
+        const bool has_next = s + 1 < u.nsteps;
+        if (!mbar_wait(&sh->v_full[st], (cur / kStages) & 1, abort_flag)) goto mma_done;
+        if (has_next && !mbar_wait(&sh->k_full[nst], ((cur + 1) / kStages) & 1, abort_flag)) goto mma_done;
+        const uint64_t v0 = dV + ((st * kTileBytes) >> 4);
+#pragma unroll
+        for (int x = 0; x < 2; ++x) {
+          if (x >= nx) break;
+          if (!mbar_wait(&sh->p_full[x], sx[x] & 1, abort_flag)) goto mma_done;
+          if (s == 0 && ux[x] > 0 && !mbar_wait(&sh->o_free[x], (ux[x] - 1) & 1, abort_flag)) goto mma_done;
+          tc_fence_after();
+          const uint32_t tP = tmem + x * 128;
+          const uint32_t tOx = tmem + 256 + x * 128;
+          if (elect_one()) {
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk)
+              mma_bf16_ts(tOx, tP + kk * 8, v0 + ((kk * 2048) >> 4), idesc_o, (s > 0 || kk > 0) ? 1u : 0u);
+          }
+          __syncwarp();
+          commit(&sh->pv_done[x]);
+          if (has_next) {
+            issue_s_half(x, 1, nst);
+            if (!mbar_wait(&sh->pv_done[x], sx[x] & 1, abort_flag)) goto mma_done;
+            tc_fence_after();
+            issue_s_half(x, 0, nst);
+            commit(&sh->s_full[x]);
+            if (s + 1 == u.nsteps - 1) commit(&sh->q_empty[x]);
+          }
+          ++sx[x];
+        }
+        commit(&sh->v_empty[st]);
+        if (has_next) commit(&sh->k_empty[nst]);
+      }
+      it += u.nsteps;
+      ux[0] += 1;
+      ux[1] += (nx > 1) ? 1 : 0;
+    }
+  mma_done:
+    // every issued MMA must finish before TMEM is released
+    __syncwarp();
+    if (elect_one()) mma_commit(&sh->drain);
+    __syncwarp();
+    {
       volatile int keep_waiting = 0;
-      mbar_wait(&sh->drain, 0, &keep_waiting, 100000000ull);
+      mbar_wait(&sh->drain, 0, &keep_waiting, (1ull << 28));
     }
   } else {
-    // ------------------------------------------------ Q gather (warps 6, 7)
-    const int gt = threadIdx.x - 192;  // 0..63
-    uint32_t n = 0;
-    for (int tile = blockIdx.x; tile < n_tiles; tile += gridDim.x, ++n) {
-      const TileInfo ti = decode_tile(p, tile);
-      const int qb = n & 1;
-      if (!mbar_wait(&sh->q_empty[qb], ((n >> 1) & 1) ^ 1, abort_flag)) break;
-      const uint32_t dst0 = smem_u32(sQ + qb * kTileBytes);
+    // ------------------------------------------------ Q gather (warps 10, 11)
+    const int gt = threadIdx.x - 320;  // 0..63
+    uint32_t ux[2] = {0, 0};
+    for (int ui = blockIdx.x; ui < n_units; ui += gridDim.x) {
+      const UnitInfo u = decode_unit(p, ui);
+      const int nx = u.has_b ? 2 : 1;
+#pragma unroll
+      for (int x = 0; x < 2; ++x) {
+        if (x >= nx) break;
+        if (!mbar_wait(&sh->q_empty[x], (ux[x] & 1) ^ 1, abort_flag)) goto gather_done;
+        const uint32_t dst0 = smem_u32(sQ + x * kTileBytes);
 #pragma unroll 4
-      for (int i = 0; i < 32; ++i) {
-        const int idx = gt + 64 * i;  // 2048 chunks of 16 B
-        const int r = idx >> 4, c16 = idx & 15;
-        const int half = c16 >> 3, c = c16 & 7;
-        const __nv_bfloat16* src = p.q;
-        uint32_t bytes = 0;
-        if (r < ti.nrows) {
-          int64_t t;
-          int h;
-          if (ti.own) {
-            t = ti.t0 + r;
-            h = ti.h;
-          } else {
-            const int rr = __ldg(p.list + ti.list_start + r);
-            t = p.w0 + rr / p.G;
-            h = ti.g * p.G + rr % p.G;
+        for (int i = 0; i < 32; ++i) {
+          const int idx = gt + 64 * i;  // 2048 chunks of 16 B
+          const int r = idx >> 4, c16 = idx & 15;
+          const int half = c16 >> 3, c = c16 & 7;
+          const __nv_bfloat16* src = p.q;
+          uint32_t bytes = 0;
+          if (r < u.rows[x]) {
+            int64_t t;
+            int h;
+            if (u.own) {
+              t = u.t0 + r;
+              h = u.h[x];
+            } else {
+              const int rr = __ldg(p.list + u.list0[x] + r);
+              t = p.w0 + rr / p.G;
+              h = u.g * p.G + rr % p.G;
+            }
+            src = p.q + (t * p.Hq + h) * kHeadDim + c16 * 8;
+            bytes = 16;
           }
-          src = p.q + (t * p.Hq + h) * kHeadDim + c16 * 8;
-          bytes = 16;
+          cp_async_16(dst0 + half * kHalfBytes + r * 128 + ((c ^ (r & 7)) << 4), src, bytes);
         }
-        cp_async_16(dst0 + half * kHalfBytes + r * 128 + ((c ^ (r & 7)) << 4), src, bytes);
+        cp_async_wait_all();
+        fence_proxy_async_smem();
+        mbar_arrive(&sh->q_full[x]);
+        ++ux[x];
       }
-      cp_async_wait_all();
-      fence_proxy_async_smem();
-      mbar_arrive(&sh->q_full[qb]);
     }
+  gather_done:
     cp_async_wait_all();
   }
 done:
   __syncwarp();
   tc_fence_before();
   __syncthreads();
-  if (warp == 5) {
+  if (warp == 9) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }

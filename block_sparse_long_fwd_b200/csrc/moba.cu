@@ -142,7 +142,7 @@ size_t window_bytes(const Plan& p, int64_t W) {
   const int64_t nbk = (int64_t)p.Hkv * p.nbp;
   const int64_t wwords = (W * p.G + 31) / 32;
   const int64_t list = W * p.Hq * p.P;
-  const int64_t tiles = list / moba::kTile + nbk + (W / moba::kTile + 1) * p.Hq;
+  const int64_t tiles = list / moba::kUnitRowsRouted + nbk + (W / moba::kTile + 1) * p.Hkv * ((p.G + 1) / 2);
   return (size_t)(nbk * wwords * 8 + list * (4 + 4 + 4 * moba::kHeadDim) + tiles * 16 +
                   W * p.Hq * (4 + 4 * moba::kHeadDim));
 }
@@ -180,7 +180,7 @@ int make_plan(Plan* pl, int64_t S, int Hq, int Hkv, int B, int topk) {
   p.wwords = (W * p.G + 31) / 32;
   const int64_t nbk = (int64_t)Hkv * p.nbp;
   p.list_cap = W * Hq * p.P;
-  p.tile_cap = p.list_cap / moba::kTile + nbk + (W / moba::kTile + 1) * Hq;
+  p.tile_cap = p.list_cap / moba::kUnitRowsRouted + nbk + (W / moba::kTile + 1) * Hkv * ((p.G + 1) / 2);
   Carve c;
   p.o_kmean = c.take((size_t)nbk * moba::kHeadDim * 4);
   p.o_sel = c.take((size_t)Hq * S * p.k_eff * 4);
@@ -310,7 +310,7 @@ int run_forward(const Plan& p, const DeviceInfo& dev, const void* q, const void*
   moba::AttnParams ap;
   ap.q = static_cast<const __nv_bfloat16*>(q);
   ap.list = list;
-  ap.tiles = tiles;
+  ap.units = tiles;
   ap.hdr = hdr;
   ap.part_o = part_o;
   ap.part_lse = part_lse;
@@ -538,7 +538,7 @@ int moba_device_status(cudaStream_t stream) {
 namespace moba {
 
 // One thread waits on an mbarrier that nothing ever arrives on.
-__global__ void selftest_wait_kernel(uint64_t timeout_ns) {
+__global__ void selftest_wait_kernel(uint64_t timeout_cycles) {
   __shared__ uint64_t bar;
   __shared__ int abort_flag;
   if (threadIdx.x == 0) {
@@ -547,7 +547,7 @@ __global__ void selftest_wait_kernel(uint64_t timeout_ns) {
     fence_barrier_init();
   }
   __syncthreads();
-  if (threadIdx.x == 0) mbar_wait(&bar, 0, &abort_flag, timeout_ns);
+  if (threadIdx.x == 0) mbar_wait(&bar, 0, &abort_flag, timeout_cycles);
 }
 
 }  // namespace moba
@@ -559,7 +559,8 @@ extern "C" int moba_selftest_bounded_wait(int timeout_us, cudaStream_t stream) {
   int rc = device_info(&dev);
   if (rc) return rc;
   rc = moba_device_status(stream);  // clear earlier state
-  moba::selftest_wait_kernel<<<1, 32, 0, stream>>>((uint64_t)timeout_us * 1000ull);
+  // the bound counts SM cycles; 2000 per microsecond is about the B200 clock
+  moba::selftest_wait_kernel<<<1, 32, 0, stream>>>((uint64_t)timeout_us * 2000ull);
   MOBA_CUDA(cudaGetLastError());
   return moba_device_status(stream);
 }

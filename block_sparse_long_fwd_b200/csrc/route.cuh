@@ -121,13 +121,19 @@ __device__ __forceinline__ int64_t block_incl_scan_1024(int64_t v, int64_t* scra
   return v;
 }
 
-// Tile descriptor: routed {list_start, nrows, g, j >= 0};
-//                  own    {t0, nrows, h, -nsteps}.
-// hdr[0] = routed tiles, hdr[1] = all tiles, hdr[2] = list entries.
+// Work-unit descriptors for the attention stage (two 128-row query tiles
+// that read the same keys):
+//   routed {list_start, nrows (1..256), g, j >= 0}: 256 consecutive list
+//          entries of bucket (g, j);
+//   own    {t0, nrows (1..128), hA | hB << 16, -nsteps}: 128 tokens of two
+//          q heads of one group (hB = 0xFFFF when the group has an odd
+//          head left over).
+// hdr[0] = routed units, hdr[1] = all units, hdr[2] = list entries.
+constexpr int kUnitRowsRouted = 256;
 // 3. one CTA of 1024 threads.
 __global__ void __launch_bounds__(1024) route_scan_kernel(const int32_t* __restrict__ cnt, int nbuckets,
                                                           WindowGeom w, int32_t* __restrict__ list_off,
-                                                          int32_t* __restrict__ tile_off, int4* __restrict__ tiles,
+                                                          int32_t* __restrict__ tile_off, int4* __restrict__ units,
                                                           int32_t* __restrict__ hdr) {
   __shared__ int64_t scratch[32];
   __shared__ int64_t last[2];
@@ -135,7 +141,7 @@ __global__ void __launch_bounds__(1024) route_scan_kernel(const int32_t* __restr
   for (int base = 0; base < nbuckets; base += 1024) {
     const int b = base + threadIdx.x;
     const int64_t c = b < nbuckets ? cnt[b] : 0;
-    const int64_t nt = (c + kTile - 1) / kTile;
+    const int64_t nt = (c + kUnitRowsRouted - 1) / kUnitRowsRouted;
     const int64_t il = block_incl_scan_1024(c, scratch);
     const int64_t it = block_incl_scan_1024(nt, scratch);
     if (b < nbuckets) {
@@ -152,11 +158,14 @@ __global__ void __launch_bounds__(1024) route_scan_kernel(const int32_t* __restr
     __syncthreads();
   }
   const int n_routed = (int)carry_t;
-  // own-block tiles: 128-token tiles u of the window, all heads; tile u of
-  // block-position p = ((w0/128 + u) mod (B/128)) has p + 1 key steps.
+  // own-block units: 128-token tiles u of the window, one unit per pair of
+  // q heads of a group; tile u of block-position p = ((w0/128 + u) mod
+  // (B/128)) has p + 1 key steps. Units are ordered longest first.
   const int period = w.B / kTile;
   const int64_t nu = (w.wlen + kTile - 1) / kTile;
   const int64_t u_off = w.w0 / kTile;
+  const int npairs = (w.G + 1) / 2;
+  const int per_u = w.Hkv * npairs;
   // count tiles per position p (period <= 1024 checked on the host)
   __shared__ int cntp[1024];
   __shared__ int basep[1024];
@@ -179,11 +188,17 @@ __global__ void __launch_bounds__(1024) route_scan_kernel(const int32_t* __restr
     const int64_t rank = basep[p] + u / period;  // u' < u with the same p: u / period of them
     const int64_t t0 = w.w0 + u * kTile;
     const int nrows = (int)min((int64_t)kTile, w.w0 + w.wlen - t0);
-    for (int h = 0; h < w.Hq; ++h) tiles[n_routed + rank * w.Hq + h] = make_int4((int)t0, nrows, h, -(p + 1));
+    for (int g = 0; g < w.Hkv; ++g) {
+      for (int q = 0; q < npairs; ++q) {
+        const int hA = g * w.G + 2 * q;
+        const int hB = (2 * q + 1 < w.G) ? hA + 1 : 0xFFFF;
+        units[n_routed + rank * per_u + g * npairs + q] = make_int4((int)t0, nrows, hA | (hB << 16), -(p + 1));
+      }
+    }
   }
   if (threadIdx.x == 0) {
     hdr[0] = n_routed;
-    hdr[1] = n_routed + (int)(nu * w.Hq);
+    hdr[1] = n_routed + (int)(nu * per_u);
     hdr[2] = (int)carry_l;
   }
 }
@@ -232,9 +247,10 @@ __global__ void __launch_bounds__(256) route_fill_kernel(const uint32_t* __restr
     running += total;
   }
   const int n = cnt[b];
-  const int ntiles = (n + kTile - 1) / kTile;
-  for (int k = threadIdx.x; k < ntiles; k += 256)
-    tiles[tile_off[b] + k] = make_int4(base + k * kTile, min(kTile, n - k * kTile), g, j);
+  const int nunits = (n + kUnitRowsRouted - 1) / kUnitRowsRouted;
+  for (int k = threadIdx.x; k < nunits; k += 256)
+    tiles[tile_off[b] + k] =
+        make_int4(base + k * kUnitRowsRouted, min(kUnitRowsRouted, n - k * kUnitRowsRouted), g, j);
 }
 
 }  // namespace moba
