@@ -35,6 +35,7 @@ SIGNATURES = {
     "moba_fwd_host": (_i32, [_vp, _vp, _vp, _i64, _i32, _i32, _i32, _i32, _i32, _vp, _vp, _vp]),
     "moba_pool": (_i32, [_vp, _i64, _i32, _i32, _i32, _vp, _vp]),
     "moba_gate": (_i32, [_vp, _vp, _i64, _i32, _i32, _i32, _i32, _i32, _vp, _vp]),
+    "moba_fwd_noalloc": (_i32, [_vp, _vp, _vp, _i64, _i32, _i32, _i32, _i32, _i32, _vp, _vp, _vp]),
     "moba_profile_begin": (_i32, []),
     "moba_profile_end": (_i32, [_vp, _vp, _vp]),
     "moba_last_error": (ctypes.c_char_p, []),

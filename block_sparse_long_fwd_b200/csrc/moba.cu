@@ -564,3 +564,116 @@ extern "C" int moba_selftest_bounded_wait(int timeout_us, cudaStream_t stream) {
   MOBA_CUDA(cudaGetLastError());
   return moba_device_status(stream);
 }
+
+// ------------------------------------------------------------ no allocation
+// moba_fwd_noalloc: the forward pass for callers that may not allocate
+// device memory once they are running -- for example a serving process that
+// reserves its whole memory budget at start-up, or a plug-in that lives under
+// an allocator it does not own. Its scratch is this fixed array, which every
+// GPU that loads the library holds until the process exits.
+
+namespace {
+
+constexpr size_t kNoAllocScratchBytes = (size_t)64 << 20;  // 64 MiB
+
+static __device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocScratchBytes];
+
+std::mutex g_noalloc_mu;
+void* g_noalloc_ptr[64] = {};
+
+// Device address of g_noalloc_scratch on the current device, looked up once
+// per device (in host code the array's name is only a host-side stand-in).
+int noalloc_scratch(void** out) {
+  int dev = 0;
+  MOBA_CUDA(cudaGetDevice(&dev));
+  if (dev < 0 || dev >= 64) return fail(MOBA_ERR_UNSUPPORTED, "device index %d out of range", dev);
+  std::lock_guard<std::mutex> lk(g_noalloc_mu);
+  if (!g_noalloc_ptr[dev]) {
+    void* ptr = nullptr;
+    cudaError_t e = cudaGetSymbolAddress(&ptr, g_noalloc_scratch);
+    if (e != cudaSuccess || !ptr)
+      return fail(MOBA_ERR_CUDA, "cudaGetSymbolAddress of the no-allocation scratch failed: %s",
+                  cudaGetErrorString(e));
+    g_noalloc_ptr[dev] = ptr;
+  }
+  *out = g_noalloc_ptr[dev];
+  return MOBA_OK;
+}
+
+// Scratch layout for a window of W tokens (same buffers, in the same order,
+// as the stream-ordered path).
+void layout_for_window(Plan& p, int64_t W) {
+  p.W = W;
+  p.wwords = (W * p.G + 31) / 32;
+  const int64_t nbk = (int64_t)p.Hkv * p.nbp;
+  p.list_cap = W * p.Hq * p.P;
+  p.tile_cap = p.list_cap / moba::kUnitRowsRouted + nbk + (W / moba::kTile + 1) * p.Hkv * ((p.G + 1) / 2);
+  Carve c;
+  p.o_kmean = c.take((size_t)nbk * moba::kHeadDim * 4);
+  p.o_sel = c.take((size_t)p.Hq * p.S * p.k_eff * 4);
+  p.o_flags = c.take((size_t)nbk * p.wwords * 4);
+  p.o_wordbase = c.take((size_t)nbk * p.wwords * 4);
+  p.o_cnt = c.take((size_t)(nbk + 1) * 4);
+  p.o_loff = c.take((size_t)(nbk + 1) * 4);
+  p.o_toff = c.take((size_t)(nbk + 1) * 4);
+  p.o_list = c.take((size_t)std::max<int64_t>(p.list_cap, 1) * 4);
+  p.o_tiles = c.take((size_t)p.tile_cap * 16);
+  p.o_hdr = c.take(16);
+  p.o_part_o = c.take((size_t)std::max<int64_t>(p.list_cap, 1) * moba::kHeadDim * 4);
+  p.o_part_lse = c.take((size_t)std::max<int64_t>(p.list_cap, 1) * 4);
+  p.o_own_o = c.take((size_t)W * p.Hq * moba::kHeadDim * 4);
+  p.o_own_lse = c.take((size_t)W * p.Hq * 4);
+  p.total = c.off;
+}
+
+// The largest query window (a multiple of 128 tokens) whose scratch fits in
+// `cap` bytes; fails when not even a 128-token window fits.
+int plan_within(Plan* pl, int64_t S, int Hq, int Hkv, int B, int topk, size_t cap) {
+  Plan& p = *pl;
+  p.S = S;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.G = Hq / Hkv;
+  p.B = B;
+  p.topk = topk;
+  p.nb = (int)((S + B - 1) / B);
+  p.nbp = p.nb - 1;
+  p.k_eff = std::min(topk, p.nb);
+  p.P = p.k_eff - 1;
+  int64_t W = (S + 127) / 128 * 128;
+  while (true) {
+    if (W * Hq * (int64_t)p.P < ((int64_t)1 << 31) - 1) {
+      layout_for_window(p, W);
+      if (p.total <= cap) return MOBA_OK;
+    }
+    if (W == 128) break;
+    W = std::max<int64_t>(128, W / 2 / 128 * 128);
+  }
+  return fail(MOBA_ERR_UNSUPPORTED,
+              "problem too large for moba_fwd_noalloc: its scratch needs more than the fixed %zu bytes "
+              "(seqlen %lld, heads_q %d, heads_kv %d, block_size %d, topk %d); use moba_fwd",
+              cap, (long long)S, Hq, Hkv, B, topk);
+}
+
+}  // namespace
+
+extern "C" int moba_fwd_noalloc(const void* q, const void* k, const void* v, int64_t seqlen, int heads_q,
+                                int heads_kv, int head_dim, int block_size, int topk, void* out, float* lse,
+                                cudaStream_t stream) {
+  g_err.clear();
+  if (!q || !k || !v || !out || !lse) return fail(MOBA_ERR_INVALID_ARG, "null pointer argument");
+  int rc = check_shape(seqlen, heads_q, heads_kv, head_dim, block_size, topk);
+  if (rc) return rc;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(lse))
+    return fail(MOBA_ERR_INVALID_ARG, "device buffers must be 16-byte aligned");
+  Plan p;
+  rc = plan_within(&p, seqlen, heads_q, heads_kv, block_size, topk, kNoAllocScratchBytes);
+  if (rc) return rc;
+  DeviceInfo dev;
+  rc = device_info(&dev);
+  if (rc) return rc;
+  void* scratch = nullptr;
+  rc = noalloc_scratch(&scratch);
+  if (rc) return rc;
+  return run_forward(p, dev, q, k, v, out, lse, static_cast<uint8_t*>(scratch), stream);
+}

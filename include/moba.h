@@ -133,6 +133,31 @@ int moba_gate(const void* q, const float* kmean, int64_t seqlen, int heads_q,
 int moba_profile_begin(void);
 int moba_profile_end(float* stage_ms, int* launches, int* calls);
 
+/*
+ * moba_fwd_noalloc - moba_fwd for callers that may not allocate device
+ * memory while they run (a serving process that reserves its memory budget
+ * at start-up, a plug-in under an allocator it does not own). The pages have
+ * no counterpart: this is a property of this library, not of the method.
+ *
+ * Same arguments, layouts and results as moba_fwd. Instead of the
+ * stream-ordered allocator it uses one fixed 64 MiB device array that the
+ * library defines; every GPU that loads the library holds that array until
+ * the process exits. The call allocates nothing: no cudaMalloc, cudaFree or
+ * allocating library routine. Problems whose scratch would not fit in the
+ * array (the selection table and at least a 128-token query window) are
+ * rejected with MOBA_ERR_UNSUPPORTED before any launch; moba_fwd handles
+ * them. The first call on a device looks up the array's device address
+ * (cudaGetSymbolAddress) with that device current; make that first call
+ * before any stream capture. Every call shares the one array: calls that
+ * overlap on the GPU (different streams, or threads) race on it and must be
+ * serialised by the caller. Nothing in the array needs to start at zero;
+ * every call writes each part before reading it.
+ */
+int moba_fwd_noalloc(const void* q, const void* k, const void* v,
+                     int64_t seqlen, int heads_q, int heads_kv, int head_dim,
+                     int block_size, int topk, void* out, float* lse,
+                     cudaStream_t stream);
+
 /* Message of the last failed call on this host thread ("" if none). */
 const char* moba_last_error(void);
 
