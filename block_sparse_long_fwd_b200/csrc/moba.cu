@@ -16,8 +16,9 @@
 
 #include "attn.cuh"
 #include "common.cuh"
+#include "gate_tc.cuh"
 #include "merge.cuh"
-#include "pool_gate.cuh"
+#include "pool.cuh"
 #include "route.cuh"
 
 namespace {
@@ -65,6 +66,20 @@ int device_info(DeviceInfo* out) {
     if (d.sm100) {
       MOBA_CUDA(cudaFuncSetAttribute(moba::attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      moba::kAttnSmemBytes));
+      MOBA_CUDA(cudaFuncSetAttribute(moba::gate_tc_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     moba::kGateSmemBytes));
+      MOBA_CUDA(cudaFuncSetAttribute(moba::gate_tc_kernel<4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     moba::kGateSmemBytes));
+      MOBA_CUDA(cudaFuncSetAttribute(moba::gate_tc_kernel<8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     moba::kGateSmemBytes));
+      MOBA_CUDA(cudaFuncSetAttribute(moba::gate_tc_kernel<12>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     moba::kGateSmemBytes));
+      MOBA_CUDA(cudaFuncSetAttribute(moba::gate_tc_kernel<16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     moba::kGateSmemBytes));
+      MOBA_CUDA(cudaFuncSetAttribute(moba::gate_tc_kernel<32>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     moba::kGateSmemBytes));
+      MOBA_CUDA(cudaFuncSetAttribute(moba::gate_tc_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     moba::kGateSmemBytes));
       // keep freed scratch in the stream-ordered pool between calls
       cudaMemPool_t pool;
       MOBA_CUDA(cudaDeviceGetDefaultMemPool(&pool, dev));
@@ -134,8 +149,8 @@ struct Plan {
   int64_t W;       // window tokens (multiple of 128)
   int64_t wwords;  // flag words per bucket for a full window
   int64_t list_cap, tile_cap;
-  size_t o_kmean, o_sel, o_flags, o_wordbase, o_cnt, o_loff, o_toff, o_list, o_tiles, o_hdr, o_part_o, o_part_lse,
-      o_own_o, o_own_lse, total;
+  size_t o_kmean, o_khi, o_klo, o_sel, o_flags, o_wordbase, o_cnt, o_loff, o_toff, o_list, o_tiles, o_hdr, o_part_o,
+      o_part_lse, o_own_o, o_own_lse, total;
 };
 
 size_t window_bytes(const Plan& p, int64_t W) {
@@ -145,6 +160,34 @@ size_t window_bytes(const Plan& p, int64_t W) {
   const int64_t tiles = list / moba::kUnitRowsRouted + nbk + (W / moba::kTile + 1) * p.Hkv * ((p.G + 1) / 2);
   return (size_t)(nbk * wwords * 8 + list * (4 + 4 + 4 * moba::kHeadDim) + tiles * 16 +
                   W * p.Hq * (4 + 4 * moba::kHeadDim));
+}
+
+// Scratch layout for a query window of W tokens.
+void layout_for_window(Plan& p, int64_t W) {
+  p.W = W;
+  p.wwords = (W * p.G + 31) / 32;
+  const int64_t nbk = (int64_t)p.Hkv * p.nbp;
+  p.list_cap = W * p.Hq * p.P;
+  p.tile_cap = p.list_cap / moba::kUnitRowsRouted + nbk + (W / moba::kTile + 1) * p.Hkv * ((p.G + 1) / 2);
+  Carve c;
+  p.o_kmean = c.take((size_t)nbk * moba::kHeadDim * 4);
+  const size_t nbk_pad = (size_t)p.Hkv * moba::gate_rows_padded(std::max(p.nbp, 1));
+  p.o_khi = c.take(nbk_pad * moba::kHeadDim * 2);
+  p.o_klo = c.take(nbk_pad * moba::kHeadDim * 2);
+  p.o_sel = c.take((size_t)p.Hq * p.S * p.k_eff * 4);
+  p.o_flags = c.take((size_t)nbk * p.wwords * 4);
+  p.o_wordbase = c.take((size_t)nbk * p.wwords * 4);
+  p.o_cnt = c.take((size_t)(nbk + 1) * 4);
+  p.o_loff = c.take((size_t)(nbk + 1) * 4);
+  p.o_toff = c.take((size_t)(nbk + 1) * 4);
+  p.o_list = c.take((size_t)std::max<int64_t>(p.list_cap, 1) * 4);
+  p.o_tiles = c.take((size_t)p.tile_cap * 16);
+  p.o_hdr = c.take(16);
+  p.o_part_o = c.take((size_t)std::max<int64_t>(p.list_cap, 1) * moba::kHeadDim * 4);
+  p.o_part_lse = c.take((size_t)std::max<int64_t>(p.list_cap, 1) * 4);
+  p.o_own_o = c.take((size_t)W * p.Hq * moba::kHeadDim * 4);
+  p.o_own_lse = c.take((size_t)W * p.Hq * 4);
+  p.total = c.off;
 }
 
 int make_plan(Plan* pl, int64_t S, int Hq, int Hkv, int B, int topk) {
@@ -176,47 +219,66 @@ int make_plan(Plan* pl, int64_t S, int Hq, int Hkv, int B, int topk) {
   // list slots and positions are 32-bit
   while (W > 128 && W * Hq * (int64_t)p.P >= ((int64_t)1 << 31) - 1) W = std::max<int64_t>(128, W / 2 / 128 * 128);
   if (W * Hq * (int64_t)p.P >= ((int64_t)1 << 31) - 1) return fail(MOBA_ERR_UNSUPPORTED, "window too large");
-  p.W = W;
-  p.wwords = (W * p.G + 31) / 32;
-  const int64_t nbk = (int64_t)Hkv * p.nbp;
-  p.list_cap = W * Hq * p.P;
-  p.tile_cap = p.list_cap / moba::kUnitRowsRouted + nbk + (W / moba::kTile + 1) * Hkv * ((p.G + 1) / 2);
-  Carve c;
-  p.o_kmean = c.take((size_t)nbk * moba::kHeadDim * 4);
-  p.o_sel = c.take((size_t)Hq * S * p.k_eff * 4);
-  p.o_flags = c.take((size_t)nbk * p.wwords * 4);
-  p.o_wordbase = c.take((size_t)nbk * p.wwords * 4);
-  p.o_cnt = c.take((size_t)(nbk + 1) * 4);
-  p.o_loff = c.take((size_t)(nbk + 1) * 4);
-  p.o_toff = c.take((size_t)(nbk + 1) * 4);
-  p.o_list = c.take((size_t)std::max<int64_t>(p.list_cap, 1) * 4);
-  p.o_tiles = c.take((size_t)p.tile_cap * 16);
-  p.o_hdr = c.take(16);
-  p.o_part_o = c.take((size_t)std::max<int64_t>(p.list_cap, 1) * moba::kHeadDim * 4);
-  p.o_part_lse = c.take((size_t)std::max<int64_t>(p.list_cap, 1) * 4);
-  p.o_own_o = c.take((size_t)W * Hq * moba::kHeadDim * 4);
-  p.o_own_lse = c.take((size_t)W * Hq * 4);
-  p.total = c.off;
+  layout_for_window(p, W);
+  return MOBA_OK;
+}
+
+// Block-mean rows as a 2-D tensor [Hkv * nbp_pad][128] bf16; box 64 x 64,
+// 128-byte swizzle (one 64-channel half of a 64-block chunk per load).
+int make_mean_map(CUtensorMap* map, const void* base, int64_t rows) {
+  cuuint64_t dims[2] = {(cuuint64_t)moba::kHeadDim, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)moba::kHeadDim * 2};
+  cuuint32_t box[2] = {64, (cuuint32_t)moba::kGateBlkChunk};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(MOBA_ERR_CUDA, "cuTensorMapEncodeTiled (block means) failed (%d)", (int)r);
   return MOBA_OK;
 }
 
 template <int KP>
-void launch_gate_kp(const Plan& p, const void* q, const float* kmean, int32_t* sel, cudaStream_t st) {
-  dim3 grid((unsigned)((p.S * p.G + moba::kGateThreads - 1) / moba::kGateThreads), p.Hkv);
-  moba::gate_kernel<KP><<<grid, moba::kGateThreads, 0, st>>>(static_cast<const __nv_bfloat16*>(q), kmean, p.S, p.Hq,
-                                                             p.G, p.B, p.nbp, p.k_eff, sel);
+void launch_gate_tc(const Plan& p, const CUtensorMap& mhi, const CUtensorMap& mlo, const moba::GateParams& gp,
+                    cudaStream_t st) {
+  dim3 grid((unsigned)((p.S * p.G + 127) / 128), p.Hkv);
+  moba::gate_tc_kernel<KP><<<grid, moba::kGateTcThreads, moba::kGateSmemBytes, st>>>(mhi, mlo, gp);
 }
 
-void launch_gate(const Plan& p, const void* q, const float* kmean, int32_t* sel, cudaStream_t st) {
+// Gate + top-k into sel. kmean (fp32) is split into khi/klo (bf16, padded
+// rows) first. Rows that need no scores (topk 1, or every past block) are
+// written directly. Returns the number of kernels launched, or -status.
+int launch_gate(const Plan& p, const void* q, const float* kmean, __nv_bfloat16* khi, __nv_bfloat16* klo,
+                int32_t* sel, cudaStream_t st) {
   const bool full = p.k_eff == p.nb;
-  const int need = full ? 1 : std::max(1, p.P);
-  if (need <= 1) launch_gate_kp<1>(p, q, kmean, sel, st);
-  else if (need <= 2) launch_gate_kp<2>(p, q, kmean, sel, st);
-  else if (need <= 4) launch_gate_kp<4>(p, q, kmean, sel, st);
-  else if (need <= 8) launch_gate_kp<8>(p, q, kmean, sel, st);
-  else if (need <= 16) launch_gate_kp<16>(p, q, kmean, sel, st);
-  else if (need <= 32) launch_gate_kp<32>(p, q, kmean, sel, st);
-  else launch_gate_kp<64>(p, q, kmean, sel, st);
+  if (p.P == 0 || full || p.nbp <= 0) {
+    const int64_t n = p.S * p.Hq;
+    moba::sel_fill_kernel<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(sel, p.S, p.Hq, p.B, p.k_eff, full ? 1 : 0);
+    return 1;
+  }
+  const int nbp_pad = moba::gate_rows_padded(p.nbp);
+  moba::kmean_split_kernel<<<dim3(nbp_pad, p.Hkv), 128, 0, st>>>(kmean, p.nbp, nbp_pad, khi, klo);
+  CUtensorMap mhi, mlo;
+  int rc = make_mean_map(&mhi, khi, (int64_t)p.Hkv * nbp_pad);
+  if (rc) return -rc;
+  rc = make_mean_map(&mlo, klo, (int64_t)p.Hkv * nbp_pad);
+  if (rc) return -rc;
+  moba::GateParams gp;
+  gp.q = static_cast<const __nv_bfloat16*>(q);
+  gp.sel = sel;
+  gp.S = p.S;
+  gp.Hq = p.Hq;
+  gp.G = p.G;
+  gp.B = p.B;
+  gp.nbp_pad = nbp_pad;
+  gp.k_eff = p.k_eff;
+  if (p.P <= 2) launch_gate_tc<2>(p, mhi, mlo, gp, st);
+  else if (p.P <= 4) launch_gate_tc<4>(p, mhi, mlo, gp, st);
+  else if (p.P <= 8) launch_gate_tc<8>(p, mhi, mlo, gp, st);
+  else if (p.P <= 12) launch_gate_tc<12>(p, mhi, mlo, gp, st);
+  else if (p.P <= 16) launch_gate_tc<16>(p, mhi, mlo, gp, st);
+  else if (p.P <= 32) launch_gate_tc<32>(p, mhi, mlo, gp, st);
+  else launch_gate_tc<64>(p, mhi, mlo, gp, st);
+  return 2;
 }
 
 void launch_pool(const Plan& p, const void* k, float* kmean, cudaStream_t st) {
@@ -302,8 +364,12 @@ int run_forward(const Plan& p, const DeviceInfo& dev, const void* q, const void*
     tm->count(1);
     tm->mark(kPool);
   }
-  launch_gate(p, q, kmean, sel, st);
-  tm->count(1);
+  {
+    const int n = launch_gate(p, q, kmean, reinterpret_cast<__nv_bfloat16*>(ws + p.o_khi),
+                              reinterpret_cast<__nv_bfloat16*>(ws + p.o_klo), sel, st);
+    if (n < 0) return -n;
+    tm->count(n);
+  }
   tm->mark(kGate);
 
   const int nbk = p.Hkv * p.nbp;
@@ -517,8 +583,20 @@ int moba_gate(const void* q, const float* kmean, int64_t seqlen, int heads_q, in
   p.nbp = nb - 1;
   p.k_eff = std::min(topk, nb);
   p.P = p.k_eff - 1;
-  launch_gate(p, q, kmean, sel, stream);
+  // bf16 hi/lo parts of the means: stream-ordered scratch for this call
+  const size_t part = (size_t)heads_kv * moba::gate_rows_padded(std::max(p.nbp, 1)) * moba::kHeadDim * 2;
+  void* parts = nullptr;
+  cudaError_t e = cudaMallocAsync(&parts, 2 * part, stream);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return fail(MOBA_ERR_OOM, "scratch allocation of %zu bytes failed: %s", 2 * part, cudaGetErrorString(e));
+  }
+  __nv_bfloat16* khi = static_cast<__nv_bfloat16*>(parts);
+  const int n = launch_gate(p, q, kmean, khi, khi + part / 2, sel, stream);
+  cudaError_t ef = cudaFreeAsync(parts, stream);
+  if (n < 0) return -n;
   MOBA_CUDA(cudaGetLastError());
+  if (ef != cudaSuccess) return fail(MOBA_ERR_CUDA, "cudaFreeAsync failed: %s", cudaGetErrorString(ef));
   return MOBA_OK;
 }
 
@@ -598,32 +676,6 @@ int noalloc_scratch(void** out) {
   }
   *out = g_noalloc_ptr[dev];
   return MOBA_OK;
-}
-
-// Scratch layout for a window of W tokens (same buffers, in the same order,
-// as the stream-ordered path).
-void layout_for_window(Plan& p, int64_t W) {
-  p.W = W;
-  p.wwords = (W * p.G + 31) / 32;
-  const int64_t nbk = (int64_t)p.Hkv * p.nbp;
-  p.list_cap = W * p.Hq * p.P;
-  p.tile_cap = p.list_cap / moba::kUnitRowsRouted + nbk + (W / moba::kTile + 1) * p.Hkv * ((p.G + 1) / 2);
-  Carve c;
-  p.o_kmean = c.take((size_t)nbk * moba::kHeadDim * 4);
-  p.o_sel = c.take((size_t)p.Hq * p.S * p.k_eff * 4);
-  p.o_flags = c.take((size_t)nbk * p.wwords * 4);
-  p.o_wordbase = c.take((size_t)nbk * p.wwords * 4);
-  p.o_cnt = c.take((size_t)(nbk + 1) * 4);
-  p.o_loff = c.take((size_t)(nbk + 1) * 4);
-  p.o_toff = c.take((size_t)(nbk + 1) * 4);
-  p.o_list = c.take((size_t)std::max<int64_t>(p.list_cap, 1) * 4);
-  p.o_tiles = c.take((size_t)p.tile_cap * 16);
-  p.o_hdr = c.take(16);
-  p.o_part_o = c.take((size_t)std::max<int64_t>(p.list_cap, 1) * moba::kHeadDim * 4);
-  p.o_part_lse = c.take((size_t)std::max<int64_t>(p.list_cap, 1) * 4);
-  p.o_own_o = c.take((size_t)W * p.Hq * moba::kHeadDim * 4);
-  p.o_own_lse = c.take((size_t)W * p.Hq * 4);
-  p.total = c.off;
 }
 
 // The largest query window (a multiple of 128 tokens) whose scratch fits in
