@@ -44,6 +44,26 @@ def load_peaks():
         return dict(FALLBACK_PEAKS), "fallback"
 
 
+def attn_traffic(workload_name: str):
+    """DRAM bytes per attention launch from the committed ncu record, or None
+    when the record is for another workload or an older attention kernel."""
+    import hashlib
+    rec = os.path.join(ROOT, "profiles", "attn_kernel_traffic.txt")
+    src = os.path.join(ROOT, "block_sparse_long_fwd_b200", "csrc", "attn.cuh")
+    try:
+        kv = {}
+        for line in open(rec):
+            if "=" in line and not line.lstrip().startswith("#"):
+                k, v = line.split("=", 1)
+                kv[k.strip()] = v.strip()
+        sha = hashlib.sha256(open(src, "rb").read()).hexdigest()
+        if kv.get("kernel_source_sha256") == sha and kv.get("workload") == workload_name:
+            return int(kv["bytes_per_launch"])
+    except (OSError, ValueError, KeyError):
+        pass
+    return None
+
+
 def routed_rows(w) -> int:
     """Past-block partials per step: sum over rows of min(k-1, t//B)."""
     nb = w.nblocks
@@ -305,7 +325,7 @@ def run_ours(args, w):
             "eff_tflops": world * flops * args.steps / (total_ms / 1e3) / 1e12,
             "stage_ms_per_step": {kk: vv / max(calls, 1) for kk, vv in stages.items()},
             "roofline": {"bound": "tensor", "kernel": "attn_kernel", "achieved": achieved, "peak": peak,
-                         "unit": "TFLOP/s", "frac": achieved / peak, "traffic": None,
+                         "unit": "TFLOP/s", "frac": achieved / peak, "traffic": attn_traffic(wr.name),
                          "peak_source": f"{peaks_src} bf16 {'sustained' if long_step else 'burst'}",
                          "algorithmic": f"{flops:.4e} selected-block FLOPs per step / attention ms per step"},
             "stage_roofline_hbm": stage_roof,
