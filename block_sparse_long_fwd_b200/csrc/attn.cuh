@@ -54,7 +54,7 @@ struct AttnParams {
   const __nv_bfloat16* q;   // [S][Hq][128]
   const int32_t* list;      // group-rows of the window, per bucket
   const int4* units;        // unit descriptors
-  const int32_t* hdr;       // [1] = number of units
+  int32_t* hdr;             // [1] = number of units, [3] = next-unit counter (starts at 0)
   float* part_o;            // [list entries][128]
   float* part_lse;          // [list entries]
   float* own_o;             // [wlen][Hq][128]
@@ -64,7 +64,12 @@ struct AttnParams {
   float scale_log2;         // log2(e) / sqrt(128)
 };
 
+constexpr int kRing = 8;                               // unit indices in flight per CTA
+constexpr uint32_t kRingReaders = 1 + 32 + 256 + 64;   // producer lane, MMA warp, softmax, gather
+
 struct AttnShared {
+  uint64_t ring_full[kRing], ring_empty[kRing];
+  int ring[kRing];
   uint64_t q_full[2], q_empty[2];
   uint64_t k_full[kStages], k_empty[kStages], v_full[kStages], v_empty[kStages];
   uint64_t s_full[2], p_full[2], pv_done[2], o_free[2];
@@ -174,7 +179,6 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   AttnShared* sh = reinterpret_cast<AttnShared*>(sV + kStages * kTileBytes);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int n_units = p.hdr[1];
 
   if (threadIdx.x == 0) {
     for (int x = 0; x < 2; ++x) {
@@ -190,6 +194,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       mbar_init(&sh->k_empty[i], 1);
       mbar_init(&sh->v_full[i], 1);
       mbar_init(&sh->v_empty[i], 1);
+    }
+    for (int i = 0; i < kRing; ++i) {
+      mbar_init(&sh->ring_full[i], 1);
+      mbar_init(&sh->ring_empty[i], kRingReaders);
     }
     mbar_init(&sh->drain, 1);
     sh->abort_flag = 0;
@@ -208,6 +216,17 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   tc_fence_after();
   const uint32_t tmem = sh->tmem_base;
   volatile int* abort_flag = &sh->abort_flag;
+  // Work units are handed out dynamically: a gather thread takes the next
+  // index from the global counter and publishes it in the CTA's ring; every
+  // role reads the same sequence from the ring (-1 ends it). Returns false
+  // on a timeout.
+  auto next_unit = [&](uint32_t n, int& ui) -> bool {
+    const int slot = n % kRing;
+    if (!mbar_wait(&sh->ring_full[slot], (n / kRing) & 1, abort_flag)) return false;
+    ui = *reinterpret_cast<volatile int*>(&sh->ring[slot]);
+    mbar_arrive(&sh->ring_empty[slot]);
+    return true;
+  };
 
   // register split: the two softmax warpgroups take 200 per thread, the
   // producer/MMA/gather warpgroup 104 (256*200 + 128*104 = 64512, exactly
@@ -226,7 +245,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     const uint32_t tS = tmem + X * 128 + lane_off;
     const uint32_t tO = tmem + 256 + X * 128 + lane_off;
     uint32_t sx = 0;  // steps done by tile X
-    for (int ui = blockIdx.x; ui < n_units; ui += gridDim.x) {
+    for (uint32_t un = 0;; ++un) {
+      int ui;
+      if (!next_unit(un, ui)) goto done;
+      if (ui < 0) break;
       const UnitInfo u = decode_unit(p, ui);
       if (X == 1 && !u.has_b) continue;
       float m_run = -INFINITY, l_run = 0.f;
@@ -346,7 +368,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     // ------------------------------------------------ K/V TMA producer
     if (lane == 0) {
       uint32_t it = 0;
-      for (int ui = blockIdx.x; ui < n_units; ui += gridDim.x) {
+      for (uint32_t un = 0;; ++un) {
+        int ui;
+        if (!next_unit(un, ui)) goto drain_kv;
+        if (ui < 0) break;
         const UnitInfo u = decode_unit(p, ui);
         for (int s = 0; s < u.nsteps; ++s, ++it) {
           const int st = it % kStages;
@@ -412,7 +437,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       if (elect_one()) mma_commit(bar);
       __syncwarp();
     };
-    for (int ui = blockIdx.x; ui < n_units; ui += gridDim.x) {
+    for (uint32_t un = 0;; ++un) {
+      int ui;
+      if (!next_unit(un, ui)) goto mma_done;
+      if (ui < 0) break;
       const UnitInfo u = decode_unit(p, ui);
       const int nx = u.has_b ? 2 : 1;
 #pragma unroll
@@ -488,7 +516,19 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     // ------------------------------------------------ Q gather (warps 10, 11)
     const int gt = threadIdx.x - 320;  // 0..63
     uint32_t ux[2] = {0, 0};
-    for (int ui = blockIdx.x; ui < n_units; ui += gridDim.x) {
+    const int n_units = p.hdr[1];
+    for (uint32_t un = 0;; ++un) {
+      if (gt == 0) {
+        // publish the next unit index (slot reuse waits for every reader)
+        const int slot = un % kRing;
+        if (!mbar_wait(&sh->ring_empty[slot], ((un / kRing) & 1) ^ 1, abort_flag)) goto gather_done;
+        int nxt = atomicAdd(p.hdr + 3, 1);
+        sh->ring[slot] = nxt < n_units ? nxt : -1;
+        mbar_arrive(&sh->ring_full[slot]);
+      }
+      int ui;
+      if (!next_unit(un, ui)) goto gather_done;
+      if (ui < 0) break;
       const UnitInfo u = decode_unit(p, ui);
       const int nx = u.has_b ? 2 : 1;
 #pragma unroll

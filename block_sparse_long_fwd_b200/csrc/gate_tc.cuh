@@ -35,15 +35,19 @@ __host__ __device__ inline int gate_rows_padded(int nbp) {
   return (nbp + kGateBlkChunk - 1) / kGateBlkChunk * kGateBlkChunk;
 }
 
-// kmean fp32 [Hkv][nbp][128] -> hi, lo bf16 [Hkv][nbp_pad][128]; padding rows
-// are zero. grid (nbp_pad, Hkv), 128 threads.
-__global__ void __launch_bounds__(128) kmean_split_kernel(const float* __restrict__ kmean, int nbp, int nbp_pad,
-                                                          __nv_bfloat16* __restrict__ hi,
+// Block means -> hi, lo bf16 [Hkv][nbp_pad][128]; padding rows are zero.
+// part holds `splits` partial means per block, [Hkv][nbp][splits][128],
+// added in order (one split: part is the mean itself). grid (nbp_pad, Hkv),
+// 128 threads.
+__global__ void __launch_bounds__(128) kmean_split_kernel(const float* __restrict__ part, int splits, int nbp,
+                                                          int nbp_pad, __nv_bfloat16* __restrict__ hi,
                                                           __nv_bfloat16* __restrict__ lo) {
   const int j = blockIdx.x, g = blockIdx.y, c = threadIdx.x;
   const int64_t o = ((int64_t)g * nbp_pad + j) * kHeadDim + c;
   if (j < nbp) {
-    const float m = kmean[((int64_t)g * nbp + j) * kHeadDim + c];
+    const float* src = part + ((int64_t)g * nbp + j) * splits * kHeadDim + c;
+    float m = 0.f;
+    for (int sp = 0; sp < splits; ++sp) m += src[(int64_t)sp * kHeadDim];
     const __nv_bfloat16 h = __float2bfloat16_rn(m);
     hi[o] = h;
     lo[o] = __float2bfloat16_rn(m - __bfloat162float(h));

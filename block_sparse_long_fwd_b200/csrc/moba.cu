@@ -146,6 +146,7 @@ struct Carve {
 struct Plan {
   int64_t S;
   int Hq, Hkv, G, B, topk, k_eff, P, nb, nbp;
+  int splits = 1;  // pool row splits per block
   int64_t W;       // window tokens (multiple of 128)
   int64_t wwords;  // flag words per bucket for a full window
   int64_t list_cap, tile_cap;
@@ -170,7 +171,8 @@ void layout_for_window(Plan& p, int64_t W) {
   p.list_cap = W * p.Hq * p.P;
   p.tile_cap = p.list_cap / moba::kUnitRowsRouted + nbk + (W / moba::kTile + 1) * p.Hkv * ((p.G + 1) / 2);
   Carve c;
-  p.o_kmean = c.take((size_t)nbk * moba::kHeadDim * 4);
+  p.splits = moba::pool_splits(std::max(p.nbp, 1), p.Hkv, p.B, 296);
+  p.o_kmean = c.take((size_t)nbk * p.splits * moba::kHeadDim * 4);
   const size_t nbk_pad = (size_t)p.Hkv * moba::gate_rows_padded(std::max(p.nbp, 1));
   p.o_khi = c.take(nbk_pad * moba::kHeadDim * 2);
   p.o_klo = c.take(nbk_pad * moba::kHeadDim * 2);
@@ -247,8 +249,8 @@ void launch_gate_tc(const Plan& p, const CUtensorMap& mhi, const CUtensorMap& ml
 // Gate + top-k into sel. kmean (fp32) is split into khi/klo (bf16, padded
 // rows) first. Rows that need no scores (topk 1, or every past block) are
 // written directly. Returns the number of kernels launched, or -status.
-int launch_gate(const Plan& p, const void* q, const float* kmean, __nv_bfloat16* khi, __nv_bfloat16* klo,
-                int32_t* sel, cudaStream_t st) {
+int launch_gate(const Plan& p, const void* q, const float* kmean, int splits, __nv_bfloat16* khi,
+                __nv_bfloat16* klo, int32_t* sel, cudaStream_t st) {
   const bool full = p.k_eff == p.nb;
   if (p.P == 0 || full || p.nbp <= 0) {
     const int64_t n = p.S * p.Hq;
@@ -256,7 +258,7 @@ int launch_gate(const Plan& p, const void* q, const float* kmean, __nv_bfloat16*
     return 1;
   }
   const int nbp_pad = moba::gate_rows_padded(p.nbp);
-  moba::kmean_split_kernel<<<dim3(nbp_pad, p.Hkv), 128, 0, st>>>(kmean, p.nbp, nbp_pad, khi, klo);
+  moba::kmean_split_kernel<<<dim3(nbp_pad, p.Hkv), 128, 0, st>>>(kmean, splits, p.nbp, nbp_pad, khi, klo);
   CUtensorMap mhi, mlo;
   int rc = make_mean_map(&mhi, khi, (int64_t)p.Hkv * nbp_pad);
   if (rc) return -rc;
@@ -281,11 +283,11 @@ int launch_gate(const Plan& p, const void* q, const float* kmean, __nv_bfloat16*
   return 2;
 }
 
-void launch_pool(const Plan& p, const void* k, float* kmean, cudaStream_t st) {
+void launch_pool(const Plan& p, const void* k, float* kmean, int splits, cudaStream_t st) {
   if (p.nbp <= 0) return;
-  dim3 grid(p.nbp, p.Hkv);
+  dim3 grid(p.nbp, p.Hkv, splits);
   moba::pool_kernel<<<grid, moba::kPoolThreads, 0, st>>>(static_cast<const __nv_bfloat16*>(k), p.Hkv, p.B, p.nbp,
-                                                         kmean);
+                                                         splits, kmean);
 }
 
 // Optional per-stage device timing: an event after every stage, tagged with
@@ -360,12 +362,12 @@ int run_forward(const Plan& p, const DeviceInfo& dev, const void* q, const void*
 
   tm->mark(-1);
   if (p.P > 0 && p.k_eff < p.nb && p.nbp > 0) {
-    launch_pool(p, k, kmean, st);
+    launch_pool(p, k, kmean, p.splits, st);
     tm->count(1);
     tm->mark(kPool);
   }
   {
-    const int n = launch_gate(p, q, kmean, reinterpret_cast<__nv_bfloat16*>(ws + p.o_khi),
+    const int n = launch_gate(p, q, kmean, p.splits, reinterpret_cast<__nv_bfloat16*>(ws + p.o_khi),
                               reinterpret_cast<__nv_bfloat16*>(ws + p.o_klo), sel, st);
     if (n < 0) return -n;
     tm->count(n);
@@ -555,7 +557,7 @@ int moba_pool(const void* k, int64_t seqlen, int heads_kv, int head_dim, int blo
   p.B = block_size;
   p.nb = (int)((seqlen + block_size - 1) / block_size);
   p.nbp = p.nb - 1;
-  launch_pool(p, k, kmean, stream);
+  launch_pool(p, k, kmean, 1, stream);
   MOBA_CUDA(cudaGetLastError());
   return MOBA_OK;
 }
@@ -592,7 +594,7 @@ int moba_gate(const void* q, const float* kmean, int64_t seqlen, int heads_q, in
     return fail(MOBA_ERR_OOM, "scratch allocation of %zu bytes failed: %s", 2 * part, cudaGetErrorString(e));
   }
   __nv_bfloat16* khi = static_cast<__nv_bfloat16*>(parts);
-  const int n = launch_gate(p, q, kmean, khi, khi + part / 2, sel, stream);
+  const int n = launch_gate(p, q, kmean, 1, khi, khi + part / 2, sel, stream);
   cudaError_t ef = cudaFreeAsync(parts, stream);
   if (n < 0) return -n;
   MOBA_CUDA(cudaGetLastError());

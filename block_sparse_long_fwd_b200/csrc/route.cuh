@@ -128,7 +128,8 @@ __device__ __forceinline__ int64_t block_incl_scan_1024(int64_t v, int64_t* scra
 //   own    {t0, nrows (1..128), hA | hB << 16, -nsteps}: 128 tokens of two
 //          q heads of one group (hB = 0xFFFF when the group has an odd
 //          head left over).
-// hdr[0] = routed units, hdr[1] = all units, hdr[2] = list entries.
+// hdr[0] = routed units, hdr[1] = all units, hdr[2] = list entries,
+// hdr[3] = the attention kernel's next-unit counter (zeroed here).
 constexpr int kUnitRowsRouted = 256;
 // 3. one CTA of 1024 threads.
 __global__ void __launch_bounds__(1024) route_scan_kernel(const int32_t* __restrict__ cnt, int nbuckets,
@@ -200,6 +201,7 @@ __global__ void __launch_bounds__(1024) route_scan_kernel(const int32_t* __restr
     hdr[0] = n_routed;
     hdr[1] = n_routed + (int)(nu * per_u);
     hdr[2] = (int)carry_l;
+    hdr[3] = 0;
   }
 }
 
