@@ -154,6 +154,23 @@ struct Plan {
       o_part_lse, o_own_o, o_own_lse, total;
 };
 
+// Scratch budget for one query window: min(8 GiB, a third of the memory
+// free when the device was first used). Measured once per device, since
+// cudaMemGetInfo costs tens of microseconds per call.
+size_t window_budget() {
+  static std::mutex mu;
+  static size_t budget[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return (size_t)1 << 30;
+  std::lock_guard<std::mutex> lk(mu);
+  if (!budget[dev]) {
+    size_t free_b = 0, total_b = 0;
+    if (cudaMemGetInfo(&free_b, &total_b) != cudaSuccess) free_b = (size_t)16 << 30;
+    budget[dev] = std::max<size_t>((size_t)64 << 20, std::min<size_t>((size_t)8 << 30, free_b / 3));
+  }
+  return budget[dev];
+}
+
 size_t window_bytes(const Plan& p, int64_t W) {
   const int64_t nbk = (int64_t)p.Hkv * p.nbp;
   const int64_t wwords = (W * p.G + 31) / 32;
@@ -210,9 +227,7 @@ int make_plan(Plan* pl, int64_t S, int Hq, int Hkv, int B, int topk) {
     W = atoll(env);
     W = std::max<int64_t>(128, (W + 127) / 128 * 128);
   } else {
-    size_t free_b = 0, total_b = 0;
-    if (cudaMemGetInfo(&free_b, &total_b) != cudaSuccess) free_b = (size_t)16 << 30;
-    const size_t budget = std::min<size_t>((size_t)8 << 30, free_b / 3);
+    const size_t budget = window_budget();
     const size_t per = window_bytes(p, 128);
     W = std::max<int64_t>(1, (int64_t)(budget / std::max<size_t>(per, 1))) * 128;
     if (W > 1024 && W % 1024) W = W / 1024 * 1024;
@@ -448,8 +463,121 @@ extern "C" const char* moba_last_error(void) { return g_err.c_str(); }
 
 namespace {
 
+// The launch sequence with stream-ordered scratch, issued on `stream`.
+int direct_forward(const Plan& p, const DeviceInfo& dev, const void* q, const void* k, const void* v, void* out,
+                   float* lse, cudaStream_t stream) {
+  void* ws = nullptr;
+  cudaError_t e = cudaMallocAsync(&ws, p.total, stream);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return fail(MOBA_ERR_OOM, "scratch allocation of %zu bytes failed: %s", p.total, cudaGetErrorString(e));
+  }
+  int rc = run_forward(p, dev, q, k, v, out, lse, static_cast<uint8_t*>(ws), stream);
+  cudaError_t ef = cudaFreeAsync(ws, stream);
+  if (rc) return rc;
+  if (ef != cudaSuccess) return fail(MOBA_ERR_CUDA, "cudaFreeAsync failed: %s", cudaGetErrorString(ef));
+  return MOBA_OK;
+}
+
+// Repeated calls with the same buffers and shape replay a CUDA graph of the
+// whole launch sequence (scratch allocation and release included as graph
+// memory nodes), so the host enqueues one graph launch instead of about ten
+// kernels. Graphs are captured on an internal stream, launched on the
+// caller's, and kept for the last kGraphCache argument sets; a set is only
+// captured the second time it is seen. MOBA_GRAPH=0 turns this off.
+struct GraphKey {
+  int dev;
+  const void *q, *k, *v;
+  void* out;
+  float* lse;
+  int64_t S, W;
+  int Hq, Hkv, B, topk;
+  bool operator==(const GraphKey& o) const {
+    return dev == o.dev && q == o.q && k == o.k && v == o.v && out == o.out && lse == o.lse && S == o.S && W == o.W &&
+           Hq == o.Hq && Hkv == o.Hkv && B == o.B && topk == o.topk;
+  }
+};
+
+struct GraphEntry {
+  GraphKey key;
+  cudaGraphExec_t exec;  // set once captured
+  int state;             // 0 seen once, 1 captured, 2 capture failed
+};
+
+constexpr size_t kGraphCache = 16;
+std::mutex g_graph_mu;
+std::vector<GraphEntry> g_graphs;
+cudaStream_t g_capture_stream[64] = {};
+
+bool graphs_enabled() {
+  const char* e = getenv("MOBA_GRAPH");
+  return !(e && e[0] == '0');
+}
+
+// MOBA_OK / error after launching a graph; -1 when the caller should launch
+// directly.
+int graph_forward(const Plan& p, const DeviceInfo& dev, const void* q, const void* k, const void* v, void* out,
+                  float* lse, cudaStream_t stream) {
+  if (!graphs_enabled()) return -1;
+  int d = 0;
+  if (cudaGetDevice(&d) != cudaSuccess || d < 0 || d >= 64) return -1;
+  GraphKey key{d, q, k, v, out, lse, p.S, p.W, p.Hq, p.Hkv, p.B, p.topk};
+  std::lock_guard<std::mutex> lk(g_graph_mu);
+  GraphEntry* hit = nullptr;
+  for (GraphEntry& en : g_graphs)
+    if (en.key == key) hit = &en;
+  if (hit && hit->state == 1) {
+    cudaError_t e = cudaGraphLaunch(hit->exec, stream);
+    if (e != cudaSuccess) return fail(MOBA_ERR_CUDA, "cudaGraphLaunch failed: %s", cudaGetErrorString(e));
+    return MOBA_OK;
+  }
+  if (hit && hit->state == 2) return -1;
+  if (!hit) {
+    // first sighting: launch directly; capture only when the same buffers
+    // and shape come back
+    if (g_graphs.size() >= kGraphCache) {
+      if (g_graphs.front().state == 1) cudaGraphExecDestroy(g_graphs.front().exec);
+      g_graphs.erase(g_graphs.begin());
+    }
+    g_graphs.push_back({key, nullptr, 0});
+    return -1;
+  }
+  if (!g_capture_stream[d] && cudaStreamCreateWithFlags(&g_capture_stream[d], cudaStreamNonBlocking) != cudaSuccess) {
+    cudaGetLastError();
+    g_capture_stream[d] = nullptr;
+    return -1;
+  }
+  cudaStream_t cs = g_capture_stream[d];
+  cudaGraph_t graph = nullptr;
+  cudaGraphExec_t exec = nullptr;
+  bool ok = cudaStreamBeginCapture(cs, cudaStreamCaptureModeThreadLocal) == cudaSuccess;
+  if (ok) {
+    void* ws = nullptr;
+    ok = cudaMallocAsync(&ws, p.total, cs) == cudaSuccess;
+    if (ok) {
+      ok = run_forward(p, dev, q, k, v, out, lse, static_cast<uint8_t*>(ws), cs) == MOBA_OK;
+      ok = (cudaFreeAsync(ws, cs) == cudaSuccess) && ok;
+    }
+    ok = (cudaStreamEndCapture(cs, &graph) == cudaSuccess) && ok;
+    ok = ok && graph && cudaGraphInstantiate(&exec, graph, 0) == cudaSuccess;
+  }
+  if (graph) cudaGraphDestroy(graph);
+  if (!ok) {
+    cudaGetLastError();
+    if (exec) cudaGraphExecDestroy(exec);
+    exec = nullptr;
+    g_err.clear();
+  }
+  hit->exec = exec;
+  hit->state = exec ? 1 : 2;
+  if (!exec) return -1;
+  cudaError_t e = cudaGraphLaunch(exec, stream);
+  if (e != cudaSuccess) return fail(MOBA_ERR_CUDA, "cudaGraphLaunch failed: %s", cudaGetErrorString(e));
+  return MOBA_OK;
+}
+
 int fwd_impl(const void* q, const void* k, const void* v, int64_t seqlen, int heads_q, int heads_kv, int head_dim,
-             int block_size, int topk, void* out, float* lse, cudaStream_t stream) {
+             int block_size, int topk, void* out, float* lse, cudaStream_t stream, bool use_graph) {
   g_err.clear();
   if (!q || !k || !v || !out || !lse) return fail(MOBA_ERR_INVALID_ARG, "null pointer argument");
   int rc = check_shape(seqlen, heads_q, heads_kv, head_dim, block_size, topk);
@@ -462,17 +590,11 @@ int fwd_impl(const void* q, const void* k, const void* v, int64_t seqlen, int he
   Plan p;
   rc = make_plan(&p, seqlen, heads_q, heads_kv, block_size, topk);
   if (rc) return rc;
-  void* ws = nullptr;
-  cudaError_t e = cudaMallocAsync(&ws, p.total, stream);
-  if (e != cudaSuccess) {
-    cudaGetLastError();
-    return fail(MOBA_ERR_OOM, "scratch allocation of %zu bytes failed: %s", p.total, cudaGetErrorString(e));
+  if (use_graph && !g_timer.on) {
+    const int g = graph_forward(p, dev, q, k, v, out, lse, stream);
+    if (g >= 0) return g;  // negative: no graph for this call, launch directly
   }
-  rc = run_forward(p, dev, q, k, v, out, lse, static_cast<uint8_t*>(ws), stream);
-  cudaError_t ef = cudaFreeAsync(ws, stream);
-  if (rc) return rc;
-  if (ef != cudaSuccess) return fail(MOBA_ERR_CUDA, "cudaFreeAsync failed: %s", cudaGetErrorString(ef));
-  return MOBA_OK;
+  return direct_forward(p, dev, q, k, v, out, lse, stream);
 }
 
 }  // namespace
@@ -481,7 +603,7 @@ extern "C" {
 
 int moba_fwd(const void* q, const void* k, const void* v, int64_t seqlen, int heads_q, int heads_kv, int head_dim,
              int block_size, int topk, void* out, float* lse, cudaStream_t stream) {
-  return fwd_impl(q, k, v, seqlen, heads_q, heads_kv, head_dim, block_size, topk, out, lse, stream);
+  return fwd_impl(q, k, v, seqlen, heads_q, heads_kv, head_dim, block_size, topk, out, lse, stream, true);
 }
 
 int moba_profile_begin(void) {
@@ -530,8 +652,8 @@ int moba_fwd_host(const void* q_host, const void* k_host, const void* v_host, in
       cudaMemcpyAsync(b + ov, v_host, kb, cudaMemcpyHostToDevice, stream) != cudaSuccess)
     rc = fail(MOBA_ERR_CUDA, "host to device copy failed: %s", cudaGetErrorString(cudaGetLastError()));
   if (!rc)
-    rc = moba_fwd(b + oq, b + ok, b + ov, seqlen, heads_q, heads_kv, head_dim, block_size, topk, b + oo,
-                  reinterpret_cast<float*>(b + ol), stream);
+    rc = fwd_impl(b + oq, b + ok, b + ov, seqlen, heads_q, heads_kv, head_dim, block_size, topk, b + oo,
+                  reinterpret_cast<float*>(b + ol), stream, false);
   if (!rc && (cudaMemcpyAsync(out_host, b + oo, qb, cudaMemcpyDeviceToHost, stream) != cudaSuccess ||
               cudaMemcpyAsync(lse_host, b + ol, lb, cudaMemcpyDeviceToHost, stream) != cudaSuccess))
     rc = fail(MOBA_ERR_CUDA, "device to host copy failed: %s", cudaGetErrorString(cudaGetLastError()));
