@@ -86,8 +86,8 @@ def stage_bytes(w) -> dict:
         "pool": nbp * w.block_size * w.heads_kv * d * 2 + nbp * w.heads_kv * d * 4,
         # read Q once and the means, write the selection table
         "gate": w.seqlen * w.heads_q * d * 2 + nbp * w.heads_kv * d * 4 + w.seqlen * w.heads_q * k_eff * 4,
-        # read the table and every partial (O fp32 + lse), write out bf16 + lse
-        "merge": w.seqlen * w.heads_q * k_eff * 4 + (r + w.seqlen * w.heads_q) * (d * 4 + 4)
+        # read the table and every partial (O fp16 + lse), write out bf16 + lse
+        "merge": w.seqlen * w.heads_q * k_eff * 4 + (r + w.seqlen * w.heads_q) * (d * 2 + 4)
         + w.seqlen * w.heads_q * (d * 2 + 4),
     }
 

@@ -10,7 +10,9 @@
 //     their own block from its start up to the tile, causal mask on the
 //     diagonal step ("MoBA - Moonshot AIが提案した新しいアテンションメカニズム",
 //     "MoBAの技術的原則": a causal mask applies inside the current block).
-// Every tile writes a normalised partial output O_i (fp32) and its
+// Every tile writes a normalised partial output O_i (fp16: a convex
+// combination of bf16 values, so |O_i| <= max |v|, at 2^-11 relative
+// rounding, four times finer than the bf16 output) and its
 // natural-log lse_i; the merge stage combines them. The online softmax
 // (FlashAttention-style; the same page credits MoBA's speed to FlashAttention
 // plus MoE techniques) runs per 128-key step, per tile X in {A, B}:
@@ -55,9 +57,9 @@ struct AttnParams {
   const int32_t* list;      // group-rows of the window, per bucket
   const int4* units;        // unit descriptors
   int32_t* hdr;             // [1] = number of units, [3] = next-unit counter (starts at 0)
-  float* part_o;            // [list entries][128]
+  __half* part_o;           // [list entries][128], fp16
   float* part_lse;          // [list entries]
-  float* own_o;             // [wlen][Hq][128]
+  __half* own_o;            // [wlen][Hq][128], fp16
   float* own_lse;           // [wlen][Hq]
   int64_t S, w0;
   int Hq, G, B;
@@ -335,7 +337,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         const float inv_l = 1.f / l_run;
         const float lse = (m_run + log2f(l_run)) * 0.69314718055994530942f;
         const bool write = row < (X ? u.rows[1] : u.rows[0]);
-        float* dst_o;
+        __half* dst_o;
         float* dst_lse;
         if (u.own) {
           const int64_t rr = (u.t0 + row - p.w0) * p.Hq + (X ? u.h[1] : u.h[0]);
@@ -353,10 +355,14 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           tmem_ld_wait();
           if (write) {
 #pragma unroll
-            for (int e = 0; e < 32; e += 4)
-              *reinterpret_cast<float4*>(dst_o + c * 32 + e) =
-                  make_float4(__uint_as_float(o[e]) * inv_l, __uint_as_float(o[e + 1]) * inv_l,
-                              __uint_as_float(o[e + 2]) * inv_l, __uint_as_float(o[e + 3]) * inv_l);
+            for (int e = 0; e < 32; e += 8) {
+              uint4 hv;
+              hv.x = pack_half2(__uint_as_float(o[e]) * inv_l, __uint_as_float(o[e + 1]) * inv_l);
+              hv.y = pack_half2(__uint_as_float(o[e + 2]) * inv_l, __uint_as_float(o[e + 3]) * inv_l);
+              hv.z = pack_half2(__uint_as_float(o[e + 4]) * inv_l, __uint_as_float(o[e + 5]) * inv_l);
+              hv.w = pack_half2(__uint_as_float(o[e + 6]) * inv_l, __uint_as_float(o[e + 7]) * inv_l);
+              *reinterpret_cast<uint4*>(dst_o + c * 32 + e) = hv;
+            }
           }
         }
         if (write) *dst_lse = lse;

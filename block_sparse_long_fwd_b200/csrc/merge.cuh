@@ -18,14 +18,22 @@ struct MergeParams {
   const int32_t* sel;
   const uint32_t* flags;
   const int32_t* wordbase;
-  const float* part_o;
+  const __half* part_o;  // fp16 partial outputs
   const float* part_lse;
-  const float* own_o;
+  const __half* own_o;
   const float* own_lse;
   __nv_bfloat16* out;  // [S][Hq][128]
   float* lse;          // [Hq][S]
   WindowGeom w;
 };
+
+// Four fp16 values (8 bytes) widened to fp32.
+__device__ __forceinline__ float4 load_half4(const __half* p) {
+  const uint2 r = __ldg(reinterpret_cast<const uint2*>(p));
+  const float2 a = __half22float2(*reinterpret_cast<const __half2*>(&r.x));
+  const float2 b = __half22float2(*reinterpret_cast<const __half2*>(&r.y));
+  return make_float4(a.x, a.y, b.x, b.y);
+}
 
 __device__ __forceinline__ float warp_max(float v) {
   for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
@@ -55,6 +63,7 @@ __global__ void __launch_bounds__(256) merge_kernel(MergeParams m) {
   const int32_t* srow = m.sel + ((int64_t)h * w.S + t) * w.k_eff;
   const int P = w.k_eff - 1;
 
+  // lane i resolves routed partial i (slot and lse) once
   auto slot = [&](int i, float& li) -> int64_t {
     li = -INFINITY;
     if (i >= P) return -1;
@@ -67,42 +76,73 @@ __global__ void __launch_bounds__(256) merge_kernel(MergeParams m) {
   };
 
   const float own_l = m.own_lse[tl * w.Hq + h];
-  float mx = own_l;
-  for (int i0 = 0; i0 < P; i0 += 32) {
-    float li;
-    slot(i0 + lane, li);
-    mx = fmaxf(mx, warp_max(li));
-  }
-  float sum = 0.f;
-  for (int i0 = 0; i0 < P; i0 += 32) {
-    float li;
-    slot(i0 + lane, li);
-    sum += warp_sum(li == -INFINITY ? 0.f : expf(li - mx));
-  }
-  sum += expf(own_l - mx);
-  const float L = mx + logf(sum);
-
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-  for (int i0 = 0; i0 < P; i0 += 32) {
+  float L;
+  if (P <= 32) {
     float li;
-    const int64_t pos = slot(i0 + lane, li);
-    const int n = min(32, P - i0);
-    for (int k = 0; k < n; ++k) {
-      const int64_t pk = __shfl_sync(0xffffffffu, pos, k);
-      const float lk = __shfl_sync(0xffffffffu, li, k);
-      if (pk >= 0) {
-        const float wk = expf(lk - L);
-        const float4 o = __ldg(reinterpret_cast<const float4*>(m.part_o + pk * kHeadDim) + lane);
-        acc.x += wk * o.x;
-        acc.y += wk * o.y;
-        acc.z += wk * o.z;
-        acc.w += wk * o.w;
+    const int64_t pos = slot(lane, li);
+    const float mx = fmaxf(own_l, warp_max(li));
+    const float sum = warp_sum(li == -INFINITY ? 0.f : expf(li - mx)) + expf(own_l - mx);
+    L = mx + logf(sum);
+    const float wl = li == -INFINITY ? 0.f : expf(li - L);  // lane i's weight
+    // partials in ascending block order, four loads in flight
+    const int n = min(P, 32);
+    for (int k0 = 0; k0 < n; k0 += 4) {
+      float4 o[4];
+      float wk[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int k = k0 + u;
+        const int64_t pk = __shfl_sync(0xffffffffu, pos, k & 31);
+        wk[u] = __shfl_sync(0xffffffffu, wl, k & 31);
+        o[u] = (k < n && pk >= 0) ? load_half4(m.part_o + pk * kHeadDim + lane * 4) : make_float4(0.f, 0.f, 0.f, 0.f);
+        if (!(k < n && pk >= 0)) wk[u] = 0.f;
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        acc.x += wk[u] * o[u].x;
+        acc.y += wk[u] * o[u].y;
+        acc.z += wk[u] * o[u].z;
+        acc.w += wk[u] * o[u].w;
+      }
+    }
+  } else {
+    // every past block selected (topk >= number of blocks): chunks of 32
+    float mx = own_l;
+    for (int i0 = 0; i0 < P; i0 += 32) {
+      float li;
+      slot(i0 + lane, li);
+      mx = fmaxf(mx, warp_max(li));
+    }
+    float sum = 0.f;
+    for (int i0 = 0; i0 < P; i0 += 32) {
+      float li;
+      slot(i0 + lane, li);
+      sum += warp_sum(li == -INFINITY ? 0.f : expf(li - mx));
+    }
+    sum += expf(own_l - mx);
+    L = mx + logf(sum);
+    for (int i0 = 0; i0 < P; i0 += 32) {
+      float li;
+      const int64_t pos = slot(i0 + lane, li);
+      const int n = min(32, P - i0);
+      for (int k = 0; k < n; ++k) {
+        const int64_t pk = __shfl_sync(0xffffffffu, pos, k);
+        const float lk = __shfl_sync(0xffffffffu, li, k);
+        if (pk >= 0) {
+          const float wk = expf(lk - L);
+          const float4 o = load_half4(m.part_o + pk * kHeadDim + lane * 4);
+          acc.x += wk * o.x;
+          acc.y += wk * o.y;
+          acc.z += wk * o.z;
+          acc.w += wk * o.w;
+        }
       }
     }
   }
   {
     const float wk = expf(own_l - L);
-    const float4 o = __ldg(reinterpret_cast<const float4*>(m.own_o + (tl * w.Hq + h) * kHeadDim) + lane);
+    const float4 o = load_half4(m.own_o + (tl * w.Hq + h) * kHeadDim + lane * 4);
     acc.x += wk * o.x;
     acc.y += wk * o.y;
     acc.z += wk * o.z;

@@ -176,8 +176,8 @@ size_t window_bytes(const Plan& p, int64_t W) {
   const int64_t wwords = (W * p.G + 31) / 32;
   const int64_t list = W * p.Hq * p.P;
   const int64_t tiles = list / moba::kUnitRowsRouted + nbk + (W / moba::kTile + 1) * p.Hkv * ((p.G + 1) / 2);
-  return (size_t)(nbk * wwords * 8 + list * (4 + 4 + 4 * moba::kHeadDim) + tiles * 16 +
-                  W * p.Hq * (4 + 4 * moba::kHeadDim));
+  return (size_t)(nbk * wwords * 8 + list * (4 + 4 + 2 * moba::kHeadDim) + tiles * 16 +
+                  W * p.Hq * (4 + 2 * moba::kHeadDim));
 }
 
 // Scratch layout for a query window of W tokens.
@@ -202,9 +202,9 @@ void layout_for_window(Plan& p, int64_t W) {
   p.o_list = c.take((size_t)std::max<int64_t>(p.list_cap, 1) * 4);
   p.o_tiles = c.take((size_t)p.tile_cap * 16);
   p.o_hdr = c.take(16);
-  p.o_part_o = c.take((size_t)std::max<int64_t>(p.list_cap, 1) * moba::kHeadDim * 4);
+  p.o_part_o = c.take((size_t)std::max<int64_t>(p.list_cap, 1) * moba::kHeadDim * 2);
   p.o_part_lse = c.take((size_t)std::max<int64_t>(p.list_cap, 1) * 4);
-  p.o_own_o = c.take((size_t)W * p.Hq * moba::kHeadDim * 4);
+  p.o_own_o = c.take((size_t)W * p.Hq * moba::kHeadDim * 2);
   p.o_own_lse = c.take((size_t)W * p.Hq * 4);
   p.total = c.off;
 }
@@ -364,9 +364,9 @@ int run_forward(const Plan& p, const DeviceInfo& dev, const void* q, const void*
   int32_t* list = reinterpret_cast<int32_t*>(ws + p.o_list);
   int4* tiles = reinterpret_cast<int4*>(ws + p.o_tiles);
   int32_t* hdr = reinterpret_cast<int32_t*>(ws + p.o_hdr);
-  float* part_o = reinterpret_cast<float*>(ws + p.o_part_o);
+  __half* part_o = reinterpret_cast<__half*>(ws + p.o_part_o);
   float* part_lse = reinterpret_cast<float*>(ws + p.o_part_lse);
-  float* own_o = reinterpret_cast<float*>(ws + p.o_own_o);
+  __half* own_o = reinterpret_cast<__half*>(ws + p.o_own_o);
   float* own_lse = reinterpret_cast<float*>(ws + p.o_own_lse);
 
   CUtensorMap tmk, tmv;
