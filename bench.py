@@ -141,6 +141,27 @@ def dist_env():
     return int(os.environ.get("RANK", 0)), int(os.environ.get("WORLD_SIZE", 1)), int(os.environ.get("LOCAL_RANK", 0))
 
 
+def replica_workload(w, rank: int):
+    """Rank r's own sequence: the workload's shape, an independent seed."""
+    return si.Workload(w.name, w.seqlen, w.heads_q, w.heads_kv, w.head_dim, w.block_size, w.topk,
+                       w.seed + 7919 * rank)
+
+
+def max_over_ranks(values, device, world: int):
+    """Element-wise MAX of per-rank timings (every rank takes this step)."""
+    import torch
+    t = torch.tensor(list(values), dtype=torch.float64, device=device)
+    if world > 1:
+        import torch.distributed as dist
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.tolist()
+
+
+def job_tokens_per_s(world: int, seqlen: int, steps: int, max_total_ms: float) -> float:
+    """Whole-job throughput: every rank's tokens over the slowest rank's time."""
+    return world * seqlen * steps / (max_total_ms / 1e3)
+
+
 # ------------------------------------------------------------------ oracle
 
 def oracle_sample(w, seconds: float, seed: int):
@@ -225,8 +246,7 @@ def run_ours(args, w):
     if world > 1:
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=dev)
     # every rank: its own sequence (independent seed), same shape
-    wr = si.Workload(w.name, w.seqlen, w.heads_q, w.heads_kv, w.head_dim, w.block_size, w.topk,
-                     w.seed + 7919 * rank)
+    wr = replica_workload(w, rank)
     S, Hq, Hkv, d = wr.seqlen, wr.heads_q, wr.heads_kv, wr.head_dim
     q_h = torch.empty((S, Hq, d), dtype=torch.bfloat16, pin_memory=True)
     k_h = torch.empty((S, Hkv, d), dtype=torch.bfloat16, pin_memory=True)
@@ -311,16 +331,13 @@ def run_ours(args, w):
     e2e_total = sum(e2e_ms)
 
     # max over ranks of the device time
-    tm = torch.tensor([total_ms, e2e_total, stages["attention"]], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(tm, op=dist.ReduceOp.MAX)
-    total_ms, e2e_total, attn_ms_max = tm.tolist()
+    total_ms, e2e_total, _ = max_over_ranks([total_ms, e2e_total, stages["attention"]], dev, world)
 
     line = None
     if rank == 0:
         peaks, peaks_src = load_peaks()
         flops = moba.effective_flops(S, Hq, wr.block_size, wr.topk, d)
-        value = world * S * args.steps / (total_ms / 1e3)
+        value = job_tokens_per_s(world, S, args.steps, total_ms)
         ms_per_step = total_ms / args.steps
         attn_ms = stages["attention"] / max(calls, 1)
         long_step = ms_per_step > 200.0
@@ -346,7 +363,7 @@ def run_ours(args, w):
                          "peak_source": f"{peaks_src} bf16 {'sustained' if long_step else 'burst'}",
                          "algorithmic": f"{flops:.4e} selected-block FLOPs per step / attention ms per step"},
             "stage_roofline_hbm": stage_roof,
-            "e2e": {"value": world * S * e2e_steps / (e2e_total / 1e3), "unit": "tokens/s",
+            "e2e": {"value": job_tokens_per_s(world, S, e2e_steps, e2e_total), "unit": "tokens/s",
                     "h2d_bytes_per_step": int(q_h.nbytes + k_h.nbytes + v_h.nbytes),
                     "d2h_bytes_per_step": int(out_h.nbytes + lse_h.nbytes)},
             "gpu_launches": launches // max(calls, 1) * args.steps,
