@@ -51,6 +51,7 @@ constexpr uint32_t kHalfBytes = kTileBytes / 2;        // one 64-column half
 constexpr int kUnitRows = 2 * kTile;                   // rows of a routed unit
 constexpr int kAttnSmemBytes = (2 + 2 * kStages) * kTileBytes + 1024 + 512;
 constexpr uint32_t kNoHead = 0xFFFFu;
+constexpr uint32_t kNextTile = 0xFFFEu;  // own tile B: the next 128 tokens of tile A's head
 
 struct AttnParams {
   const __nv_bfloat16* q;   // [S][Hq][128]
@@ -90,7 +91,8 @@ struct UnitInfo {
   int rows[2];     // valid rows of tile A, B
   int h[2];        // own: q heads of tile A, B
   int list0[2];    // routed: first list slot of tile A, B
-  int64_t t0;      // own: first token
+  int64_t tq[2];   // own: first token of tile A, B
+  int diag[2];     // own: the step whose keys start at tile X's first token
 };
 
 __device__ __forceinline__ UnitInfo decode_unit(const AttnParams& p, int idx) {
@@ -99,19 +101,31 @@ __device__ __forceinline__ UnitInfo decode_unit(const AttnParams& p, int idx) {
   if (d.w < 0) {
     u.own = true;
     u.nsteps = -d.w;
-    u.t0 = d.x;
+    u.tq[0] = d.x;
     u.h[0] = d.z & 0xFFFF;
-    u.h[1] = (int)((uint32_t)d.z >> 16);
-    u.has_b = (uint32_t)u.h[1] != kNoHead;
+    const uint32_t hb = (uint32_t)d.z >> 16;
     u.g = u.h[0] / p.G;
-    u.key0 = u.t0 - (int64_t)(u.nsteps - 1) * kTile;
     u.rows[0] = d.y;
-    u.rows[1] = u.has_b ? d.y : 0;
     u.list0[0] = u.list0[1] = 0;
+    if (hb == kNextTile) {
+      // the same head's next 128 tokens: one more key step than tile A
+      u.has_b = true;
+      u.h[1] = u.h[0];
+      u.tq[1] = u.tq[0] + kTile;
+      u.rows[1] = (int)min((int64_t)kTile, p.S - u.tq[1]);
+      u.diag[0] = u.nsteps - 2;
+      u.diag[1] = u.nsteps - 1;
+    } else {
+      u.has_b = hb != kNoHead;
+      u.h[1] = (int)hb;
+      u.tq[1] = u.tq[0];
+      u.rows[1] = u.has_b ? d.y : 0;
+      u.diag[0] = u.diag[1] = u.nsteps - 1;
+    }
+    u.key0 = u.tq[0] - (int64_t)u.diag[0] * kTile;
   } else {
     u.own = false;
     u.nsteps = p.B / kTile;
-    u.t0 = 0;
     u.g = d.z;
     u.key0 = (int64_t)d.w * p.B;
     u.rows[0] = min(d.y, kTile);
@@ -120,6 +134,8 @@ __device__ __forceinline__ UnitInfo decode_unit(const AttnParams& p, int idx) {
     u.list0[0] = d.x;
     u.list0[1] = d.x + kTile;
     u.h[0] = u.h[1] = 0;
+    u.tq[0] = u.tq[1] = 0;
+    u.diag[0] = u.diag[1] = u.nsteps;
   }
   return u;
 }
@@ -230,13 +246,13 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     return true;
   };
 
-  // register split: the two softmax warpgroups take 200 per thread, the
-  // producer/MMA/gather warpgroup 104 (256*200 + 128*104 = 64512, exactly
+  // register split: the two softmax warpgroups take 192 per thread, the
+  // producer/MMA/gather warpgroup 120 (256*192 + 128*120 = 64512, exactly
   // the 384*168 registers the block is launched with)
   if (warp < 8) {
-    asm volatile("setmaxnreg.inc.sync.aligned.u32 200;\n" ::: "memory");
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 192;\n" ::: "memory");
   } else {
-    asm volatile("setmaxnreg.dec.sync.aligned.u32 104;\n" ::: "memory");
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 120;\n" ::: "memory");
   }
 
   if (warp < 8) {
@@ -253,6 +269,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       if (ui < 0) break;
       const UnitInfo u = decode_unit(p, ui);
       if (X == 1 && !u.has_b) continue;
+      // own unit: from step dstep on, tile X's keys reach its first token
+      const int dstep = u.own ? (X ? u.diag[1] : u.diag[0]) : u.nsteps;
       float m_run = -INFINITY, l_run = 0.f;
       for (int s = 0; s < u.nsteps; ++s, ++sx) {
         if (!mbar_wait(&sh->s_full[X], sx & 1, abort_flag)) goto done;
@@ -270,12 +288,14 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           tmem_ld32(tS + 96, r3);
           tmem_ld_wait();
         }
-        // causal mask on the diagonal step of an own unit: key > query
-        const bool diag = u.own && (s == u.nsteps - 1);
+        // causal mask in an own unit from the step whose keys start at the
+        // tile's first token: key > query (a later step is fully masked)
+        const bool diag = s >= dstep;
         if (diag) {
+          const int lim = row - (s - dstep) * kTile;  // keys e > lim are masked
 #pragma unroll
           for (int e = 0; e < 128; ++e)
-            if (e > row) r[e] = __float_as_uint(-INFINITY);
+            if (e > lim) r[e] = __float_as_uint(-INFINITY);
         }
         // row max: eight independent chains of 3-input max over columns
         // c, c+8, ..., c+120
@@ -340,7 +360,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         __half* dst_o;
         float* dst_lse;
         if (u.own) {
-          const int64_t rr = (u.t0 + row - p.w0) * p.Hq + (X ? u.h[1] : u.h[0]);
+          const int64_t rr = ((X ? u.tq[1] : u.tq[0]) + row - p.w0) * p.Hq + (X ? u.h[1] : u.h[0]);
           dst_o = p.own_o + rr * kHeadDim;
           dst_lse = p.own_lse + rr;
         } else {
@@ -537,36 +557,56 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       if (ui < 0) break;
       const UnitInfo u = decode_unit(p, ui);
       const int nx = u.has_b ? 2 : 1;
+      // Thread gt copies whole rows gt and gt + 64 of each tile (16 chunks of
+      // 16 B each). Their element offsets in q are found first (a routed
+      // tile reads its row list), before waiting for the tiles' buffers, so
+      // the list reads overlap the previous unit's last step; then both
+      // tiles' copies are in flight together and complete with one wait.
+      int64_t off[2][2];
 #pragma unroll
       for (int x = 0; x < 2; ++x) {
-        if (x >= nx) break;
-        if (!mbar_wait(&sh->q_empty[x], (ux[x] & 1) ^ 1, abort_flag)) goto gather_done;
-        const uint32_t dst0 = smem_u32(sQ + x * kTileBytes);
-#pragma unroll 4
-        for (int i = 0; i < 32; ++i) {
-          const int idx = gt + 64 * i;  // 2048 chunks of 16 B
-          const int r = idx >> 4, c16 = idx & 15;
-          const int half = c16 >> 3, c = c16 & 7;
-          const __nv_bfloat16* src = p.q;
-          uint32_t bytes = 0;
-          if (r < u.rows[x]) {
+#pragma unroll
+        for (int k = 0; k < 2; ++k) {
+          const int r = gt + 64 * k;
+          off[x][k] = -1;
+          if (x < nx && r < u.rows[x]) {
             int64_t t;
             int h;
             if (u.own) {
-              t = u.t0 + r;
+              t = u.tq[x] + r;
               h = u.h[x];
             } else {
               const int rr = __ldg(p.list + u.list0[x] + r);
               t = p.w0 + rr / p.G;
               h = u.g * p.G + rr % p.G;
             }
-            src = p.q + (t * p.Hq + h) * kHeadDim + c16 * 8;
-            bytes = 16;
+            off[x][k] = (t * p.Hq + h) * kHeadDim;
           }
-          cp_async_16(dst0 + half * kHalfBytes + r * 128 + ((c ^ (r & 7)) << 4), src, bytes);
         }
-        cp_async_wait_all();
-        fence_proxy_async_smem();
+      }
+#pragma unroll
+      for (int x = 0; x < 2; ++x) {
+        if (x >= nx) break;
+        if (!mbar_wait(&sh->q_empty[x], (ux[x] & 1) ^ 1, abort_flag)) goto gather_done;
+        const uint32_t dst0 = smem_u32(sQ + x * kTileBytes);
+#pragma unroll
+        for (int k = 0; k < 2; ++k) {
+          const int r = gt + 64 * k;
+          const bool valid = off[x][k] >= 0;
+          const __nv_bfloat16* src = valid ? p.q + off[x][k] : p.q;
+#pragma unroll
+          for (int c16 = 0; c16 < 16; ++c16) {
+            const int half = c16 >> 3, c = c16 & 7;
+            cp_async_16(dst0 + half * kHalfBytes + r * 128 + ((c ^ (r & 7)) << 4), src + (valid ? c16 * 8 : 0),
+                        valid ? 16u : 0u);
+          }
+        }
+      }
+      cp_async_wait_all();
+      fence_proxy_async_smem();
+#pragma unroll
+      for (int x = 0; x < 2; ++x) {
+        if (x >= nx) break;
         mbar_arrive(&sh->q_full[x]);
         ++ux[x];
       }

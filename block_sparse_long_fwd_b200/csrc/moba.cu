@@ -180,8 +180,15 @@ size_t window_bytes(const Plan& p, int64_t W) {
                   W * p.Hq * (4 + 2 * moba::kHeadDim));
 }
 
+// Own-block work units pair two consecutive 128-token tiles of one head when
+// a group has a single q head (else they pair two heads of a group); pairs
+// stay inside a block, so B / 128 must be even, and inside a window, so
+// windows then start at multiples of 256 tokens.
+bool pair_tokens(const Plan& p) { return p.G == 1 && (p.B / moba::kTile) % 2 == 0; }
+
 // Scratch layout for a query window of W tokens.
 void layout_for_window(Plan& p, int64_t W) {
+  if (pair_tokens(p) && W < (p.S + 127) / 128 * 128) W = std::max<int64_t>(256, W / 256 * 256);
   p.W = W;
   p.wwords = (W * p.G + 31) / 32;
   const int64_t nbk = (int64_t)p.Hkv * p.nbp;
@@ -417,6 +424,7 @@ int run_forward(const Plan& p, const DeviceInfo& dev, const void* q, const void*
     wg.w0 = w0;
     wg.wlen = std::min(p.W, p.S - w0);
     wg.wwords = (wg.wlen * p.G + 31) / 32;
+    wg.pair_tokens = pair_tokens(p) ? 1 : 0;
     const bool routed = p.P > 0 && p.nbp > 0 && (w0 + wg.wlen) > p.B;
     if (routed) {
       dim3 gf((unsigned)((wg.wwords + 7) / 8), p.Hkv);

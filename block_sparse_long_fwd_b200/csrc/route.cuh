@@ -30,6 +30,7 @@ struct WindowGeom {
   int k_eff, nbp;   // blocks per row; number of poolable (past-able) blocks
   int64_t w0, wlen;  // window start token and length
   int64_t wwords;    // flag words per bucket: ceil(wlen * G / 32)
+  int pair_tokens;   // own units pair consecutive 128-token tiles of one head
 };
 
 // First flag word of bucket j that can hold a set bit: rows with t >= (j+1)B.
@@ -127,7 +128,9 @@ __device__ __forceinline__ int64_t block_incl_scan_1024(int64_t v, int64_t* scra
 //          entries of bucket (g, j);
 //   own    {t0, nrows (1..128), hA | hB << 16, -nsteps}: 128 tokens of two
 //          q heads of one group (hB = 0xFFFF when the group has an odd
-//          head left over).
+//          head left over); with one head per group (pair_tokens), tile A
+//          is tokens [t0, t0 + 128) and tile B (hB = 0xFFFE) the next 128
+//          tokens of the same head and block.
 // hdr[0] = routed units, hdr[1] = all units, hdr[2] = list entries,
 // hdr[3] = the attention kernel's next-unit counter (zeroed here).
 constexpr int kUnitRowsRouted = 256;
@@ -162,10 +165,15 @@ __global__ void __launch_bounds__(1024) route_scan_kernel(const int32_t* __restr
   // own-block units: 128-token tiles u of the window, one unit per pair of
   // q heads of a group; tile u of block-position p = ((w0/128 + u) mod
   // (B/128)) has p + 1 key steps. Units are ordered longest first.
-  const int period = w.B / kTile;
-  const int64_t nu = (w.wlen + kTile - 1) / kTile;
-  const int64_t u_off = w.w0 / kTile;
-  const int npairs = (w.G + 1) / 2;
+  // With pair_tokens (one head per group, B/128 even, w0 a multiple of 256)
+  // the same scheme runs over 256-token pairs of tiles: pair v of pair
+  // position p has 2p + 2 key steps (2p + 1 when the window ends after its
+  // first tile).
+  const int period = w.pair_tokens ? w.B / (2 * kTile) : w.B / kTile;
+  const int span = w.pair_tokens ? 2 * kTile : kTile;
+  const int64_t nu = (w.wlen + span - 1) / span;
+  const int64_t u_off = w.w0 / span;
+  const int npairs = w.pair_tokens ? 1 : (w.G + 1) / 2;
   const int per_u = w.Hkv * npairs;
   // count tiles per position p (period <= 1024 checked on the host)
   __shared__ int cntp[1024];
@@ -187,8 +195,15 @@ __global__ void __launch_bounds__(1024) route_scan_kernel(const int32_t* __restr
   for (int64_t u = threadIdx.x; u < nu; u += 1024) {
     const int p = (int)((u_off + u) % period);
     const int64_t rank = basep[p] + u / period;  // u' < u with the same p: u / period of them
-    const int64_t t0 = w.w0 + u * kTile;
+    const int64_t t0 = w.w0 + u * span;
     const int nrows = (int)min((int64_t)kTile, w.w0 + w.wlen - t0);
+    if (w.pair_tokens) {
+      const bool has_b = t0 + kTile < w.w0 + w.wlen;
+      for (int g = 0; g < w.Hkv; ++g)
+        units[n_routed + rank * per_u + g] =
+            make_int4((int)t0, nrows, g | ((has_b ? 0xFFFE : 0xFFFF) << 16), -(2 * p + (has_b ? 2 : 1)));
+      continue;
+    }
     for (int g = 0; g < w.Hkv; ++g) {
       for (int q = 0; q < npairs; ++q) {
         const int hA = g * w.G + 2 * q;

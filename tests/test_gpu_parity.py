@@ -32,6 +32,8 @@ SMALL = [
     (1536,  2,  1,   128, 20,   7),     # topk >= blocks: full causal attention
     (2125,  2,  1,   256, 5,    8),     # ragged, several routed blocks
     (8192,  4,  1,   512, 9,    9),     # many past blocks per row
+    (3000,  1,  1,   256, 4,    10),    # one head per group: own tiles paired by token, ragged last pair
+    (2900,  2,  2,   512, 3,    11),    # paired own tiles, last pair without its second tile
 ]
 
 
@@ -42,10 +44,11 @@ def test_small_all_rows(S, Hq, Hkv, B, topk, seed):
     print(stats)
 
 
-@pytest.mark.parametrize("window", [128, 384, 1024])
-def test_query_windows(monkeypatch, window):
-    S, Hq, Hkv, B, topk = 2125, 4, 2, 256, 4
-    w, q, k, v = make_inputs(S, Hq, Hkv, B, topk, 40 + window)
+@pytest.mark.parametrize("window,heads", [(128, (4, 2)), (384, (4, 2)), (1024, (4, 2)), (384, (2, 2)), (640, (1, 1))])
+def test_query_windows(monkeypatch, window, heads):
+    # (1, 1) and (2, 2): one head per group, windows rounded to 256 tokens for paired own tiles
+    S, (Hq, Hkv), B, topk = 2125, heads, 256, 4
+    w, q, k, v = make_inputs(S, Hq, Hkv, B, topk, 40 + window + Hq)
     monkeypatch.setenv("MOBA_WINDOW", str(window))
     stats = full_check(q, k, v, B, topk)
     print(window, stats)
