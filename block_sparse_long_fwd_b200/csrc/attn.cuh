@@ -189,6 +189,7 @@ __device__ __forceinline__ void exp_row(const uint32_t (&r)[128], uint64_t c2, u
 __global__ void __launch_bounds__(kAttnThreads, 1)
     attn_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant__ CUtensorMap tmap_v,
                 AttnParams p) {
+  grid_dependency_sync();
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sQ = smem;                         // tile A, tile B

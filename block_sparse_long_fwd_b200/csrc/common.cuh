@@ -87,6 +87,18 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
   }
 }
 
+// ------------------------------------------------ programmatic dependent launch
+
+// The kernels of one forward pass are launched with programmatic stream
+// serialization, so a kernel may be scheduled while its predecessor is still
+// running. Each kernel first waits until its predecessor grid has completed
+// and its writes are visible (so the wait is transitive along the chain),
+// then lets its own successor launch. Outside such a launch both are no-ops.
+__device__ __forceinline__ void grid_dependency_sync() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // ------------------------------------------------------------ async copies
 
 __device__ __forceinline__ void fence_proxy_async_smem() {

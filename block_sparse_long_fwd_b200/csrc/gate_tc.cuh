@@ -42,6 +42,7 @@ __host__ __device__ inline int gate_rows_padded(int nbp) {
 __global__ void __launch_bounds__(128) kmean_split_kernel(const float* __restrict__ part, int splits, int nbp,
                                                           int nbp_pad, __nv_bfloat16* __restrict__ hi,
                                                           __nv_bfloat16* __restrict__ lo) {
+  grid_dependency_sync();
   const int j = blockIdx.x, g = blockIdx.y, c = threadIdx.x;
   const int64_t o = ((int64_t)g * nbp_pad + j) * kHeadDim + c;
   if (j < nbp) {
@@ -109,6 +110,7 @@ template <int KP>
 __global__ void __launch_bounds__(kGateTcThreads)
     gate_tc_kernel(const __grid_constant__ CUtensorMap tm_hi, const __grid_constant__ CUtensorMap tm_lo,
                    GateParams p) {
+  grid_dependency_sync();
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sQ = smem;
@@ -305,6 +307,7 @@ __global__ void __launch_bounds__(kGateTcThreads)
 // (every past block). grid ceil(S*Hq / 256), 256 threads.
 __global__ void __launch_bounds__(256) sel_fill_kernel(int32_t* __restrict__ sel, int64_t S, int Hq, int B,
                                                         int k_eff, int full) {
+  grid_dependency_sync();
   const int64_t i = (int64_t)blockIdx.x * 256 + threadIdx.x;
   if (i >= S * Hq) return;
   const int h = (int)(i / S);

@@ -48,6 +48,7 @@ __device__ __forceinline__ float warp_sum(float v) {
 // grid ceil(wlen * Hq / 8), 256 threads: one warp per (token, q head) row,
 // lane c owns channels 4c..4c+3.
 __global__ void __launch_bounds__(256) merge_kernel(MergeParams m) {
+  grid_dependency_sync();
   const WindowGeom& w = m.w;
   const int lane = threadIdx.x & 31;
   const int64_t row = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);

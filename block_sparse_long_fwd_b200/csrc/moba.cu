@@ -261,11 +261,30 @@ int make_mean_map(CUtensorMap* map, const void* base, int64_t rows) {
   return MOBA_OK;
 }
 
+// Launches a pipeline kernel with programmatic stream serialization: it may
+// be scheduled while the previous kernel on the stream is still running; the
+// kernel itself waits for that kernel's completion before reading anything
+// (grid_dependency_sync in common.cuh).
+template <typename... KArgs, typename... Args>
+void launch_chained(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaLaunchKernelEx(&cfg, kernel, args...);
+}
+
 template <int KP>
 void launch_gate_tc(const Plan& p, const CUtensorMap& mhi, const CUtensorMap& mlo, const moba::GateParams& gp,
                     cudaStream_t st) {
   dim3 grid((unsigned)((p.S * p.G + 127) / 128), p.Hkv);
-  moba::gate_tc_kernel<KP><<<grid, moba::kGateTcThreads, moba::kGateSmemBytes, st>>>(mhi, mlo, gp);
+  launch_chained(moba::gate_tc_kernel<KP>, grid, dim3(moba::kGateTcThreads), moba::kGateSmemBytes, st, mhi, mlo, gp);
 }
 
 // Gate + top-k into sel. kmean (fp32) is split into khi/klo (bf16, padded
@@ -276,11 +295,13 @@ int launch_gate(const Plan& p, const void* q, const float* kmean, int splits, __
   const bool full = p.k_eff == p.nb;
   if (p.P == 0 || full || p.nbp <= 0) {
     const int64_t n = p.S * p.Hq;
-    moba::sel_fill_kernel<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(sel, p.S, p.Hq, p.B, p.k_eff, full ? 1 : 0);
+    launch_chained(moba::sel_fill_kernel, dim3((unsigned)((n + 255) / 256)), dim3(256), 0, st, sel, p.S, p.Hq, p.B,
+                   p.k_eff, full ? 1 : 0);
     return 1;
   }
   const int nbp_pad = moba::gate_rows_padded(p.nbp);
-  moba::kmean_split_kernel<<<dim3(nbp_pad, p.Hkv), 128, 0, st>>>(kmean, splits, p.nbp, nbp_pad, khi, klo);
+  launch_chained(moba::kmean_split_kernel, dim3(nbp_pad, p.Hkv), dim3(128), 0, st, kmean, splits, p.nbp, nbp_pad, khi,
+                 klo);
   CUtensorMap mhi, mlo;
   int rc = make_mean_map(&mhi, khi, (int64_t)p.Hkv * nbp_pad);
   if (rc) return -rc;
@@ -308,8 +329,8 @@ int launch_gate(const Plan& p, const void* q, const float* kmean, int splits, __
 void launch_pool(const Plan& p, const void* k, float* kmean, int splits, cudaStream_t st) {
   if (p.nbp <= 0) return;
   dim3 grid(p.nbp, p.Hkv, splits);
-  moba::pool_kernel<<<grid, moba::kPoolThreads, 0, st>>>(static_cast<const __nv_bfloat16*>(k), p.Hkv, p.B, p.nbp,
-                                                         splits, kmean);
+  launch_chained(moba::pool_kernel, grid, dim3(moba::kPoolThreads), 0, st, static_cast<const __nv_bfloat16*>(k), p.Hkv,
+                 p.B, p.nbp, splits, kmean);
 }
 
 // Optional per-stage device timing: an event after every stage, tagged with
@@ -428,21 +449,24 @@ int run_forward(const Plan& p, const DeviceInfo& dev, const void* q, const void*
     const bool routed = p.P > 0 && p.nbp > 0 && (w0 + wg.wlen) > p.B;
     if (routed) {
       dim3 gf((unsigned)((wg.wwords + 7) / 8), p.Hkv);
-      moba::route_flags_kernel<<<gf, 256, 0, st>>>(sel, wg, flags);
+      launch_chained(moba::route_flags_kernel, gf, dim3(256), 0, st, static_cast<const int32_t*>(sel), wg, flags);
       dim3 gb(p.nbp, p.Hkv);
-      moba::route_count_kernel<<<gb, 256, 0, st>>>(flags, wg, cnt);
+      launch_chained(moba::route_count_kernel, gb, dim3(256), 0, st, static_cast<const uint32_t*>(flags), wg, cnt);
       tm->count(2);
     }
-    moba::route_scan_kernel<<<1, 1024, 0, st>>>(cnt, routed ? nbk : 0, wg, loff, toff, tiles, hdr);
+    launch_chained(moba::route_scan_kernel, dim3(1), dim3(1024), 0, st, static_cast<const int32_t*>(cnt), routed ? nbk : 0,
+                   wg, loff, toff, tiles, hdr);
     tm->count(1);
     if (routed) {
       dim3 gb(p.nbp, p.Hkv);
-      moba::route_fill_kernel<<<gb, 256, 0, st>>>(flags, cnt, loff, toff, wg, wordbase, list, tiles);
+      launch_chained(moba::route_fill_kernel, gb, dim3(256), 0, st, static_cast<const uint32_t*>(flags),
+                     static_cast<const int32_t*>(cnt), static_cast<const int32_t*>(loff),
+                     static_cast<const int32_t*>(toff), wg, wordbase, list, tiles);
       tm->count(1);
     }
     tm->mark(kRoute);
     ap.w0 = w0;
-    moba::attn_kernel<<<dev.sms, moba::kAttnThreads, moba::kAttnSmemBytes, st>>>(tmk, tmv, ap);
+    launch_chained(moba::attn_kernel, dim3(dev.sms), dim3(moba::kAttnThreads), moba::kAttnSmemBytes, st, tmk, tmv, ap);
     tm->count(1);
     tm->mark(kAttn);
     moba::MergeParams mp;
@@ -457,7 +481,7 @@ int run_forward(const Plan& p, const DeviceInfo& dev, const void* q, const void*
     mp.lse = lse;
     mp.w = wg;
     const int64_t rows = wg.wlen * p.Hq;
-    moba::merge_kernel<<<(unsigned)((rows + 7) / 8), 256, 0, st>>>(mp);
+    launch_chained(moba::merge_kernel, dim3((unsigned)((rows + 7) / 8)), dim3(256), 0, st, mp);
     tm->count(1);
     tm->mark(kMerge);
   }

@@ -23,6 +23,7 @@ constexpr int kPoolThreads = 256;
 
 __global__ void __launch_bounds__(kPoolThreads) pool_kernel(const __nv_bfloat16* __restrict__ k, int Hkv, int B,
                                                             int nbp, int splits, float* __restrict__ out) {
+  grid_dependency_sync();
   const int j = blockIdx.x, g = blockIdx.y, sp = blockIdx.z;
   const int rows = B / splits;
   const int chunk = threadIdx.x & 15, rg = threadIdx.x >> 4;

@@ -44,6 +44,7 @@ __device__ __forceinline__ int64_t bucket_word_begin(const WindowGeom& w, int j)
 // 1. grid (ceil(wwords / 8), Hkv), 256 threads: one warp per flag word.
 __global__ void __launch_bounds__(256) route_flags_kernel(const int32_t* __restrict__ sel, WindowGeom w,
                                                           uint32_t* __restrict__ flags) {
+  grid_dependency_sync();
   const int g = blockIdx.y;
   const int lane = threadIdx.x & 31;
   const int64_t word = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
@@ -90,6 +91,7 @@ __device__ __forceinline__ int block_sum_256(int v, int* scratch) {
 // 2. grid (nbp, Hkv), 256 threads.
 __global__ void __launch_bounds__(256) route_count_kernel(const uint32_t* __restrict__ flags, WindowGeom w,
                                                           int32_t* __restrict__ cnt) {
+  grid_dependency_sync();
   const int j = blockIdx.x, g = blockIdx.y;
   const uint32_t* f = flags + ((int64_t)g * w.nbp + j) * w.wwords;
   int c = 0;
@@ -139,6 +141,7 @@ __global__ void __launch_bounds__(1024) route_scan_kernel(const int32_t* __restr
                                                           WindowGeom w, int32_t* __restrict__ list_off,
                                                           int32_t* __restrict__ tile_off, int4* __restrict__ units,
                                                           int32_t* __restrict__ hdr) {
+  grid_dependency_sync();
   __shared__ int64_t scratch[32];
   __shared__ int64_t last[2];
   int64_t carry_l = 0, carry_t = 0;
@@ -227,6 +230,7 @@ __global__ void __launch_bounds__(256) route_fill_kernel(const uint32_t* __restr
                                                          const int32_t* __restrict__ tile_off, WindowGeom w,
                                                          int32_t* __restrict__ wordbase, int32_t* __restrict__ list,
                                                          int4* __restrict__ tiles) {
+  grid_dependency_sync();
   const int j = blockIdx.x, g = blockIdx.y;
   const int b = g * w.nbp + j;
   const int64_t foff = (int64_t)b * w.wwords;
