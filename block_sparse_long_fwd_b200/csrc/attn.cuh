@@ -334,8 +334,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           m_run = m_ref;
         }
         // O rescale: S_X(s) was issued after PV_X(s-1) completed, so O_X is
-        // settled here, and PV_X(s) waits for p_full below
-        if (rescale) {
+        // settled here, and PV_X(s) waits for p_full below. The decision is
+        // per row, but tcgen05.ld/st are warp-collective: the whole warp
+        // takes the branch when any of its rows moves its reference (the
+        // others multiply by factor 1).
+        if (__any_sync(0xffffffffu, rescale)) {
 #pragma unroll
           for (int c = 0; c < 4; ++c) {
             uint32_t o[32];

@@ -216,6 +216,21 @@ void layout_for_window(Plan& p, int64_t W) {
   p.total = c.off;
 }
 
+// Full causal attention (topk >= the number of blocks) does not depend on the
+// block size: every row attends all keys up to itself. It then runs with the
+// largest block the kernels take (a single block when the sequence fits in
+// one), so the work is own-block units (a causal FlashAttention-style pass):
+// no gate scores, no routing, one partial per row.
+void dense_blocks(Plan& p) {
+  if (p.nb <= 1 || p.k_eff < p.nb) return;
+  const int64_t S256 = (p.S + 255) / 256 * 256;
+  p.B = (int)std::min<int64_t>(S256, 128 * 1024);
+  p.nb = (int)((p.S + p.B - 1) / p.B);
+  p.nbp = p.nb - 1;
+  p.k_eff = p.nb;
+  p.P = p.k_eff - 1;
+}
+
 int make_plan(Plan* pl, int64_t S, int Hq, int Hkv, int B, int topk) {
   Plan& p = *pl;
   p.S = S;
@@ -228,6 +243,7 @@ int make_plan(Plan* pl, int64_t S, int Hq, int Hkv, int B, int topk) {
   p.nbp = p.nb - 1;
   p.k_eff = std::min(topk, p.nb);
   p.P = p.k_eff - 1;
+  dense_blocks(p);
   const int64_t S128 = (S + 127) / 128 * 128;
   int64_t W = 0;
   if (const char* env = getenv("MOBA_WINDOW")) {
@@ -848,6 +864,7 @@ int plan_within(Plan* pl, int64_t S, int Hq, int Hkv, int B, int topk, size_t ca
   p.nbp = p.nb - 1;
   p.k_eff = std::min(topk, p.nb);
   p.P = p.k_eff - 1;
+  dense_blocks(p);
   int64_t W = (S + 127) / 128 * 128;
   while (true) {
     if (W * Hq * (int64_t)p.P < ((int64_t)1 << 31) - 1) {

@@ -53,6 +53,10 @@ WORKLOADS = {
     "128k": Workload("moba_128k_h32kv8_b4096_k12", 131072, 32, 8, 128, 4096, 12, 20250218 + 2),
     "1m": Workload("moba_1m_h32kv8_b4096_k12", 1048576, 32, 8, 128, 4096, 12, 20250218 + 3),
     "10m": Workload("moba_10m_h1_b8192_k12", 10485760, 1, 1, 128, 8192, 12, 20250218 + 4),
+    # topk >= number of blocks: full causal attention (the dense path), on the
+    # inputs of the 32K and 128K workloads
+    "32k_dense": Workload("moba_32k_h1_b2048_k16_dense", 32768, 1, 1, 128, 2048, 16, 20250218 + 1),
+    "128k_dense": Workload("moba_128k_h32kv8_b4096_k32_dense", 131072, 32, 8, 128, 4096, 32, 20250218 + 2),
 }
 
 

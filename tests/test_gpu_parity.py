@@ -34,6 +34,8 @@ SMALL = [
     (8192,  4,  1,   512, 9,    9),     # many past blocks per row
     (3000,  1,  1,   256, 4,    10),    # one head per group: own tiles paired by token, ragged last pair
     (2900,  2,  2,   512, 3,    11),    # paired own tiles, last pair without its second tile
+    (4096,  1,  1,   512, 8,    12),    # topk >= blocks, one head: the dense path, paired own tiles
+    (3000,  4,  2,   256, 64,   13),    # dense path, GQA, ragged
 ]
 
 
@@ -89,6 +91,53 @@ def test_large_workload_sampled_rows(name, nrows):
     rows = sample_rows(w, nrows, w.seed + 1000)
     stats = full_check(q, k, v, w.block_size, w.topk, rows=rows)
     print(name, stats)
+
+
+@pytest.mark.parametrize("name,nrows", [("32k_dense", 512), ("128k_dense", 128)])
+def test_dense_workload_sampled_rows(name, nrows):
+    # topk >= number of blocks is full causal attention; the library runs it
+    # as one causal pass (no gate scores, no routing) and must match the oracle
+    w = si.WORKLOADS[name]
+    q, k, v = si.make_qkv(w)
+    rows = sample_rows(w, nrows, w.seed + 2000)
+    stats = full_check(q, k, v, w.block_size, w.topk, rows=rows)
+    print(name, stats)
+
+
+def test_dense_path_launches_no_router():
+    import block_sparse_long_fwd_b200 as moba
+    S, Hq, Hkv, B, topk = 8192, 2, 2, 512, 16
+    from parity_helpers import to_dev
+    w, q, k, v = make_inputs(S, Hq, Hkv, B, topk, 21)
+    qd, kd, vd = to_dev(q), to_dev(k), to_dev(v)
+    moba.profile_begin()
+    moba.fwd(qd, kd, vd, B, topk)
+    _, launches, calls = moba.profile_end()
+    torch.cuda.synchronize()
+    # one window: selection fill, unit list, attention, merge
+    assert calls == 1 and launches == 4, launches
+
+
+def _bf16_bits(x):
+    u = np.ascontiguousarray(x, dtype=np.float32).view(np.uint32).astype(np.uint64)
+    return ((u + 0x7FFF + ((u >> 16) & 1)) >> 16).astype(np.uint16)
+
+
+def test_rescale_decided_per_row():
+    # Rows of one warp that move their softmax reference at different steps:
+    # in the second 128-key step, even rows see logits ~10 nats above the
+    # first step's (a reference move) and odd rows ~10 nats below (none).
+    # The O rescale is per row but its TMEM accesses are warp-collective.
+    S, B = 512, 512
+    rng = np.random.default_rng(5)
+    q = rng.normal(0, 0.1, (S, 1, 128)).astype(np.float32)
+    k = rng.normal(0, 0.1, (S, 1, 128)).astype(np.float32)
+    v = rng.normal(0, 1.0, (S, 1, 128)).astype(np.float32)
+    sign = np.where(np.arange(S) % 2 == 0, 1.0, -1.0)
+    q[:, 0, 0] = 10.6 * sign
+    k[128:, 0, 0] = 10.6
+    stats = full_check(_bf16_bits(q), _bf16_bits(k), _bf16_bits(v), B, 1)
+    print(stats)
 
 
 def test_bounded_wait_reports_timeout():
