@@ -81,6 +81,11 @@ def stage_bytes(w) -> dict:
     k_eff = min(w.topk, w.nblocks)
     nbp = max(w.nblocks - 1, 0)
     r = routed_rows(w)
+    if w.nblocks > 1 and k_eff == w.nblocks:
+        # full causal attention runs as one causal pass: no means, no scores,
+        # one selection entry and one partial per row
+        rows = w.seqlen * w.heads_q
+        return {"pool": 0, "gate": rows * 4, "merge": rows * 4 + 2 * rows * (d * 2 + 4)}
     return {
         # read every key that can be pooled once, write the means
         "pool": nbp * w.block_size * w.heads_kv * d * 2 + nbp * w.heads_kv * d * 4,
