@@ -230,6 +230,103 @@ def run_reference(args, w):
     return 0
 
 
+def chunk_flops(w, q0: int) -> float:
+    """Selected-block FLOPs of the rows q0..S-1 (4*d*Hq per unmasked pair)."""
+    B, S = w.block_size, w.seqlen
+    k_eff = min(w.topk, w.nblocks)
+    t = np.arange(q0, S, dtype=np.int64)
+    b = t // B
+    keys = np.where(k_eff >= w.nblocks, t + 1, np.minimum(k_eff - 1, b) * B + (t % B) + 1)
+    return 4.0 * w.head_dim * w.heads_q * float(keys.sum())
+
+
+def run_chunk(args, w):
+    """--chunk N: the last N tokens' queries against the whole cache
+    (moba_fwd_chunk; N = 1 is one decode step). One GPU."""
+    import torch
+
+    import block_sparse_long_fwd_b200 as moba
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    S, Hq, Hkv, d = w.seqlen, w.heads_q, w.heads_kv, w.head_dim
+    n = args.chunk
+    q0 = S - n
+    q_h = torch.empty((S, Hq, d), dtype=torch.bfloat16, pin_memory=True)
+    k_h = torch.empty((S, Hkv, d), dtype=torch.bfloat16, pin_memory=True)
+    v_h = torch.empty((S, Hkv, d), dtype=torch.bfloat16, pin_memory=True)
+    si.fill_q(q_h.data_ptr(), w)
+    si.fill_k(k_h.data_ptr(), w)
+    si.fill_v(v_h.data_ptr(), w)
+    qc = q_h[q0:].to(dev)
+    k, v = k_h.to(dev), v_h.to(dev)
+    out = torch.empty((n, Hq, d), dtype=torch.bfloat16, device=dev)
+    lse = torch.empty((Hq, n), dtype=torch.float32, device=dev)
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+    for _ in range(args.warmup):
+        flush.zero_()
+        moba.fwd_chunk(qc, k, v, w.block_size, w.topk, out=out, lse=lse)
+    sampler = ClockSampler(None)
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    for a, b in ev:
+        flush.zero_()
+        a.record(stream)
+        moba.fwd_chunk(qc, k, v, w.block_size, w.topk, out=out, lse=lse)
+        b.record(stream)
+    torch.cuda.synchronize()
+    total_ms = sum(a.elapsed_time(b) for a, b in ev)
+    moba.profile_begin()
+    for _ in range(args.steps):
+        flush.zero_()
+        moba.fwd_chunk(qc, k, v, w.block_size, w.topk, out=out, lse=lse)
+    stages, launches, calls = moba.profile_end()
+    torch.cuda.synchronize()
+    clocks = sampler.stop()
+    if moba.device_status() != 0:
+        raise RuntimeError("device status set: " + moba.last_error())
+    # end to end: each step uploads the chunk's new q, k, v rows into the
+    # resident cache, runs the chunk and reads out and lse back
+    out_h = torch.empty((n, Hq, d), dtype=torch.bfloat16, pin_memory=True)
+    lse_h = torch.empty((Hq, n), dtype=torch.float32, pin_memory=True)
+    e2e_steps = max(1, min(args.steps, 10))
+    t0 = time.perf_counter()
+    for _ in range(e2e_steps):
+        qc.copy_(q_h[q0:], non_blocking=True)
+        k[q0:].copy_(k_h[q0:], non_blocking=True)
+        v[q0:].copy_(v_h[q0:], non_blocking=True)
+        moba.fwd_chunk(qc, k, v, w.block_size, w.topk, out=out, lse=lse)
+        out_h.copy_(out, non_blocking=True)
+        lse_h.copy_(lse, non_blocking=True)
+        torch.cuda.synchronize()
+    e2e_ms = 1e3 * (time.perf_counter() - t0)
+    peaks, peaks_src = load_peaks()
+    flops = chunk_flops(w, q0)
+    attn_ms = stages["attention"] / max(calls, 1)
+    achieved = flops / (attn_ms / 1e3) / 1e12
+    line = {
+        "metric": METRIC, "value": n * args.steps / (total_ms / 1e3), "unit": "tokens/s", "n_gpus": 1,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": dict(workload_config(w, 1), mode="decode" if n == 1 else "chunked prefill", q_start=q0, chunk=n),
+        "eff_tflops": flops * args.steps / (total_ms / 1e3) / 1e12,
+        "stage_ms_per_step": {kk: vv / max(calls, 1) for kk, vv in stages.items()},
+        "roofline": {"bound": "tensor", "kernel": "attn_kernel", "achieved": achieved,
+                     "peak": peaks["bf16_tflops"], "unit": "TFLOP/s", "frac": achieved / peaks["bf16_tflops"],
+                     "traffic": None, "peak_source": f"{peaks_src} bf16 burst",
+                     "algorithmic": f"{flops:.4e} selected-block FLOPs of the chunk's rows / attention ms"},
+        "e2e": {"value": n * e2e_steps / (e2e_ms / 1e3), "unit": "tokens/s",
+                "h2d_bytes_per_step": int(n * (Hq + 2 * Hkv) * d * 2),
+                "d2h_bytes_per_step": int(out_h.nbytes + lse_h.nbytes)},
+        "gpu_launches": launches // max(calls, 1) * args.steps,
+        "gpu_launches_per_step": launches / max(calls, 1),
+        "clocks": clocks,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def workload_config(w, n):
     return {"workload": w.name, "seqlen": w.seqlen, "heads_q": w.heads_q, "heads_kv": w.heads_kv,
             "head_dim": w.head_dim, "block_size": w.block_size, "topk": w.topk, "batch_per_gpu": 1,
@@ -404,6 +501,8 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--seqlen", type=int, default=0, help="override the workload's seqlen (profiling cases)")
     ap.add_argument("--no-pad", action="store_true", help="no untimed load after the timed steps (profiling)")
+    ap.add_argument("--chunk", type=int, default=0,
+                    help="time only the last N tokens' queries against the whole cache (1 = one decode step)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -413,6 +512,10 @@ def main():
                         w.topk, w.seed)
     if args.impl == "reference":
         return run_reference(args, w)
+    if args.chunk:
+        if not 1 <= args.chunk <= w.seqlen:
+            ap.error("--chunk must be in [1, seqlen]")
+        return run_chunk(args, w)
     return run_ours(args, w)
 
 

@@ -32,6 +32,7 @@ MAX_TOPK = 64
 _vp, _i64, _i32 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int
 SIGNATURES = {
     "moba_fwd": (_i32, [_vp, _vp, _vp, _i64, _i32, _i32, _i32, _i32, _i32, _vp, _vp, _vp]),
+    "moba_fwd_chunk": (_i32, [_vp, _vp, _vp, _i64, _i64, _i32, _i32, _i32, _i32, _i32, _vp, _vp, _vp]),
     "moba_fwd_host": (_i32, [_vp, _vp, _vp, _i64, _i32, _i32, _i32, _i32, _i32, _vp, _vp, _vp]),
     "moba_pool": (_i32, [_vp, _i64, _i32, _i32, _i32, _vp, _vp]),
     "moba_gate": (_i32, [_vp, _vp, _i64, _i32, _i32, _i32, _i32, _i32, _vp, _vp]),
@@ -110,6 +111,29 @@ def fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, block_size: int, topk
         lse = torch.empty((Hq, S), dtype=torch.float32, device=q.device)
     _check(lib().moba_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), S, Hq, Hkv, d, block_size, topk,
                           out.data_ptr(), lse.data_ptr(), _stream(stream)))
+    return out, lse
+
+
+def fwd_chunk(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, block_size: int, topk: int, out=None, lse=None,
+              stream=None):
+    """MoBA forward for the last n = q.shape[0] tokens of a sequence of
+    S = k.shape[0] tokens (chunked prefill; n = 1 is a decode step).
+
+    q [n,Hq,128] holds the queries of tokens S-n .. S-1; k/v [S,Hkv,128] the
+    keys and values of all S tokens. Returns (out [n,Hq,128] bf16,
+    lse [Hq,n] fp32), equal to those rows of ``fwd`` on the whole sequence.
+    """
+    _dev_bf16(q, "q"), _dev_bf16(k, "k"), _dev_bf16(v, "v")
+    n, Hq, d = q.shape
+    S, Hkv = k.shape[0], k.shape[1]
+    if v.shape != k.shape or k.shape[2] != d or not 1 <= n <= S:
+        raise ValueError("q must be [n, heads_q, head_dim] with 1 <= n <= S; k and v [S, heads_kv, head_dim]")
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((Hq, n), dtype=torch.float32, device=q.device)
+    _check(lib().moba_fwd_chunk(q.data_ptr(), k.data_ptr(), v.data_ptr(), S, S - n, Hq, Hkv, d, block_size, topk,
+                                out.data_ptr(), lse.data_ptr(), _stream(stream)))
     return out, lse
 
 

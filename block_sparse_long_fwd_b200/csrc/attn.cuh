@@ -54,7 +54,7 @@ constexpr uint32_t kNoHead = 0xFFFFu;
 constexpr uint32_t kNextTile = 0xFFFEu;  // own tile B: the next 128 tokens of tile A's head
 
 struct AttnParams {
-  const __nv_bfloat16* q;   // [S][Hq][128]
+  const __nv_bfloat16* q;   // [S - q0][Hq][128]: the tokens with a query
   const int32_t* list;      // group-rows of the window, per bucket
   const int4* units;        // unit descriptors
   int32_t* hdr;             // [1] = number of units, [3] = next-unit counter (starts at 0)
@@ -62,7 +62,7 @@ struct AttnParams {
   float* part_lse;          // [list entries]
   __half* own_o;            // [wlen][Hq][128], fp16
   float* own_lse;           // [wlen][Hq]
-  int64_t S, w0;
+  int64_t S, w0, q0;        // q0: first token with a query
   int Hq, G, B;
   float scale_log2;         // log2(e) / sqrt(128)
 };
@@ -360,7 +360,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         tc_fence_after();
         const float inv_l = 1.f / l_run;
         const float lse = (m_run + log2f(l_run)) * 0.69314718055994530942f;
-        const bool write = row < (X ? u.rows[1] : u.rows[0]);
+        const bool write = row < (X ? u.rows[1] : u.rows[0]) && (!u.own || (X ? u.tq[1] : u.tq[0]) + row >= p.q0);
         __half* dst_o;
         float* dst_lse;
         if (u.own) {
@@ -584,7 +584,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
               t = p.w0 + rr / p.G;
               h = u.g * p.G + rr % p.G;
             }
-            off[x][k] = (t * p.Hq + h) * kHeadDim;
+            // a token before q0 has no query: its row stays zero and is not written
+            if (t >= p.q0) off[x][k] = ((t - p.q0) * p.Hq + h) * kHeadDim;
           }
         }
       }

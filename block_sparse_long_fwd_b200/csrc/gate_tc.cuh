@@ -59,9 +59,9 @@ __global__ void __launch_bounds__(128) kmean_split_kernel(const float* __restric
 }
 
 struct GateParams {
-  const __nv_bfloat16* q;  // [S][Hq][128]
-  int32_t* sel;            // [Hq][S][k_eff]
-  int64_t S;
+  const __nv_bfloat16* q;  // [S - q0][Hq][128]: the tokens with a query
+  int32_t* sel;            // [Hq][S - q0][k_eff]
+  int64_t S, q0;           // q0: first token with a query
   int Hq, G, B, nbp_pad, k_eff;
 };
 
@@ -104,7 +104,7 @@ __device__ __forceinline__ void gate_write_row(int32_t* out, const int (&ti)[KP]
   for (int i = npast + 1; i < k_eff; ++i) out[i] = -1;
 }
 
-// grid (ceil(S*G / 128), Hkv), 128 threads; row = TMEM lane = group-row
+// grid (ceil((S - q0)*G / 128), Hkv), 128 threads; row = TMEM lane = group-row
 // blockIdx.x*128 + threadIdx.x.
 template <int KP>
 __global__ void __launch_bounds__(kGateTcThreads)
@@ -122,13 +122,14 @@ __global__ void __launch_bounds__(kGateTcThreads)
   const int g = blockIdx.y;
   const int warp = threadIdx.x >> 5;
   const int row = threadIdx.x;
-  const int64_t rr = (int64_t)blockIdx.x * 128 + row;
+  const int64_t rr0 = p.q0 * p.G + (int64_t)blockIdx.x * 128;  // this CTA's first group-row
+  const int64_t rr = rr0 + row;
   const int64_t t = rr / p.G;
   const int h = g * p.G + (int)(rr % p.G);
   const bool valid = t < p.S;
   const int bt = valid ? (int)(t / p.B) : 0;
   const int P = p.k_eff - 1;
-  int64_t t_last = ((int64_t)blockIdx.x * 128 + 127) / p.G;
+  int64_t t_last = (rr0 + 127) / p.G;
   if (t_last > p.S - 1) t_last = p.S - 1;
   const int b_cta = (int)(t_last / p.B);  // past blocks of this CTA: j < b_cta
   const int nchunks = (b_cta + kGateBlkChunk - 1) / kGateBlkChunk;
@@ -163,12 +164,12 @@ __global__ void __launch_bounds__(kGateTcThreads)
         const int idx = threadIdx.x + 128 * i;  // 2048 chunks of 16 B
         const int r = idx >> 4, c16 = idx & 15;
         const int half = c16 >> 3, c = c16 & 7;
-        const int64_t rr_r = (int64_t)blockIdx.x * 128 + r;
+        const int64_t rr_r = rr0 + r;
         const int64_t t_r = rr_r / p.G;
         const __nv_bfloat16* src = p.q;
         uint32_t bytes = 0;
         if (t_r < p.S) {
-          src = p.q + (t_r * p.Hq + g * p.G + (int)(rr_r % p.G)) * kHeadDim + c16 * 8;
+          src = p.q + ((t_r - p.q0) * p.Hq + g * p.G + (int)(rr_r % p.G)) * kHeadDim + c16 * 8;
           bytes = 16;
         }
         cp_async_16(dst0 + half * (kGateQBytes / 2) + r * 128 + ((c ^ (r & 7)) << 4), src, bytes);
@@ -300,20 +301,22 @@ __global__ void __launch_bounds__(kGateTcThreads)
   }
   if (!valid) return;
   const int npast = min(P, bt);
-  gate_write_row<KP>(p.sel + ((int64_t)h * p.S + t) * p.k_eff, ti, npast, bt, p.k_eff);
+  gate_write_row<KP>(p.sel + ((int64_t)h * (p.S - p.q0) + (t - p.q0)) * p.k_eff, ti, npast, bt, p.k_eff);
 }
 
 // Rows that need no scores: topk = 1 (own block only) or topk >= nblocks
-// (every past block). grid ceil(S*Hq / 256), 256 threads.
-__global__ void __launch_bounds__(256) sel_fill_kernel(int32_t* __restrict__ sel, int64_t S, int Hq, int B,
-                                                        int k_eff, int full) {
+// (every past block), for the tokens [q0, S). grid ceil((S - q0)*Hq / 256),
+// 256 threads.
+__global__ void __launch_bounds__(256) sel_fill_kernel(int32_t* __restrict__ sel, int64_t S, int64_t q0, int Hq,
+                                                        int B, int k_eff, int full) {
   grid_dependency_sync();
+  const int64_t n = S - q0;
   const int64_t i = (int64_t)blockIdx.x * 256 + threadIdx.x;
-  if (i >= S * Hq) return;
-  const int h = (int)(i / S);
-  const int64_t t = i % S;
+  if (i >= n * Hq) return;
+  const int h = (int)(i / n);
+  const int64_t t = q0 + i % n;
   const int bt = (int)(t / B);
-  int32_t* out = sel + ((int64_t)h * S + t) * k_eff;
+  int32_t* out = sel + ((int64_t)h * n + (t - q0)) * k_eff;
   if (full) {
     for (int j = 0; j < k_eff; ++j) out[j] = (j <= bt) ? j : -1;
   } else {

@@ -22,8 +22,8 @@ struct MergeParams {
   const float* part_lse;
   const __half* own_o;
   const float* own_lse;
-  __nv_bfloat16* out;  // [S][Hq][128]
-  float* lse;          // [Hq][S]
+  __nv_bfloat16* out;  // [S - q0][Hq][128]: rows of the tokens with a query
+  float* lse;          // [Hq][S - q0]
   WindowGeom w;
 };
 
@@ -56,12 +56,14 @@ __global__ void __launch_bounds__(256) merge_kernel(MergeParams m) {
   const int64_t tl = row / w.Hq;
   const int h = (int)(row % w.Hq);
   const int64_t t = w.w0 + tl;
+  if (t < w.q0) return;  // no query at this token (padding of a window's first tile)
+  const int64_t tq = t - w.q0, nq = w.S - w.q0;
   const int g = h / w.G, hl = h % w.G;
   const int bt = (int)(t / w.B);
   const int64_t rr = tl * w.G + hl;
   const int64_t word = rr >> 5;
   const uint32_t below = (1u << (rr & 31)) - 1u;
-  const int32_t* srow = m.sel + ((int64_t)h * w.S + t) * w.k_eff;
+  const int32_t* srow = m.sel + ((int64_t)h * nq + tq) * w.k_eff;
   const int P = w.k_eff - 1;
 
   // lane i resolves routed partial i (slot and lse) once
@@ -150,8 +152,8 @@ __global__ void __launch_bounds__(256) merge_kernel(MergeParams m) {
     acc.w += wk * o.w;
   }
   uint2 packed = make_uint2(pack_bf16x2(acc.x, acc.y), pack_bf16x2(acc.z, acc.w));
-  *reinterpret_cast<uint2*>(m.out + (t * w.Hq + h) * kHeadDim + lane * 4) = packed;
-  if (lane == 0) m.lse[(int64_t)h * w.S + t] = L;
+  *reinterpret_cast<uint2*>(m.out + (tq * w.Hq + h) * kHeadDim + lane * 4) = packed;
+  if (lane == 0) m.lse[(int64_t)h * nq + tq] = L;
 }
 
 }  // namespace moba

@@ -145,6 +145,8 @@ struct Carve {
 
 struct Plan {
   int64_t S;
+  int64_t q0 = 0;     // first token with a query (0: a whole prefill)
+  int64_t wbase = 0;  // first window start: q0 rounded down to 256 tokens
   int Hq, Hkv, G, B, topk, k_eff, P, nb, nbp;
   int splits = 1;  // pool row splits per block
   int64_t W;       // window tokens (multiple of 128)
@@ -188,7 +190,7 @@ bool pair_tokens(const Plan& p) { return p.G == 1 && (p.B / moba::kTile) % 2 == 
 
 // Scratch layout for a query window of W tokens.
 void layout_for_window(Plan& p, int64_t W) {
-  if (pair_tokens(p) && W < (p.S + 127) / 128 * 128) W = std::max<int64_t>(256, W / 256 * 256);
+  if (pair_tokens(p) && W < (p.S - p.wbase + 127) / 128 * 128) W = std::max<int64_t>(256, W / 256 * 256);
   p.W = W;
   p.wwords = (W * p.G + 31) / 32;
   const int64_t nbk = (int64_t)p.Hkv * p.nbp;
@@ -200,7 +202,7 @@ void layout_for_window(Plan& p, int64_t W) {
   const size_t nbk_pad = (size_t)p.Hkv * moba::gate_rows_padded(std::max(p.nbp, 1));
   p.o_khi = c.take(nbk_pad * moba::kHeadDim * 2);
   p.o_klo = c.take(nbk_pad * moba::kHeadDim * 2);
-  p.o_sel = c.take((size_t)p.Hq * p.S * p.k_eff * 4);
+  p.o_sel = c.take((size_t)p.Hq * (p.S - p.q0) * p.k_eff * 4);
   p.o_flags = c.take((size_t)nbk * p.wwords * 4);
   p.o_wordbase = c.take((size_t)nbk * p.wwords * 4);
   p.o_cnt = c.take((size_t)(nbk + 1) * 4);
@@ -231,9 +233,11 @@ void dense_blocks(Plan& p) {
   p.P = p.k_eff - 1;
 }
 
-int make_plan(Plan* pl, int64_t S, int Hq, int Hkv, int B, int topk) {
+int make_plan(Plan* pl, int64_t S, int64_t q0, int Hq, int Hkv, int B, int topk) {
   Plan& p = *pl;
   p.S = S;
+  p.q0 = q0;
+  p.wbase = q0 / 256 * 256;
   p.Hq = Hq;
   p.Hkv = Hkv;
   p.G = Hq / Hkv;
@@ -244,7 +248,7 @@ int make_plan(Plan* pl, int64_t S, int Hq, int Hkv, int B, int topk) {
   p.k_eff = std::min(topk, p.nb);
   p.P = p.k_eff - 1;
   dense_blocks(p);
-  const int64_t S128 = (S + 127) / 128 * 128;
+  const int64_t S128 = (S - p.wbase + 127) / 128 * 128;  // tokens the windows cover
   int64_t W = 0;
   if (const char* env = getenv("MOBA_WINDOW")) {
     W = atoll(env);
@@ -299,7 +303,7 @@ void launch_chained(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem
 template <int KP>
 void launch_gate_tc(const Plan& p, const CUtensorMap& mhi, const CUtensorMap& mlo, const moba::GateParams& gp,
                     cudaStream_t st) {
-  dim3 grid((unsigned)((p.S * p.G + 127) / 128), p.Hkv);
+  dim3 grid((unsigned)(((p.S - p.q0) * p.G + 127) / 128), p.Hkv);
   launch_chained(moba::gate_tc_kernel<KP>, grid, dim3(moba::kGateTcThreads), moba::kGateSmemBytes, st, mhi, mlo, gp);
 }
 
@@ -310,9 +314,9 @@ int launch_gate(const Plan& p, const void* q, const float* kmean, int splits, __
                 __nv_bfloat16* klo, int32_t* sel, cudaStream_t st) {
   const bool full = p.k_eff == p.nb;
   if (p.P == 0 || full || p.nbp <= 0) {
-    const int64_t n = p.S * p.Hq;
-    launch_chained(moba::sel_fill_kernel, dim3((unsigned)((n + 255) / 256)), dim3(256), 0, st, sel, p.S, p.Hq, p.B,
-                   p.k_eff, full ? 1 : 0);
+    const int64_t n = (p.S - p.q0) * p.Hq;
+    launch_chained(moba::sel_fill_kernel, dim3((unsigned)((n + 255) / 256)), dim3(256), 0, st, sel, p.S, p.q0, p.Hq,
+                   p.B, p.k_eff, full ? 1 : 0);
     return 1;
   }
   const int nbp_pad = moba::gate_rows_padded(p.nbp);
@@ -327,6 +331,7 @@ int launch_gate(const Plan& p, const void* q, const float* kmean, int splits, __
   gp.q = static_cast<const __nv_bfloat16*>(q);
   gp.sel = sel;
   gp.S = p.S;
+  gp.q0 = p.q0;
   gp.Hq = p.Hq;
   gp.G = p.G;
   gp.B = p.B;
@@ -444,12 +449,13 @@ int run_forward(const Plan& p, const DeviceInfo& dev, const void* q, const void*
   ap.own_o = own_o;
   ap.own_lse = own_lse;
   ap.S = p.S;
+  ap.q0 = p.q0;
   ap.Hq = p.Hq;
   ap.G = p.G;
   ap.B = p.B;
   ap.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)moba::kHeadDim));
 
-  for (int64_t w0 = 0; w0 < p.S; w0 += p.W) {
+  for (int64_t w0 = p.wbase; w0 < p.S; w0 += p.W) {
     moba::WindowGeom wg;
     wg.S = p.S;
     wg.Hq = p.Hq;
@@ -460,6 +466,7 @@ int run_forward(const Plan& p, const DeviceInfo& dev, const void* q, const void*
     wg.nbp = p.nbp;
     wg.w0 = w0;
     wg.wlen = std::min(p.W, p.S - w0);
+    wg.q0 = p.q0;
     wg.wwords = (wg.wlen * p.G + 31) / 32;
     wg.pair_tokens = pair_tokens(p) ? 1 : 0;
     const bool routed = p.P > 0 && p.nbp > 0 && (w0 + wg.wlen) > p.B;
@@ -538,11 +545,11 @@ struct GraphKey {
   const void *q, *k, *v;
   void* out;
   float* lse;
-  int64_t S, W;
+  int64_t S, q0, W;
   int Hq, Hkv, B, topk;
   bool operator==(const GraphKey& o) const {
-    return dev == o.dev && q == o.q && k == o.k && v == o.v && out == o.out && lse == o.lse && S == o.S && W == o.W &&
-           Hq == o.Hq && Hkv == o.Hkv && B == o.B && topk == o.topk;
+    return dev == o.dev && q == o.q && k == o.k && v == o.v && out == o.out && lse == o.lse && S == o.S &&
+           q0 == o.q0 && W == o.W && Hq == o.Hq && Hkv == o.Hkv && B == o.B && topk == o.topk;
   }
 };
 
@@ -569,7 +576,7 @@ int graph_forward(const Plan& p, const DeviceInfo& dev, const void* q, const voi
   if (!graphs_enabled()) return -1;
   int d = 0;
   if (cudaGetDevice(&d) != cudaSuccess || d < 0 || d >= 64) return -1;
-  GraphKey key{d, q, k, v, out, lse, p.S, p.W, p.Hq, p.Hkv, p.B, p.topk};
+  GraphKey key{d, q, k, v, out, lse, p.S, p.q0, p.W, p.Hq, p.Hkv, p.B, p.topk};
   std::lock_guard<std::mutex> lk(g_graph_mu);
   GraphEntry* hit = nullptr;
   for (GraphEntry& en : g_graphs)
@@ -624,19 +631,22 @@ int graph_forward(const Plan& p, const DeviceInfo& dev, const void* q, const voi
   return MOBA_OK;
 }
 
-int fwd_impl(const void* q, const void* k, const void* v, int64_t seqlen, int heads_q, int heads_kv, int head_dim,
-             int block_size, int topk, void* out, float* lse, cudaStream_t stream, bool use_graph) {
+int fwd_impl(const void* q, const void* k, const void* v, int64_t seqlen, int64_t q_start, int heads_q, int heads_kv,
+             int head_dim, int block_size, int topk, void* out, float* lse, cudaStream_t stream, bool use_graph) {
   g_err.clear();
   if (!q || !k || !v || !out || !lse) return fail(MOBA_ERR_INVALID_ARG, "null pointer argument");
   int rc = check_shape(seqlen, heads_q, heads_kv, head_dim, block_size, topk);
   if (rc) return rc;
+  if (q_start < 0 || q_start >= seqlen)
+    return fail(MOBA_ERR_INVALID_ARG, "q_start must be in [0, seqlen) (got %lld, seqlen %lld)", (long long)q_start,
+                (long long)seqlen);
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(lse))
     return fail(MOBA_ERR_INVALID_ARG, "device buffers must be 16-byte aligned");
   DeviceInfo dev;
   rc = device_info(&dev);
   if (rc) return rc;
   Plan p;
-  rc = make_plan(&p, seqlen, heads_q, heads_kv, block_size, topk);
+  rc = make_plan(&p, seqlen, q_start, heads_q, heads_kv, block_size, topk);
   if (rc) return rc;
   if (use_graph && !g_timer.on) {
     const int g = graph_forward(p, dev, q, k, v, out, lse, stream);
@@ -651,7 +661,12 @@ extern "C" {
 
 int moba_fwd(const void* q, const void* k, const void* v, int64_t seqlen, int heads_q, int heads_kv, int head_dim,
              int block_size, int topk, void* out, float* lse, cudaStream_t stream) {
-  return fwd_impl(q, k, v, seqlen, heads_q, heads_kv, head_dim, block_size, topk, out, lse, stream, true);
+  return fwd_impl(q, k, v, seqlen, 0, heads_q, heads_kv, head_dim, block_size, topk, out, lse, stream, true);
+}
+
+int moba_fwd_chunk(const void* q, const void* k, const void* v, int64_t seqlen, int64_t q_start, int heads_q,
+                   int heads_kv, int head_dim, int block_size, int topk, void* out, float* lse, cudaStream_t stream) {
+  return fwd_impl(q, k, v, seqlen, q_start, heads_q, heads_kv, head_dim, block_size, topk, out, lse, stream, true);
 }
 
 int moba_profile_begin(void) {
@@ -700,7 +715,7 @@ int moba_fwd_host(const void* q_host, const void* k_host, const void* v_host, in
       cudaMemcpyAsync(b + ov, v_host, kb, cudaMemcpyHostToDevice, stream) != cudaSuccess)
     rc = fail(MOBA_ERR_CUDA, "host to device copy failed: %s", cudaGetErrorString(cudaGetLastError()));
   if (!rc)
-    rc = fwd_impl(b + oq, b + ok, b + ov, seqlen, heads_q, heads_kv, head_dim, block_size, topk, b + oo,
+    rc = fwd_impl(b + oq, b + ok, b + ov, seqlen, 0, heads_q, heads_kv, head_dim, block_size, topk, b + oo,
                   reinterpret_cast<float*>(b + ol), stream, false);
   if (!rc && (cudaMemcpyAsync(out_host, b + oo, qb, cudaMemcpyDeviceToHost, stream) != cudaSuccess ||
               cudaMemcpyAsync(lse_host, b + ol, lb, cudaMemcpyDeviceToHost, stream) != cudaSuccess))

@@ -31,6 +31,7 @@ struct WindowGeom {
   int64_t w0, wlen;  // window start token and length
   int64_t wwords;    // flag words per bucket: ceil(wlen * G / 32)
   int pair_tokens;   // own units pair consecutive 128-token tiles of one head
+  int64_t q0;        // first token with a query (0 for a whole prefill); sel rows start there
 };
 
 // First flag word of bucket j that can hold a set bit: rows with t >= (j+1)B.
@@ -51,13 +52,17 @@ __global__ void __launch_bounds__(256) route_flags_kernel(const int32_t* __restr
   if (word >= w.wwords) return;
   const int64_t rr = word * 32 + lane;
   const int64_t tl = rr / w.G;
-  const bool valid = tl < w.wlen;
   const int64_t t = w.w0 + tl;
+  const bool in_window = tl < w.wlen;
+  const bool valid = in_window && t >= w.q0;  // a token before q0 has no query: no bits
   const int h = g * w.G + (int)(rr % w.G);
-  const int bt = valid ? (int)(t / w.B) : 0;
+  // every word writes its bits for all blocks below its rows' own blocks
+  // (zeros for rows without a query), since the count and fill kernels read
+  // every word from the first one that can hold a bit of the block
+  const int bt = in_window ? (int)(t / w.B) : 0;
   const int bmax = __reduce_max_sync(0xffffffffu, bt);
   const int P = w.k_eff - 1;
-  const int32_t* srow = sel + ((int64_t)h * w.S + t) * w.k_eff;
+  const int32_t* srow = sel + ((int64_t)h * (w.S - w.q0) + (valid ? t - w.q0 : 0)) * w.k_eff;
   int ptr = 0;
   auto entry = [&](int i) -> int {
     if (!valid || i >= P) return 0x7fffffff;

@@ -92,6 +92,34 @@ int moba_fwd(const void* q, const void* k, const void* v, int64_t seqlen,
              void* out, float* lse, cudaStream_t stream);
 
 /*
+ * moba_fwd_chunk - the forward pass for the queries of the last
+ * seqlen - q_start tokens only, against keys and values of all seqlen
+ * tokens: a chunk of prefill (or, with q_start = seqlen - 1, one decode step)
+ * appended to a cache. By causality the result equals rows q_start..seqlen-1
+ * of moba_fwd on the whole sequence (the queries of earlier tokens never
+ * enter them); the pages' causal gate and own-block mask ("MoBA - Moonshot
+ * AIが提案した新しいアテンションメカニズム", "MoBAの技術的原則") are applied
+ * at the tokens' absolute positions. The pages describe no such entry point;
+ * it serves the serving use they mention (Kimi's long-context requests).
+ *
+ * q          device bf16 [seqlen - q_start][heads_q][head_dim]: the queries
+ *            of tokens q_start .. seqlen - 1.
+ * k, v       device bf16 [seqlen][heads_kv][head_dim]: every token's keys and
+ *            values (the cache followed by the chunk's own).
+ * q_start    first token with a query, 0 <= q_start < seqlen (0 is moba_fwd).
+ * out        device bf16 [seqlen - q_start][heads_q][head_dim].
+ * lse        device fp32 [heads_q][seqlen - q_start].
+ * Other arguments, ownership and errors as moba_fwd; a q_start outside
+ * [0, seqlen) returns MOBA_ERR_INVALID_ARG. Each call pools the means of all
+ * complete blocks again (they do not change while the cache grows inside the
+ * last block; a caller may not keep them across calls).
+ */
+int moba_fwd_chunk(const void* q, const void* k, const void* v, int64_t seqlen,
+                   int64_t q_start, int heads_q, int heads_kv, int head_dim,
+                   int block_size, int topk, void* out, float* lse,
+                   cudaStream_t stream);
+
+/*
  * moba_fwd_host - moba_fwd on HOST buffers (same layouts): copies q, k, v to
  * the device, runs the forward pass and copies out and lse back, all on
  * `stream`, and synchronises the stream before returning. Host buffers that

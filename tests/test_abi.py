@@ -80,3 +80,10 @@ def test_effective_flops_counts_selected_pairs():
     S, B, k = 6, 2, 2
     pairs = sum(min(k - 1, t // B) * B + t % B + 1 for t in range(S))
     assert moba.effective_flops(S, 1, B, k, head_dim=1) == 4 * pairs
+
+
+@pytest.mark.parametrize("q_start", [-1, 4096, 5000])
+def test_chunk_rejects_a_query_start_outside_the_sequence(lib, q_start):
+    rc = lib.moba_fwd_chunk(FAKE, FAKE, FAKE, 4096, q_start, 1, 1, 128, 512, 3, FAKE, FAKE, None)
+    assert rc == moba.MOBA_ERR_INVALID_ARG
+    assert "q_start" in moba.last_error()
