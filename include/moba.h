@@ -111,8 +111,7 @@ int moba_fwd(const void* q, const void* k, const void* v, int64_t seqlen,
  * lse        device fp32 [heads_q][seqlen - q_start].
  * Other arguments, ownership and errors as moba_fwd; a q_start outside
  * [0, seqlen) returns MOBA_ERR_INVALID_ARG. Each call pools the means of all
- * complete blocks again (they do not change while the cache grows inside the
- * last block; a caller may not keep them across calls).
+ * complete blocks again: the library keeps nothing between calls.
  */
 int moba_fwd_chunk(const void* q, const void* k, const void* v, int64_t seqlen,
                    int64_t q_start, int heads_q, int heads_kv, int head_dim,
