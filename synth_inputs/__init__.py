@@ -57,6 +57,9 @@ WORKLOADS = {
     # inputs of the 32K and 128K workloads
     "32k_dense": Workload("moba_32k_h1_b2048_k16_dense", 32768, 1, 1, 128, 2048, 16, 20250218 + 1),
     "128k_dense": Workload("moba_128k_h32kv8_b4096_k32_dense", 131072, 32, 8, 128, 4096, 32, 20250218 + 2),
+    # finer blocks: 512-token blocks, top-48 (about the 128K workload's
+    # selected keys per query), on the 128K workload's seed
+    "128k_b512": Workload("moba_128k_h32kv8_b512_k48", 131072, 32, 8, 128, 512, 48, 20250218 + 2),
 }
 
 

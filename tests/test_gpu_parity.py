@@ -93,10 +93,11 @@ def test_large_workload_sampled_rows(name, nrows):
     print(name, stats)
 
 
-@pytest.mark.parametrize("name,nrows", [("32k_dense", 512), ("128k_dense", 128)])
+@pytest.mark.parametrize("name,nrows", [("32k_dense", 512), ("128k_dense", 128), ("128k_b512", 256)])
 def test_dense_workload_sampled_rows(name, nrows):
     # topk >= number of blocks is full causal attention; the library runs it
-    # as one causal pass (no gate scores, no routing) and must match the oracle
+    # as one causal pass (no gate scores, no routing) and must match the
+    # oracle. 128k_b512: finer blocks (512 tokens, top-48) through the same path
     w = si.WORKLOADS[name]
     q, k, v = si.make_qkv(w)
     rows = sample_rows(w, nrows, w.seed + 2000)
