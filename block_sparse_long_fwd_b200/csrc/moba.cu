@@ -76,6 +76,10 @@ int device_info(DeviceInfo* out) {
                                      moba::kGateSmemBytes));
       MOBA_CUDA(cudaFuncSetAttribute(moba::gate_tc_kernel<16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      moba::kGateSmemBytes));
+      MOBA_CUDA(cudaFuncSetAttribute(moba::gate_tc_kernel<24>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     moba::kGateSmemBytes));
+      MOBA_CUDA(cudaFuncSetAttribute(moba::gate_tc_kernel<48>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     moba::kGateSmemBytes));
       MOBA_CUDA(cudaFuncSetAttribute(moba::gate_tc_kernel<32>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      moba::kGateSmemBytes));
       MOBA_CUDA(cudaFuncSetAttribute(moba::gate_tc_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -342,7 +346,9 @@ int launch_gate(const Plan& p, const void* q, const float* kmean, int splits, __
   else if (p.P <= 8) launch_gate_tc<8>(p, mhi, mlo, gp, st);
   else if (p.P <= 12) launch_gate_tc<12>(p, mhi, mlo, gp, st);
   else if (p.P <= 16) launch_gate_tc<16>(p, mhi, mlo, gp, st);
+  else if (p.P <= 24) launch_gate_tc<24>(p, mhi, mlo, gp, st);
   else if (p.P <= 32) launch_gate_tc<32>(p, mhi, mlo, gp, st);
+  else if (p.P <= 48) launch_gate_tc<48>(p, mhi, mlo, gp, st);
   else launch_gate_tc<64>(p, mhi, mlo, gp, st);
   return 2;
 }

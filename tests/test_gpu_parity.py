@@ -36,6 +36,8 @@ SMALL = [
     (2900,  2,  2,   512, 3,    11),    # paired own tiles, last pair without its second tile
     (4096,  1,  1,   512, 8,    12),    # topk >= blocks, one head: the dense path, paired own tiles
     (3000,  4,  2,   256, 64,   13),    # dense path, GQA, ragged
+    (8192,  2,  1,   128, 20,   14),    # 19 past blocks kept per row (24-entry top-k lists)
+    (12000, 2,  1,   128, 40,   15),    # 39 past blocks kept per row (48-entry lists), ragged
 ]
 
 
