@@ -46,7 +46,15 @@ __device__ __forceinline__ float warp_sum(float v) {
 }
 
 // grid ceil(wlen * Hq / 8), 256 threads: one warp per (token, q head) row,
-// lane c owns channels 4c..4c+3.
+// lane c owns channels 4c..4c+3. With NP > 0 and at most NP routed partials
+// per row, every partial row is loaded as soon as its slot is known, before
+// the weights (which wait for the partials' lse) are formed: the row then
+// costs three dependent memory round trips (selection, flag words, partials)
+// instead of four. It pays off for a few partials per row (small, latency
+// bound problems); with many, the registers it holds cost more occupancy
+// than it gains (measured: 1M workload merge 35 -> 39 ms with NP = 12), so
+// the host uses it for up to 4. The sums run in the same order either way.
+template <int NP>
 __global__ void __launch_bounds__(256) merge_kernel(MergeParams m) {
   grid_dependency_sync();
   const WindowGeom& w = m.w;
@@ -79,9 +87,31 @@ __global__ void __launch_bounds__(256) merge_kernel(MergeParams m) {
   };
 
   const float own_l = m.own_lse[tl * w.Hq + h];
+  const float4 own_v = load_half4(m.own_o + (tl * w.Hq + h) * kHeadDim + lane * 4);
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
   float L;
-  if (P <= 32) {
+  if (NP > 0 && P <= NP) {
+    float li;
+    const int64_t pos = slot(lane, li);
+    float4 o[NP > 0 ? NP : 1];
+#pragma unroll
+    for (int k = 0; k < NP; ++k) {
+      const int64_t pk = __shfl_sync(0xffffffffu, pos, k);
+      o[k] = (k < P && pk >= 0) ? load_half4(m.part_o + pk * kHeadDim + lane * 4) : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+    const float mx = fmaxf(own_l, warp_max(li));
+    const float sum = warp_sum(li == -INFINITY ? 0.f : expf(li - mx)) + expf(own_l - mx);
+    L = mx + logf(sum);
+    const float wl = li == -INFINITY ? 0.f : expf(li - L);  // lane i's weight (0 past P)
+#pragma unroll
+    for (int k = 0; k < NP; ++k) {
+      const float wk = __shfl_sync(0xffffffffu, wl, k);
+      acc.x += wk * o[k].x;
+      acc.y += wk * o[k].y;
+      acc.z += wk * o[k].z;
+      acc.w += wk * o[k].w;
+    }
+  } else if (P <= 32) {
     float li;
     const int64_t pos = slot(lane, li);
     const float mx = fmaxf(own_l, warp_max(li));
@@ -145,11 +175,10 @@ __global__ void __launch_bounds__(256) merge_kernel(MergeParams m) {
   }
   {
     const float wk = expf(own_l - L);
-    const float4 o = load_half4(m.own_o + (tl * w.Hq + h) * kHeadDim + lane * 4);
-    acc.x += wk * o.x;
-    acc.y += wk * o.y;
-    acc.z += wk * o.z;
-    acc.w += wk * o.w;
+    acc.x += wk * own_v.x;
+    acc.y += wk * own_v.y;
+    acc.z += wk * own_v.z;
+    acc.w += wk * own_v.w;
   }
   uint2 packed = make_uint2(pack_bf16x2(acc.x, acc.y), pack_bf16x2(acc.z, acc.w));
   *reinterpret_cast<uint2*>(m.out + (tq * w.Hq + h) * kHeadDim + lane * 4) = packed;

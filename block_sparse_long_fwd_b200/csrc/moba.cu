@@ -510,7 +510,10 @@ int run_forward(const Plan& p, const DeviceInfo& dev, const void* q, const void*
     mp.lse = lse;
     mp.w = wg;
     const int64_t rows = wg.wlen * p.Hq;
-    launch_chained(moba::merge_kernel, dim3((unsigned)((rows + 7) / 8)), dim3(256), 0, st, mp);
+    const dim3 mg((unsigned)((rows + 7) / 8));
+    if (p.P <= 2) launch_chained(moba::merge_kernel<2>, mg, dim3(256), 0, st, mp);
+    else if (p.P <= 4) launch_chained(moba::merge_kernel<4>, mg, dim3(256), 0, st, mp);
+    else launch_chained(moba::merge_kernel<0>, mg, dim3(256), 0, st, mp);
     tm->count(1);
     tm->mark(kMerge);
   }
