@@ -87,7 +87,9 @@ __global__ void __launch_bounds__(256) merge_kernel(MergeParams m) {
   };
 
   const float own_l = m.own_lse[tl * w.Hq + h];
-  const float4 own_v = load_half4(m.own_o + (tl * w.Hq + h) * kHeadDim + lane * 4);
+  const __half* own_row = m.own_o + (tl * w.Hq + h) * kHeadDim + lane * 4;
+  float4 own_v = make_float4(0.f, 0.f, 0.f, 0.f);
+  if (NP > 0) own_v = load_half4(own_row);  // early only where registers are cheap
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
   float L;
   if (NP > 0 && P <= NP) {
@@ -174,6 +176,7 @@ __global__ void __launch_bounds__(256) merge_kernel(MergeParams m) {
     }
   }
   {
+    if (NP == 0) own_v = load_half4(own_row);
     const float wk = expf(own_l - L);
     acc.x += wk * own_v.x;
     acc.y += wk * own_v.y;
