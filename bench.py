@@ -264,23 +264,26 @@ def run_chunk(args, w):
     lse = torch.empty((Hq, n), dtype=torch.float32, device=dev)
     flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream()
+    # --cached-means: block means pooled once, outside the timed steps (a
+    # decode loop pools again only when the cache completes a block)
+    kmean = moba.pool(k, w.block_size) if args.cached_means else None
     for _ in range(args.warmup):
         flush.zero_()
-        moba.fwd_chunk(qc, k, v, w.block_size, w.topk, out=out, lse=lse)
+        moba.fwd_chunk(qc, k, v, w.block_size, w.topk, out=out, lse=lse, kmean=kmean)
     sampler = ClockSampler(None)
     torch.cuda.synchronize()
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
     for a, b in ev:
         flush.zero_()
         a.record(stream)
-        moba.fwd_chunk(qc, k, v, w.block_size, w.topk, out=out, lse=lse)
+        moba.fwd_chunk(qc, k, v, w.block_size, w.topk, out=out, lse=lse, kmean=kmean)
         b.record(stream)
     torch.cuda.synchronize()
     total_ms = sum(a.elapsed_time(b) for a, b in ev)
     moba.profile_begin()
     for _ in range(args.steps):
         flush.zero_()
-        moba.fwd_chunk(qc, k, v, w.block_size, w.topk, out=out, lse=lse)
+        moba.fwd_chunk(qc, k, v, w.block_size, w.topk, out=out, lse=lse, kmean=kmean)
     stages, launches, calls = moba.profile_end()
     torch.cuda.synchronize()
     clocks = sampler.stop()
@@ -296,7 +299,7 @@ def run_chunk(args, w):
         qc.copy_(q_h[q0:], non_blocking=True)
         k[q0:].copy_(k_h[q0:], non_blocking=True)
         v[q0:].copy_(v_h[q0:], non_blocking=True)
-        moba.fwd_chunk(qc, k, v, w.block_size, w.topk, out=out, lse=lse)
+        moba.fwd_chunk(qc, k, v, w.block_size, w.topk, out=out, lse=lse, kmean=kmean)
         out_h.copy_(out, non_blocking=True)
         lse_h.copy_(lse, non_blocking=True)
         torch.cuda.synchronize()
@@ -309,7 +312,8 @@ def run_chunk(args, w):
         "metric": METRIC, "value": n * args.steps / (total_ms / 1e3), "unit": "tokens/s", "n_gpus": 1,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": dict(workload_config(w, 1), mode="decode" if n == 1 else "chunked prefill", q_start=q0, chunk=n),
+        "config": dict(workload_config(w, 1), mode="decode" if n == 1 else "chunked prefill", q_start=q0, chunk=n,
+                       block_means="cached (pooled once)" if args.cached_means else "pooled every call"),
         "eff_tflops": flops * args.steps / (total_ms / 1e3) / 1e12,
         "stage_ms_per_step": {kk: vv / max(calls, 1) for kk, vv in stages.items()},
         "roofline": {"bound": "tensor", "kernel": "attn_kernel", "achieved": achieved,
@@ -503,6 +507,8 @@ def main():
     ap.add_argument("--no-pad", action="store_true", help="no untimed load after the timed steps (profiling)")
     ap.add_argument("--chunk", type=int, default=0,
                     help="time only the last N tokens' queries against the whole cache (1 = one decode step)")
+    ap.add_argument("--cached-means", action="store_true",
+                    help="with --chunk: pool the block means once instead of on every call")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

@@ -33,6 +33,7 @@ _vp, _i64, _i32 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int
 SIGNATURES = {
     "moba_fwd": (_i32, [_vp, _vp, _vp, _i64, _i32, _i32, _i32, _i32, _i32, _vp, _vp, _vp]),
     "moba_fwd_chunk": (_i32, [_vp, _vp, _vp, _i64, _i64, _i32, _i32, _i32, _i32, _i32, _vp, _vp, _vp]),
+    "moba_fwd_chunk_means": (_i32, [_vp, _vp, _vp, _vp, _i64, _i64, _i32, _i32, _i32, _i32, _i32, _vp, _vp, _vp]),
     "moba_fwd_host": (_i32, [_vp, _vp, _vp, _i64, _i32, _i32, _i32, _i32, _i32, _vp, _vp, _vp]),
     "moba_pool": (_i32, [_vp, _i64, _i32, _i32, _i32, _vp, _vp]),
     "moba_gate": (_i32, [_vp, _vp, _i64, _i32, _i32, _i32, _i32, _i32, _vp, _vp]),
@@ -115,7 +116,7 @@ def fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, block_size: int, topk
 
 
 def fwd_chunk(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, block_size: int, topk: int, out=None, lse=None,
-              stream=None):
+              stream=None, kmean=None):
     """MoBA forward for the last n = q.shape[0] tokens of a sequence of
     S = k.shape[0] tokens (chunked prefill; n = 1 is a decode step).
 
@@ -132,6 +133,13 @@ def fwd_chunk(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, block_size: int
         out = torch.empty_like(q)
     if lse is None:
         lse = torch.empty((Hq, n), dtype=torch.float32, device=q.device)
+    if kmean is not None:
+        # block means from pool() for these k and block_size, kept by the caller
+        if kmean.dtype != torch.float32 or not kmean.is_cuda or not kmean.is_contiguous():
+            raise ValueError("kmean must be a contiguous fp32 CUDA tensor from pool()")
+        _check(lib().moba_fwd_chunk_means(q.data_ptr(), k.data_ptr(), v.data_ptr(), kmean.data_ptr(), S, S - n, Hq,
+                                          Hkv, d, block_size, topk, out.data_ptr(), lse.data_ptr(), _stream(stream)))
+        return out, lse
     _check(lib().moba_fwd_chunk(q.data_ptr(), k.data_ptr(), v.data_ptr(), S, S - n, Hq, Hkv, d, block_size, topk,
                                 out.data_ptr(), lse.data_ptr(), _stream(stream)))
     return out, lse

@@ -150,6 +150,7 @@ struct Carve {
 struct Plan {
   int64_t S;
   int64_t q0 = 0;     // first token with a query (0: a whole prefill)
+  const float* means = nullptr;  // caller's block means [Hkv][nbp][128] (then no pooling)
   int64_t wbase = 0;  // first window start: q0 rounded down to 256 tokens
   int Hq, Hkv, G, B, topk, k_eff, P, nb, nbp;
   int splits = 1;  // pool row splits per block
@@ -409,7 +410,8 @@ int run_forward(const Plan& p, const DeviceInfo& dev, const void* q, const void*
   StageTimer* tm = &g_timer;
   tm->st = st;
   if (tm->on) tm->calls++;
-  float* kmean = reinterpret_cast<float*>(ws + p.o_kmean);
+  float* kmean = p.means ? const_cast<float*>(p.means) : reinterpret_cast<float*>(ws + p.o_kmean);
+  const int mean_splits = p.means ? 1 : p.splits;
   int32_t* sel = reinterpret_cast<int32_t*>(ws + p.o_sel);
   uint32_t* flags = reinterpret_cast<uint32_t*>(ws + p.o_flags);
   int32_t* wordbase = reinterpret_cast<int32_t*>(ws + p.o_wordbase);
@@ -431,13 +433,13 @@ int run_forward(const Plan& p, const DeviceInfo& dev, const void* q, const void*
   if (rc) return rc;
 
   tm->mark(-1);
-  if (p.P > 0 && p.k_eff < p.nb && p.nbp > 0) {
+  if (p.P > 0 && p.k_eff < p.nb && p.nbp > 0 && !p.means) {
     launch_pool(p, k, kmean, p.splits, st);
     tm->count(1);
     tm->mark(kPool);
   }
   {
-    const int n = launch_gate(p, q, kmean, p.splits, reinterpret_cast<__nv_bfloat16*>(ws + p.o_khi),
+    const int n = launch_gate(p, q, kmean, mean_splits, reinterpret_cast<__nv_bfloat16*>(ws + p.o_khi),
                               reinterpret_cast<__nv_bfloat16*>(ws + p.o_klo), sel, st);
     if (n < 0) return -n;
     tm->count(n);
@@ -554,10 +556,12 @@ struct GraphKey {
   const void *q, *k, *v;
   void* out;
   float* lse;
+  const float* means;
   int64_t S, q0, W;
   int Hq, Hkv, B, topk;
   bool operator==(const GraphKey& o) const {
-    return dev == o.dev && q == o.q && k == o.k && v == o.v && out == o.out && lse == o.lse && S == o.S &&
+    return dev == o.dev && q == o.q && k == o.k && v == o.v && out == o.out && lse == o.lse && means == o.means &&
+           S == o.S &&
            q0 == o.q0 && W == o.W && Hq == o.Hq && Hkv == o.Hkv && B == o.B && topk == o.topk;
   }
 };
@@ -585,7 +589,7 @@ int graph_forward(const Plan& p, const DeviceInfo& dev, const void* q, const voi
   if (!graphs_enabled()) return -1;
   int d = 0;
   if (cudaGetDevice(&d) != cudaSuccess || d < 0 || d >= 64) return -1;
-  GraphKey key{d, q, k, v, out, lse, p.S, p.q0, p.W, p.Hq, p.Hkv, p.B, p.topk};
+  GraphKey key{d, q, k, v, out, lse, p.means, p.S, p.q0, p.W, p.Hq, p.Hkv, p.B, p.topk};
   std::lock_guard<std::mutex> lk(g_graph_mu);
   GraphEntry* hit = nullptr;
   for (GraphEntry& en : g_graphs)
@@ -641,7 +645,8 @@ int graph_forward(const Plan& p, const DeviceInfo& dev, const void* q, const voi
 }
 
 int fwd_impl(const void* q, const void* k, const void* v, int64_t seqlen, int64_t q_start, int heads_q, int heads_kv,
-             int head_dim, int block_size, int topk, void* out, float* lse, cudaStream_t stream, bool use_graph) {
+             int head_dim, int block_size, int topk, void* out, float* lse, cudaStream_t stream, bool use_graph,
+             const float* means = nullptr) {
   g_err.clear();
   if (!q || !k || !v || !out || !lse) return fail(MOBA_ERR_INVALID_ARG, "null pointer argument");
   int rc = check_shape(seqlen, heads_q, heads_kv, head_dim, block_size, topk);
@@ -657,6 +662,8 @@ int fwd_impl(const void* q, const void* k, const void* v, int64_t seqlen, int64_
   Plan p;
   rc = make_plan(&p, seqlen, q_start, heads_q, heads_kv, block_size, topk);
   if (rc) return rc;
+  if (means && !aligned16(means)) return fail(MOBA_ERR_INVALID_ARG, "kmean must be 16-byte aligned");
+  p.means = means;
   if (use_graph && !g_timer.on) {
     const int g = graph_forward(p, dev, q, k, v, out, lse, stream);
     if (g >= 0) return g;  // negative: no graph for this call, launch directly
@@ -676,6 +683,14 @@ int moba_fwd(const void* q, const void* k, const void* v, int64_t seqlen, int he
 int moba_fwd_chunk(const void* q, const void* k, const void* v, int64_t seqlen, int64_t q_start, int heads_q,
                    int heads_kv, int head_dim, int block_size, int topk, void* out, float* lse, cudaStream_t stream) {
   return fwd_impl(q, k, v, seqlen, q_start, heads_q, heads_kv, head_dim, block_size, topk, out, lse, stream, true);
+}
+
+int moba_fwd_chunk_means(const void* q, const void* k, const void* v, const float* kmean, int64_t seqlen,
+                         int64_t q_start, int heads_q, int heads_kv, int head_dim, int block_size, int topk, void* out,
+                         float* lse, cudaStream_t stream) {
+  if (!kmean) return fail(MOBA_ERR_INVALID_ARG, "null pointer argument (kmean)");
+  return fwd_impl(q, k, v, seqlen, q_start, heads_q, heads_kv, head_dim, block_size, topk, out, lse, stream, true,
+                  kmean);
 }
 
 int moba_profile_begin(void) {

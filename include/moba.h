@@ -119,6 +119,25 @@ int moba_fwd_chunk(const void* q, const void* k, const void* v, int64_t seqlen,
                    cudaStream_t stream);
 
 /*
+ * moba_fwd_chunk_means - moba_fwd_chunk with the block means supplied by the
+ * caller instead of pooled from k on every call: a decode loop computes them
+ * once with moba_pool and pools again only when the cache completes a block.
+ *
+ * kmean      device fp32 [heads_kv][nblocks - 1][head_dim], exactly what
+ *            moba_pool writes for these k and block_size (nblocks =
+ *            ceil(seqlen / block_size)); means of blocks that cannot be past
+ *            blocks of any token are not read. The caller keeps it matching k;
+ *            a stale kmean silently changes the gate's choices. NULL returns
+ *            MOBA_ERR_INVALID_ARG.
+ * Other arguments, ownership and errors as moba_fwd_chunk.
+ */
+int moba_fwd_chunk_means(const void* q, const void* k, const void* v,
+                         const float* kmean, int64_t seqlen, int64_t q_start,
+                         int heads_q, int heads_kv, int head_dim,
+                         int block_size, int topk, void* out, float* lse,
+                         cudaStream_t stream);
+
+/*
  * moba_fwd_host - moba_fwd on HOST buffers (same layouts): copies q, k, v to
  * the device, runs the forward pass and copies out and lse back, all on
  * `stream`, and synchronises the stream before returning. Host buffers that

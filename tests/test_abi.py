@@ -87,3 +87,9 @@ def test_chunk_rejects_a_query_start_outside_the_sequence(lib, q_start):
     rc = lib.moba_fwd_chunk(FAKE, FAKE, FAKE, 4096, q_start, 1, 1, 128, 512, 3, FAKE, FAKE, None)
     assert rc == moba.MOBA_ERR_INVALID_ARG
     assert "q_start" in moba.last_error()
+
+
+def test_chunk_with_means_rejects_null_means(lib):
+    rc = lib.moba_fwd_chunk_means(FAKE, FAKE, FAKE, None, 4096, 4000, 1, 1, 128, 512, 3, FAKE, FAKE, None)
+    assert rc == moba.MOBA_ERR_INVALID_ARG
+    assert "kmean" in moba.last_error()

@@ -68,3 +68,19 @@ def test_decode_row_against_the_oracle():
     err = np.abs(out_c[0].float().cpu().numpy() - out_o).max()
     assert err <= OUT_MAX_ABS, err
     assert np.abs(lse_c[:, 0].cpu().numpy() - lse_o).max() <= LSE_ABS
+
+
+@pytest.mark.parametrize("S,Hq,Hkv,B,topk,q0", [(5000, 8, 2, 512, 6, 4999), (3000, 4, 2, 256, 4, 1000)])
+def test_chunk_with_the_callers_means(S, Hq, Hkv, B, topk, q0):
+    # means from pool() replace the per-call pooling; they only steer the
+    # gate, so the chunk's rows come out the same
+    _, q, k, v = make_inputs(S, Hq, Hkv, B, topk, 300 + q0 % 89)
+    qd, kd, vd = to_dev(q), to_dev(k), to_dev(v)
+    qc = qd[q0:].contiguous()
+    ref = moba.fwd_chunk(qc, kd, vd, B, topk)
+    kmean = moba.pool(kd, B)
+    got = moba.fwd_chunk(qc, kd, vd, B, topk, kmean=kmean)
+    torch.cuda.synchronize()
+    assert moba.device_status() == moba.MOBA_OK
+    assert torch.equal(got[0], ref[0])
+    assert torch.equal(got[1], ref[1])
