@@ -331,6 +331,103 @@ def run_chunk(args, w):
     return 0
 
 
+def varlen_lengths(w, n: int):
+    """--varlen N: the workload's tokens cut into N sequences at seeded
+    uniform cut points (each at least 1 token)."""
+    rng = np.random.default_rng(w.seed + 7919)
+    cuts = np.sort(rng.choice(np.arange(1, w.seqlen), size=n - 1, replace=False)) if n > 1 else np.array([], int)
+    edges = np.concatenate([[0], cuts, [w.seqlen]]).astype(np.int64)
+    return np.diff(edges), edges
+
+
+def run_varlen(args, w):
+    """--varlen N: one packed batch of N independent sequences of the
+    workload's head shape, block size and top-k (moba_fwd_varlen). One GPU."""
+    import torch
+
+    import block_sparse_long_fwd_b200 as moba
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    T, Hq, Hkv, d = w.seqlen, w.heads_q, w.heads_kv, w.head_dim
+    lengths, cu = varlen_lengths(w, args.varlen)
+    subs = [si.Workload(f"{w.name}_seq{b}", int(L), Hq, Hkv, d, w.block_size, w.topk, w.seed + 1000 + b)
+            for b, L in enumerate(lengths)]
+    q_h = torch.empty((T, Hq, d), dtype=torch.bfloat16, pin_memory=True)
+    k_h = torch.empty((T, Hkv, d), dtype=torch.bfloat16, pin_memory=True)
+    v_h = torch.empty((T, Hkv, d), dtype=torch.bfloat16, pin_memory=True)
+    for b, sw in enumerate(subs):
+        a, e = int(cu[b]), int(cu[b + 1])
+        si.fill_q(q_h[a:e].data_ptr(), sw)
+        si.fill_k(k_h[a:e].data_ptr(), sw)
+        si.fill_v(v_h[a:e].data_ptr(), sw)
+    q, k, v = q_h.to(dev), k_h.to(dev), v_h.to(dev)
+    out = torch.empty((T, Hq, d), dtype=torch.bfloat16, device=dev)
+    lse = torch.empty((Hq, T), dtype=torch.float32, device=dev)
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+    for _ in range(args.warmup):
+        flush.zero_()
+        moba.fwd_varlen(q, k, v, cu, w.block_size, w.topk, out=out, lse=lse)
+    sampler = ClockSampler(None)
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    for a, b in ev:
+        flush.zero_()
+        a.record(stream)
+        moba.fwd_varlen(q, k, v, cu, w.block_size, w.topk, out=out, lse=lse)
+        b.record(stream)
+    torch.cuda.synchronize()
+    total_ms = sum(a.elapsed_time(b) for a, b in ev)
+    moba.profile_begin()
+    for _ in range(args.steps):
+        flush.zero_()
+        moba.fwd_varlen(q, k, v, cu, w.block_size, w.topk, out=out, lse=lse)
+    stages, launches, calls = moba.profile_end()
+    torch.cuda.synchronize()
+    clocks = sampler.stop()
+    if moba.device_status() != 0:
+        raise RuntimeError("device status set: " + moba.last_error())
+    out_h = torch.empty((T, Hq, d), dtype=torch.bfloat16, pin_memory=True)
+    lse_h = torch.empty((Hq, T), dtype=torch.float32, pin_memory=True)
+    e2e_steps = max(1, min(args.steps, 5))
+    t0 = time.perf_counter()
+    for _ in range(e2e_steps):
+        q.copy_(q_h, non_blocking=True)
+        k.copy_(k_h, non_blocking=True)
+        v.copy_(v_h, non_blocking=True)
+        moba.fwd_varlen(q, k, v, cu, w.block_size, w.topk, out=out, lse=lse)
+        out_h.copy_(out, non_blocking=True)
+        lse_h.copy_(lse, non_blocking=True)
+        torch.cuda.synchronize()
+    e2e_ms = 1e3 * (time.perf_counter() - t0)
+    peaks, peaks_src = load_peaks()
+    flops = sum(chunk_flops(sw, 0) for sw in subs)
+    attn_ms = stages["attention"] / args.steps
+    achieved = flops / (attn_ms / 1e3) / 1e12
+    line = {
+        "metric": METRIC, "value": T * args.steps / (total_ms / 1e3), "unit": "tokens/s", "n_gpus": 1,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": dict(workload_config(w, 1), mode="packed batch", batch_per_gpu=int(args.varlen),
+                       lengths=[int(x) for x in lengths]),
+        "eff_tflops": flops * args.steps / (total_ms / 1e3) / 1e12,
+        "stage_ms_per_step": {kk: vv / args.steps for kk, vv in stages.items()},
+        "roofline": {"bound": "tensor", "kernel": "attn_kernel", "achieved": achieved,
+                     "peak": peaks["bf16_tflops"], "unit": "TFLOP/s", "frac": achieved / peaks["bf16_tflops"],
+                     "traffic": None, "peak_source": f"{peaks_src} bf16 burst",
+                     "algorithmic": f"{flops:.4e} selected-block FLOPs of all sequences / attention ms"},
+        "e2e": {"value": T * e2e_steps / (e2e_ms / 1e3), "unit": "tokens/s",
+                "h2d_bytes_per_step": int(q_h.nbytes + k_h.nbytes + v_h.nbytes),
+                "d2h_bytes_per_step": int(out_h.nbytes + lse_h.nbytes)},
+        "gpu_launches": launches // args.steps * args.steps,
+        "gpu_launches_per_step": launches / args.steps,
+        "clocks": clocks,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def workload_config(w, n):
     return {"workload": w.name, "seqlen": w.seqlen, "heads_q": w.heads_q, "heads_kv": w.heads_kv,
             "head_dim": w.head_dim, "block_size": w.block_size, "topk": w.topk, "batch_per_gpu": 1,
@@ -509,6 +606,8 @@ def main():
                     help="time only the last N tokens' queries against the whole cache (1 = one decode step)")
     ap.add_argument("--cached-means", action="store_true",
                     help="with --chunk: pool the block means once instead of on every call")
+    ap.add_argument("--varlen", type=int, default=0,
+                    help="time one packed batch of N independent sequences that together hold the workload's tokens")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -522,6 +621,10 @@ def main():
         if not 1 <= args.chunk <= w.seqlen:
             ap.error("--chunk must be in [1, seqlen]")
         return run_chunk(args, w)
+    if args.varlen:
+        if not 1 <= args.varlen <= w.seqlen or args.chunk:
+            ap.error("--varlen must be in [1, seqlen] and not combined with --chunk")
+        return run_varlen(args, w)
     return run_ours(args, w)
 
 

@@ -34,6 +34,7 @@ SIGNATURES = {
     "moba_fwd": (_i32, [_vp, _vp, _vp, _i64, _i32, _i32, _i32, _i32, _i32, _vp, _vp, _vp]),
     "moba_fwd_chunk": (_i32, [_vp, _vp, _vp, _i64, _i64, _i32, _i32, _i32, _i32, _i32, _vp, _vp, _vp]),
     "moba_fwd_chunk_means": (_i32, [_vp, _vp, _vp, _vp, _i64, _i64, _i32, _i32, _i32, _i32, _i32, _vp, _vp, _vp]),
+    "moba_fwd_varlen": (_i32, [_vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _i32, _vp, _vp, _vp]),
     "moba_fwd_host": (_i32, [_vp, _vp, _vp, _i64, _i32, _i32, _i32, _i32, _i32, _vp, _vp, _vp]),
     "moba_pool": (_i32, [_vp, _i64, _i32, _i32, _i32, _vp, _vp]),
     "moba_gate": (_i32, [_vp, _vp, _i64, _i32, _i32, _i32, _i32, _i32, _vp, _vp]),
@@ -142,6 +143,32 @@ def fwd_chunk(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, block_size: int
         return out, lse
     _check(lib().moba_fwd_chunk(q.data_ptr(), k.data_ptr(), v.data_ptr(), S, S - n, Hq, Hkv, d, block_size, topk,
                                 out.data_ptr(), lse.data_ptr(), _stream(stream)))
+    return out, lse
+
+
+def fwd_varlen(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, cu_seqlens, block_size: int, topk: int, out=None,
+               lse=None, stream=None):
+    """MoBA forward over a packed batch of independent sequences.
+
+    q [T,Hq,128], k/v [T,Hkv,128] bf16 on the GPU hold the sequences one after
+    another; ``cu_seqlens`` (a sequence of ints or a CPU tensor, length
+    batch + 1, starting at 0) gives their offsets. Returns (out [T,Hq,128]
+    bf16, lse [Hq,T] fp32); sequence b's rows equal ``fwd`` on its tokens.
+    """
+    _dev_bf16(q, "q"), _dev_bf16(k, "k"), _dev_bf16(v, "v")
+    T, Hq, d = q.shape
+    Hkv = k.shape[1]
+    if k.shape != (T, Hkv, d) or v.shape != k.shape:
+        raise ValueError("k and v must be [T, heads_kv, head_dim] matching q")
+    cu = torch.as_tensor(cu_seqlens, dtype=torch.int64, device="cpu").contiguous()
+    if cu.dim() != 1 or cu.numel() < 2 or int(cu[-1]) != T:
+        raise ValueError("cu_seqlens must be 1-D with batch + 1 entries ending at q.shape[0]")
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((Hq, T), dtype=torch.float32, device=q.device)
+    _check(lib().moba_fwd_varlen(q.data_ptr(), k.data_ptr(), v.data_ptr(), cu.data_ptr(), cu.numel() - 1, Hq, Hkv, d,
+                                 block_size, topk, out.data_ptr(), lse.data_ptr(), _stream(stream)))
     return out, lse
 
 

@@ -23,7 +23,8 @@ struct MergeParams {
   const __half* own_o;
   const float* own_lse;
   __nv_bfloat16* out;  // [S - q0][Hq][128]: rows of the tokens with a query
-  float* lse;          // [Hq][S - q0]
+  float* lse;          // [Hq][lse_ld]: row h, column t - q0
+  int64_t lse_ld;      // S - q0, or the packed token count of a batch
   WindowGeom w;
 };
 
@@ -185,7 +186,7 @@ __global__ void __launch_bounds__(256) merge_kernel(MergeParams m) {
   }
   uint2 packed = make_uint2(pack_bf16x2(acc.x, acc.y), pack_bf16x2(acc.z, acc.w));
   *reinterpret_cast<uint2*>(m.out + (tq * w.Hq + h) * kHeadDim + lane * 4) = packed;
-  if (lane == 0) m.lse[(int64_t)h * nq + tq] = L;
+  if (lane == 0) m.lse[(int64_t)h * m.lse_ld + tq] = L;
 }
 
 }  // namespace moba

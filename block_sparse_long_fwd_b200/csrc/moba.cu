@@ -10,6 +10,7 @@
 #include <cstdio>
 #include <cstdlib>
 #include <cstring>
+#include <functional>
 #include <mutex>
 #include <string>
 #include <vector>
@@ -152,6 +153,7 @@ struct Plan {
   int64_t q0 = 0;     // first token with a query (0: a whole prefill)
   const float* means = nullptr;  // caller's block means [Hkv][nbp][128] (then no pooling)
   int64_t wbase = 0;  // first window start: q0 rounded down to 256 tokens
+  int64_t lse_ld = 0;  // lse row stride: S - q0, or a packed batch's tokens
   int Hq, Hkv, G, B, topk, k_eff, P, nb, nbp;
   int splits = 1;  // pool row splits per block
   int64_t W;       // window tokens (multiple of 128)
@@ -238,11 +240,12 @@ void dense_blocks(Plan& p) {
   p.P = p.k_eff - 1;
 }
 
-int make_plan(Plan* pl, int64_t S, int64_t q0, int Hq, int Hkv, int B, int topk) {
-  Plan& p = *pl;
+// The problem's shape; the scratch layout comes after.
+void plan_shape(Plan& p, int64_t S, int64_t q0, int Hq, int Hkv, int B, int topk) {
   p.S = S;
   p.q0 = q0;
   p.wbase = q0 / 256 * 256;
+  p.lse_ld = S - q0;
   p.Hq = Hq;
   p.Hkv = Hkv;
   p.G = Hq / Hkv;
@@ -253,6 +256,11 @@ int make_plan(Plan* pl, int64_t S, int64_t q0, int Hq, int Hkv, int B, int topk)
   p.k_eff = std::min(topk, p.nb);
   p.P = p.k_eff - 1;
   dense_blocks(p);
+}
+
+int make_plan(Plan* pl, int64_t S, int64_t q0, int Hq, int Hkv, int B, int topk) {
+  Plan& p = *pl;
+  plan_shape(p, S, q0, Hq, Hkv, B, topk);
   const int64_t S128 = (S - p.wbase + 127) / 128 * 128;  // tokens the windows cover
   int64_t W = 0;
   if (const char* env = getenv("MOBA_WINDOW")) {
@@ -510,6 +518,7 @@ int run_forward(const Plan& p, const DeviceInfo& dev, const void* q, const void*
     mp.own_lse = own_lse;
     mp.out = static_cast<__nv_bfloat16*>(out);
     mp.lse = lse;
+    mp.lse_ld = p.lse_ld;
     mp.w = wg;
     const int64_t rows = wg.wlen * p.Hq;
     const dim3 mg((unsigned)((rows + 7) / 8));
@@ -529,16 +538,18 @@ extern "C" const char* moba_last_error(void) { return g_err.c_str(); }
 
 namespace {
 
+// A launch sequence over one scratch buffer of `total` bytes.
+using Runner = std::function<int(uint8_t* ws, cudaStream_t st)>;
+
 // The launch sequence with stream-ordered scratch, issued on `stream`.
-int direct_forward(const Plan& p, const DeviceInfo& dev, const void* q, const void* k, const void* v, void* out,
-                   float* lse, cudaStream_t stream) {
+int direct_run(size_t total, const Runner& run, cudaStream_t stream) {
   void* ws = nullptr;
-  cudaError_t e = cudaMallocAsync(&ws, p.total, stream);
+  cudaError_t e = cudaMallocAsync(&ws, total, stream);
   if (e != cudaSuccess) {
     cudaGetLastError();
-    return fail(MOBA_ERR_OOM, "scratch allocation of %zu bytes failed: %s", p.total, cudaGetErrorString(e));
+    return fail(MOBA_ERR_OOM, "scratch allocation of %zu bytes failed: %s", total, cudaGetErrorString(e));
   }
-  int rc = run_forward(p, dev, q, k, v, out, lse, static_cast<uint8_t*>(ws), stream);
+  int rc = run(static_cast<uint8_t*>(ws), stream);
   cudaError_t ef = cudaFreeAsync(ws, stream);
   if (rc) return rc;
   if (ef != cudaSuccess) return fail(MOBA_ERR_CUDA, "cudaFreeAsync failed: %s", cudaGetErrorString(ef));
@@ -548,21 +559,22 @@ int direct_forward(const Plan& p, const DeviceInfo& dev, const void* q, const vo
 // Repeated calls with the same buffers and shape replay a CUDA graph of the
 // whole launch sequence (scratch allocation and release included as graph
 // memory nodes), so the host enqueues one graph launch instead of about ten
-// kernels. Graphs are captured on an internal stream, launched on the
-// caller's, and kept for the last kGraphCache argument sets; a set is only
-// captured the second time it is seen. MOBA_GRAPH=0 turns this off.
+// kernels per sequence. Graphs are captured on an internal stream, launched
+// on the caller's, and kept for the last kGraphCache argument sets; a set is
+// only captured the second time it is seen. MOBA_GRAPH=0 turns this off.
 struct GraphKey {
   int dev;
   const void *q, *k, *v;
   void* out;
   float* lse;
   const float* means;
-  int64_t S, q0, W;
+  int64_t S, q0, W, lse_ld;
   int Hq, Hkv, B, topk;
+  std::vector<int64_t> cu;  // a packed batch's sequence offsets (empty: one sequence)
   bool operator==(const GraphKey& o) const {
     return dev == o.dev && q == o.q && k == o.k && v == o.v && out == o.out && lse == o.lse && means == o.means &&
-           S == o.S &&
-           q0 == o.q0 && W == o.W && Hq == o.Hq && Hkv == o.Hkv && B == o.B && topk == o.topk;
+           S == o.S && q0 == o.q0 && W == o.W && lse_ld == o.lse_ld && Hq == o.Hq && Hkv == o.Hkv && B == o.B &&
+           topk == o.topk && cu == o.cu;
   }
 };
 
@@ -583,13 +595,12 @@ bool graphs_enabled() {
 }
 
 // MOBA_OK / error after launching a graph; -1 when the caller should launch
-// directly.
-int graph_forward(const Plan& p, const DeviceInfo& dev, const void* q, const void* k, const void* v, void* out,
-                  float* lse, cudaStream_t stream) {
+// directly. key.dev is filled in here.
+int graph_run(GraphKey key, size_t total, const Runner& run, cudaStream_t stream) {
   if (!graphs_enabled()) return -1;
   int d = 0;
   if (cudaGetDevice(&d) != cudaSuccess || d < 0 || d >= 64) return -1;
-  GraphKey key{d, q, k, v, out, lse, p.means, p.S, p.q0, p.W, p.Hq, p.Hkv, p.B, p.topk};
+  key.dev = d;
   std::lock_guard<std::mutex> lk(g_graph_mu);
   GraphEntry* hit = nullptr;
   for (GraphEntry& en : g_graphs)
@@ -607,7 +618,7 @@ int graph_forward(const Plan& p, const DeviceInfo& dev, const void* q, const voi
       if (g_graphs.front().state == 1) cudaGraphExecDestroy(g_graphs.front().exec);
       g_graphs.erase(g_graphs.begin());
     }
-    g_graphs.push_back({key, nullptr, 0});
+    g_graphs.push_back({std::move(key), nullptr, 0});
     return -1;
   }
   if (!g_capture_stream[d] && cudaStreamCreateWithFlags(&g_capture_stream[d], cudaStreamNonBlocking) != cudaSuccess) {
@@ -621,9 +632,9 @@ int graph_forward(const Plan& p, const DeviceInfo& dev, const void* q, const voi
   bool ok = cudaStreamBeginCapture(cs, cudaStreamCaptureModeThreadLocal) == cudaSuccess;
   if (ok) {
     void* ws = nullptr;
-    ok = cudaMallocAsync(&ws, p.total, cs) == cudaSuccess;
+    ok = cudaMallocAsync(&ws, total, cs) == cudaSuccess;
     if (ok) {
-      ok = run_forward(p, dev, q, k, v, out, lse, static_cast<uint8_t*>(ws), cs) == MOBA_OK;
+      ok = run(static_cast<uint8_t*>(ws), cs) == MOBA_OK;
       ok = (cudaFreeAsync(ws, cs) == cudaSuccess) && ok;
     }
     ok = (cudaStreamEndCapture(cs, &graph) == cudaSuccess) && ok;
@@ -664,11 +675,71 @@ int fwd_impl(const void* q, const void* k, const void* v, int64_t seqlen, int64_
   if (rc) return rc;
   if (means && !aligned16(means)) return fail(MOBA_ERR_INVALID_ARG, "kmean must be 16-byte aligned");
   p.means = means;
+  const Runner run = [&](uint8_t* ws, cudaStream_t st) { return run_forward(p, dev, q, k, v, out, lse, ws, st); };
   if (use_graph && !g_timer.on) {
-    const int g = graph_forward(p, dev, q, k, v, out, lse, stream);
+    GraphKey key{0, q, k, v, out, lse, p.means, p.S, p.q0, p.W, p.lse_ld, p.Hq, p.Hkv, p.B, p.topk, {}};
+    const int g = graph_run(std::move(key), p.total, run, stream);
     if (g >= 0) return g;  // negative: no graph for this call, launch directly
   }
-  return direct_forward(p, dev, q, k, v, out, lse, stream);
+  return direct_run(p.total, run, stream);
+}
+
+// A packed batch of independent sequences: sequence b holds tokens
+// cu[b] .. cu[b+1]-1 of q, k, v and out, and columns cu[b] .. of lse. The
+// sequences run one after another on one scratch buffer (the largest any of
+// them needs), as one graph when the same batch comes back.
+int varlen_impl(const void* q, const void* k, const void* v, const int64_t* cu, int batch, int heads_q, int heads_kv,
+                int head_dim, int block_size, int topk, void* out, float* lse, cudaStream_t stream) {
+  g_err.clear();
+  if (!q || !k || !v || !out || !lse || !cu) return fail(MOBA_ERR_INVALID_ARG, "null pointer argument");
+  if (batch < 1) return fail(MOBA_ERR_INVALID_ARG, "batch must be >= 1 (got %d)", batch);
+  if (cu[0] != 0) return fail(MOBA_ERR_INVALID_ARG, "cu_seqlens[0] must be 0 (got %lld)", (long long)cu[0]);
+  for (int b = 0; b < batch; ++b)
+    if (cu[b + 1] < cu[b])
+      return fail(MOBA_ERR_INVALID_ARG, "cu_seqlens must be non-decreasing (cu_seqlens[%d] = %lld < %lld)", b + 1,
+                  (long long)cu[b + 1], (long long)cu[b]);
+  const int64_t T = cu[batch];
+  if (T < 1) return fail(MOBA_ERR_INVALID_ARG, "the batch holds no tokens");
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out))
+    return fail(MOBA_ERR_INVALID_ARG, "device buffers must be 16-byte aligned");
+  if (reinterpret_cast<uintptr_t>(lse) & 3) return fail(MOBA_ERR_INVALID_ARG, "lse must be 4-byte aligned");
+  std::vector<Plan> plans;
+  std::vector<int64_t> starts;
+  size_t total = 0;
+  for (int b = 0; b < batch; ++b) {
+    const int64_t L = cu[b + 1] - cu[b];
+    if (!L) continue;  // an empty sequence has nothing to compute
+    int rc = check_shape(L, heads_q, heads_kv, head_dim, block_size, topk);
+    if (rc) return rc;
+    Plan p;
+    rc = make_plan(&p, L, 0, heads_q, heads_kv, block_size, topk);
+    if (rc) return rc;
+    p.lse_ld = T;
+    total = std::max(total, p.total);
+    plans.push_back(p);
+    starts.push_back(cu[b]);
+  }
+  DeviceInfo dev;
+  int rc = device_info(&dev);
+  if (rc) return rc;
+  const size_t qrow = (size_t)heads_q * head_dim * 2, kvrow = (size_t)heads_kv * head_dim * 2;
+  const Runner run = [&](uint8_t* ws, cudaStream_t st) {
+    for (size_t i = 0; i < plans.size(); ++i) {
+      const size_t t0 = (size_t)starts[i];
+      const int r = run_forward(plans[i], dev, static_cast<const uint8_t*>(q) + t0 * qrow,
+                                static_cast<const uint8_t*>(k) + t0 * kvrow, static_cast<const uint8_t*>(v) + t0 * kvrow,
+                                static_cast<uint8_t*>(out) + t0 * qrow, lse + t0, ws, st);
+      if (r) return r;
+    }
+    return (int)MOBA_OK;
+  };
+  if (!g_timer.on) {
+    GraphKey key{0, q, k, v, out, lse, nullptr, T, 0, 0, T, heads_q, heads_kv, block_size, topk,
+                 std::vector<int64_t>(cu, cu + batch + 1)};
+    const int g = graph_run(std::move(key), total, run, stream);
+    if (g >= 0) return g;
+  }
+  return direct_run(total, run, stream);
 }
 
 }  // namespace
@@ -691,6 +762,12 @@ int moba_fwd_chunk_means(const void* q, const void* k, const void* v, const floa
   if (!kmean) return fail(MOBA_ERR_INVALID_ARG, "null pointer argument (kmean)");
   return fwd_impl(q, k, v, seqlen, q_start, heads_q, heads_kv, head_dim, block_size, topk, out, lse, stream, true,
                   kmean);
+}
+
+int moba_fwd_varlen(const void* q, const void* k, const void* v, const int64_t* cu_seqlens, int batch, int heads_q,
+                    int heads_kv, int head_dim, int block_size, int topk, void* out, float* lse,
+                    cudaStream_t stream) {
+  return varlen_impl(q, k, v, cu_seqlens, batch, heads_q, heads_kv, head_dim, block_size, topk, out, lse, stream);
 }
 
 int moba_profile_begin(void) {
@@ -893,17 +970,7 @@ int noalloc_scratch(void** out) {
 // `cap` bytes; fails when not even a 128-token window fits.
 int plan_within(Plan* pl, int64_t S, int Hq, int Hkv, int B, int topk, size_t cap) {
   Plan& p = *pl;
-  p.S = S;
-  p.Hq = Hq;
-  p.Hkv = Hkv;
-  p.G = Hq / Hkv;
-  p.B = B;
-  p.topk = topk;
-  p.nb = (int)((S + B - 1) / B);
-  p.nbp = p.nb - 1;
-  p.k_eff = std::min(topk, p.nb);
-  p.P = p.k_eff - 1;
-  dense_blocks(p);
+  plan_shape(p, S, 0, Hq, Hkv, B, topk);
   int64_t W = (S + 127) / 128 * 128;
   while (true) {
     if (W * Hq * (int64_t)p.P < ((int64_t)1 << 31) - 1) {

@@ -138,6 +138,33 @@ int moba_fwd_chunk_means(const void* q, const void* k, const void* v,
                          cudaStream_t stream);
 
 /*
+ * moba_fwd_varlen - moba_fwd over a packed batch of independent sequences
+ * (serving several long-context requests in one call: "MoBA (Mixture of
+ * Block Attention)" project summary, "Deployment"; "MoBA: Mixture of Block
+ * Attention for Long-Context LLMs" abstract). Sequence b is tokens
+ * cu_seqlens[b] .. cu_seqlens[b+1]-1 of the packed buffers. Each sequence is
+ * its own causal problem: its blocks start at its first token, and no query
+ * attends across a sequence boundary, so sequence b's rows equal moba_fwd
+ * called on its tokens alone.
+ *
+ * q, k, v    device bf16 [T][heads][head_dim], T = cu_seqlens[batch].
+ * cu_seqlens HOST int64 [batch + 1]: 0 = cu_seqlens[0] <= cu_seqlens[1] <=
+ *            ...; a zero-length sequence is skipped. Read during the call
+ *            only.
+ * batch      number of sequences, >= 1.
+ * out        device bf16 output [T][heads_q][head_dim].
+ * lse        device fp32 output [heads_q][T] (column = packed token index),
+ *            4-byte aligned.
+ * Shape rules per sequence, stream, graph replay, ownership and errors as
+ * moba_fwd; cu_seqlens that are not 0-based and non-decreasing, or hold no
+ * token, return MOBA_ERR_INVALID_ARG before any launch.
+ */
+int moba_fwd_varlen(const void* q, const void* k, const void* v,
+                    const int64_t* cu_seqlens, int batch, int heads_q,
+                    int heads_kv, int head_dim, int block_size, int topk,
+                    void* out, float* lse, cudaStream_t stream);
+
+/*
  * moba_fwd_host - moba_fwd on HOST buffers (same layouts): copies q, k, v to
  * the device, runs the forward pass and copies out and lse back, all on
  * `stream`, and synchronises the stream before returning. Host buffers that

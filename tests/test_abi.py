@@ -93,3 +93,35 @@ def test_chunk_with_means_rejects_null_means(lib):
     rc = lib.moba_fwd_chunk_means(FAKE, FAKE, FAKE, None, 4096, 4000, 1, 1, 128, 512, 3, FAKE, FAKE, None)
     assert rc == moba.MOBA_ERR_INVALID_ARG
     assert "kmean" in moba.last_error()
+
+
+def _cu(vals):
+    arr = (ctypes.c_int64 * len(vals))(*vals)
+    return arr, len(vals) - 1
+
+
+@pytest.mark.parametrize("cu, what", [
+    ([1, 4096], "cu_seqlens[0]"),
+    ([0, 4096, 2048], "non-decreasing"),
+    ([0, 0, 0], "no tokens"),
+    ([0], "batch"),
+])
+def test_varlen_rejects_bad_offsets_before_launch(lib, cu, what):
+    arr, batch = _cu(cu)
+    rc = lib.moba_fwd_varlen(FAKE, FAKE, FAKE, ctypes.cast(arr, ctypes.c_void_p), batch, 1, 1, 128, 512, 3, FAKE,
+                             FAKE, None)
+    assert rc == moba.MOBA_ERR_INVALID_ARG
+    assert what in moba.last_error()
+
+
+def test_varlen_checks_each_sequence_shape_and_pointers(lib):
+    arr, batch = _cu([0, 4096, 8192])
+    rc = lib.moba_fwd_varlen(FAKE, FAKE, FAKE, None, batch, 1, 1, 128, 512, 3, FAKE, FAKE, None)
+    assert rc == moba.MOBA_ERR_INVALID_ARG and "null" in moba.last_error()
+    # lse only needs 4-byte alignment (a sequence's lse columns start anywhere)
+    rc = lib.moba_fwd_varlen(FAKE, FAKE, FAKE, ctypes.cast(arr, ctypes.c_void_p), batch, 1, 1, 128, 512, 3, FAKE,
+                             FAKE + 2, None)
+    assert rc == moba.MOBA_ERR_INVALID_ARG and "lse" in moba.last_error()
+    rc = lib.moba_fwd_varlen(FAKE, FAKE, FAKE, ctypes.cast(arr, ctypes.c_void_p), batch, 3, 2, 128, 512, 3, FAKE,
+                             FAKE + 4, None)
+    assert rc == moba.MOBA_ERR_INVALID_ARG and "multiple" in moba.last_error()
