@@ -24,7 +24,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 _SRC = os.path.join(_HERE, "gen.c")
 _LIB = os.path.join(_HERE, "libsynth.so")
 
-STREAM_Q, STREAM_K, STREAM_V, STREAM_MU = 1, 2, 3, 4
+STREAM_Q, STREAM_K, STREAM_V, STREAM_MU, STREAM_DO = 1, 2, 3, 4, 5
 
 
 @dataclass(frozen=True)
@@ -122,6 +122,20 @@ def fill_v(ptr: int, w: Workload, t0: int = 0, nrows: int | None = None, threads
     nrows = w.seqlen - t0 if nrows is None else nrows
     per = w.heads_kv * w.head_dim
     lib().synth_fill_normal_bf16(ptr, nrows * per, w.seed, STREAM_V, t0 * per, threads or default_threads())
+
+
+def fill_dout(ptr: int, w: Workload, t0: int = 0, nrows: int | None = None, threads: int | None = None) -> None:
+    """Upstream gradient dO [S][Hq][d] for the backward pass: i.i.d. N(0, 1) bf16."""
+    nrows = w.seqlen - t0 if nrows is None else nrows
+    per = w.heads_q * w.head_dim
+    lib().synth_fill_normal_bf16(ptr, nrows * per, w.seed, STREAM_DO, t0 * per, threads or default_threads())
+
+
+def make_dout(w: Workload, threads: int | None = None) -> np.ndarray:
+    """Host numpy uint16 (bf16 bit patterns) dO [S,Hq,d]."""
+    do = np.empty((w.seqlen, w.heads_q, w.head_dim), dtype=np.uint16)
+    fill_dout(do.ctypes.data, w, threads=threads)
+    return do
 
 
 def fill_k(ptr: int, w: Workload, mu: np.ndarray | None = None, t0: int = 0, nrows: int | None = None,

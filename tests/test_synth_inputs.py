@@ -51,3 +51,14 @@ def test_key_offsets_have_stated_norm_and_shift_blocks():
     kf = si.bf16_bits_to_f64(k).reshape(w.nblocks, w.block_size, w.heads_kv, w.head_dim)
     blk_mean = kf.mean(axis=1).transpose(1, 0, 2)
     assert np.abs(blk_mean - mu).max() < 0.35  # N(0,1)/sqrt(256) noise, 128*8*2 draws
+
+
+def test_upstream_gradient_stream_is_standard_normal_and_its_own():
+    w = si.Workload("dout", 4096, 2, 1, 128, 512, 3, 5)
+    do = si.bf16_bits_to_f64(si.make_dout(w, threads=2))
+    q = si.bf16_bits_to_f64(si.make_qkv(w, threads=2)[0])
+    assert abs(do.mean()) < 0.01 and abs(do.std() - 1.0) < 0.01
+    assert not np.array_equal(do, q)
+    part = np.empty((100, 2, 128), dtype=np.uint16)
+    si.fill_dout(part.ctypes.data, w, t0=1000, nrows=100, threads=1)
+    assert np.array_equal(si.bf16_bits_to_f64(part), do[1000:1100])
