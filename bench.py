@@ -331,6 +331,97 @@ def run_chunk(args, w):
     return 0
 
 
+def run_backward(args, w):
+    """--backward: the gradient (moba_bwd) of the workload's forward pass,
+    given its out and lse; one GPU. FLOPs: the five products of attention's
+    gradient per attended pair (S recomputed, dP, dV, dK, dQ: 2.5 times the
+    forward's), plus dP and S recomputed once more in the dQ kernel."""
+    import torch
+
+    import block_sparse_long_fwd_b200 as moba
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    S, Hq, Hkv, d = w.seqlen, w.heads_q, w.heads_kv, w.head_dim
+    q_h = torch.empty((S, Hq, d), dtype=torch.bfloat16, pin_memory=True)
+    k_h = torch.empty((S, Hkv, d), dtype=torch.bfloat16, pin_memory=True)
+    v_h = torch.empty((S, Hkv, d), dtype=torch.bfloat16, pin_memory=True)
+    do_h = torch.empty((S, Hq, d), dtype=torch.bfloat16, pin_memory=True)
+    si.fill_q(q_h.data_ptr(), w)
+    si.fill_k(k_h.data_ptr(), w)
+    si.fill_v(v_h.data_ptr(), w)
+    si.fill_dout(do_h.data_ptr(), w)
+    q, k, v, do = q_h.to(dev), k_h.to(dev), v_h.to(dev), do_h.to(dev)
+    out, lse = moba.fwd(q, k, v, w.block_size, w.topk)
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+    for _ in range(args.warmup):
+        flush.zero_()
+        moba.bwd(q, k, v, out, lse, do, w.block_size, w.topk)
+    sampler = ClockSampler(None)
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    for a, b in ev:
+        flush.zero_()
+        a.record(stream)
+        moba.bwd(q, k, v, out, lse, do, w.block_size, w.topk)
+        b.record(stream)
+    torch.cuda.synchronize()
+    total_ms = sum(a.elapsed_time(b) for a, b in ev)
+    moba.profile_begin()
+    for _ in range(args.steps):
+        flush.zero_()
+        moba.bwd(q, k, v, out, lse, do, w.block_size, w.topk)
+    stages, launches, calls = moba.profile_end()
+    torch.cuda.synchronize()
+    clocks = sampler.stop()
+    if moba.device_status() != 0:
+        raise RuntimeError("device status set: " + moba.last_error())
+    # end to end: upload q, k, v, out, lse, dO; read dq, dk, dv back
+    out_h, lse_h = out.cpu().pin_memory(), lse.cpu().pin_memory()
+    dq_h = torch.empty((S, Hq, d), dtype=torch.bfloat16, pin_memory=True)
+    dk_h = torch.empty((S, Hkv, d), dtype=torch.bfloat16, pin_memory=True)
+    dv_h = torch.empty((S, Hkv, d), dtype=torch.bfloat16, pin_memory=True)
+    e2e_steps = max(1, min(args.steps, 5))
+    t0 = time.perf_counter()
+    for _ in range(e2e_steps):
+        for dst, src in ((q, q_h), (k, k_h), (v, v_h), (out, out_h), (lse, lse_h), (do, do_h)):
+            dst.copy_(src, non_blocking=True)
+        dq, dk, dv = moba.bwd(q, k, v, out, lse, do, w.block_size, w.topk)
+        dq_h.copy_(dq, non_blocking=True)
+        dk_h.copy_(dk, non_blocking=True)
+        dv_h.copy_(dv, non_blocking=True)
+        torch.cuda.synchronize()
+    e2e_ms = 1e3 * (time.perf_counter() - t0)
+    peaks, peaks_src = load_peaks()
+    fwd_flops = chunk_flops(w, 0)
+    per = {kk: vv / max(calls, 1) for kk, vv in stages.items()}
+    dkdv_flops = 2.0 * fwd_flops  # S^T, dP^T, dV, dK
+    achieved = dkdv_flops / (per["bwd_dkdv"] / 1e3) / 1e12
+    line = {
+        "metric": METRIC, "value": S * args.steps / (total_ms / 1e3), "unit": "tokens/s", "n_gpus": 1,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": dict(workload_config(w, 1), mode="backward (dq, dk, dv given out, lse, dout)"),
+        "eff_tflops": 2.5 * fwd_flops * args.steps / (total_ms / 1e3) / 1e12,
+        "stage_ms_per_step": per,
+        "roofline": {"bound": "tensor", "kernel": "bwd_dkdv_kernel", "achieved": achieved,
+                     "peak": peaks["bf16_tflops"], "unit": "TFLOP/s", "frac": achieved / peaks["bf16_tflops"],
+                     "traffic": None, "peak_source": f"{peaks_src} bf16 burst",
+                     "algorithmic": f"{dkdv_flops:.4e} FLOPs (S^T, dP^T, dV, dK per attended pair) / dK-dV ms",
+                     "dq_kernel_tflops": 1.5 * fwd_flops / (per["bwd_dq"] / 1e3) / 1e12},
+        "e2e": {"value": S * e2e_steps / (e2e_ms / 1e3), "unit": "tokens/s",
+                "h2d_bytes_per_step": int(q_h.nbytes + k_h.nbytes + v_h.nbytes + out_h.nbytes + lse_h.nbytes
+                                          + do_h.nbytes),
+                "d2h_bytes_per_step": int(dq_h.nbytes + dk_h.nbytes + dv_h.nbytes)},
+        "gpu_launches": launches // max(calls, 1) * args.steps,
+        "gpu_launches_per_step": launches / max(calls, 1),
+        "clocks": clocks,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def varlen_lengths(w, n: int):
     """--varlen N: the workload's tokens cut into N sequences at seeded
     uniform cut points (each at least 1 token)."""
@@ -608,6 +699,8 @@ def main():
                     help="with --chunk: pool the block means once instead of on every call")
     ap.add_argument("--varlen", type=int, default=0,
                     help="time one packed batch of N independent sequences that together hold the workload's tokens")
+    ap.add_argument("--backward", action="store_true",
+                    help="time the backward pass (moba_bwd) of the workload instead of the forward")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -621,6 +714,10 @@ def main():
         if not 1 <= args.chunk <= w.seqlen:
             ap.error("--chunk must be in [1, seqlen]")
         return run_chunk(args, w)
+    if args.backward:
+        if args.chunk or args.varlen:
+            ap.error("--backward does not combine with --chunk or --varlen")
+        return run_backward(args, w)
     if args.varlen:
         if not 1 <= args.varlen <= w.seqlen or args.chunk:
             ap.error("--varlen must be in [1, seqlen] and not combined with --chunk")

@@ -35,6 +35,7 @@ SIGNATURES = {
     "moba_fwd_chunk": (_i32, [_vp, _vp, _vp, _i64, _i64, _i32, _i32, _i32, _i32, _i32, _vp, _vp, _vp]),
     "moba_fwd_chunk_means": (_i32, [_vp, _vp, _vp, _vp, _i64, _i64, _i32, _i32, _i32, _i32, _i32, _vp, _vp, _vp]),
     "moba_fwd_varlen": (_i32, [_vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _i32, _vp, _vp, _vp]),
+    "moba_bwd": (_i32, [_vp, _vp, _vp, _vp, _vp, _vp, _i64, _i32, _i32, _i32, _i32, _i32, _vp, _vp, _vp, _vp]),
     "moba_fwd_host": (_i32, [_vp, _vp, _vp, _i64, _i32, _i32, _i32, _i32, _i32, _vp, _vp, _vp]),
     "moba_pool": (_i32, [_vp, _i64, _i32, _i32, _i32, _vp, _vp]),
     "moba_gate": (_i32, [_vp, _vp, _i64, _i32, _i32, _i32, _i32, _i32, _vp, _vp]),
@@ -172,7 +173,31 @@ def fwd_varlen(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, cu_seqlens, bl
     return out, lse
 
 
-STAGES = ("pool", "gate", "route", "attention", "merge")
+def bwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, out: torch.Tensor, lse: torch.Tensor,
+        dout: torch.Tensor, block_size: int, topk: int, stream=None):
+    """Gradient of ``fwd`` with the gate's choice held fixed.
+
+    q [S,Hq,128], k/v [S,Hkv,128], out and dout [S,Hq,128] bf16 and lse
+    [Hq,S] fp32 (``fwd``'s outputs) on the GPU. Returns (dq, dk, dv) bf16.
+    """
+    for name, x in (("q", q), ("k", k), ("v", v), ("out", out), ("dout", dout)):
+        _dev_bf16(x, name)
+    S, Hq, d = q.shape
+    Hkv = k.shape[1]
+    if k.shape != (S, Hkv, d) or v.shape != k.shape or out.shape != q.shape or dout.shape != q.shape:
+        raise ValueError("k, v must be [S, heads_kv, head_dim]; out and dout [S, heads_q, head_dim]")
+    if lse.dtype != torch.float32 or not lse.is_cuda or not lse.is_contiguous() or lse.shape != (Hq, S):
+        raise ValueError("lse must be a contiguous fp32 CUDA tensor [heads_q, S]")
+    dq = torch.empty_like(q)
+    dk = torch.empty_like(k)
+    dv = torch.empty_like(v)
+    _check(lib().moba_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(), dout.data_ptr(),
+                          S, Hq, Hkv, d, block_size, topk, dq.data_ptr(), dk.data_ptr(), dv.data_ptr(),
+                          _stream(stream)))
+    return dq, dk, dv
+
+
+STAGES = ("pool", "gate", "route", "attention", "merge", "bwd_prep", "bwd_dq", "bwd_dkdv")
 
 
 def profile_begin() -> None:

@@ -1,0 +1,642 @@
+// The backward pass: dQ, dK, dV of the MoBA forward with the gate's choice
+// held fixed (the top-k choice is piecewise constant, so the block means get
+// no gradient). MoBA is meant to be trained further from a full-attention
+// model ("MoBA (Mixture of Block Attention)" project summary, "Key Features";
+// "Efficient Long-Context Attention with MoBA", "How MoBA Works"), which
+// needs this gradient. Per q head h of kv head g, with c = 1/sqrt(128), the
+// row's attended keys (its selected past blocks and the causal part of its
+// own block), P = softmax(c Q K^T) there, D = rowsum(dO * O):
+//   dV = sum over the group's heads of P^T dO
+//   dS = P * (dO V^T - D)
+//   dQ = c dS K,   dK = sum over the group's heads of c dS^T Q.
+// P is rebuilt from the forward's lse: P = 2^(S c log2(e) - lse log2(e)).
+//
+// The work follows the forward's routing (pool, gate and router run again,
+// so the selection is the forward's):
+//   bwd_dq_kernel    per forward work unit and tile of 128 query rows:
+//                    S = Q K^T and dP = dO V^T on the tensor cores for each
+//                    128-key step of the unit's block, dS written back over
+//                    S in TMEM as bf16, dQ += dS K accumulated in TMEM; the
+//                    unit's c*dQ goes out as an fp16 partial into the slot
+//                    the forward uses for its partial output.
+//   bwd_dq_reduce    dQ = sum of a row's partials in a fixed order (its
+//                    selected past blocks ascending, its own block last).
+//   bwd_dkdv_kernel  per (kv head, block, 128-key tile): the transposed
+//                    products S^T = K Q^T and dP^T = V dO^T for every
+//                    128-row tile of the rows that attend the block (its
+//                    router list, then its own causal rows), P^T and dS^T
+//                    written back as bf16, dV += P^T dO and dK += dS^T Q
+//                    accumulated in TMEM over all of them; one fp32
+//                    read-add-write per key row and query window.
+// Both tensor-core kernels take K, V, Q and dO tiles in the 128-byte-swizzled
+// layout, read K-major for S / dP and MN-major for the dQ / dK / dV products.
+// Every mbarrier wait is bounded and sets the device status on a timeout.
+#pragma once
+
+#include "attn.cuh"
+#include "merge.cuh"
+#include "route.cuh"
+
+namespace moba {
+
+constexpr int kBwdThreads = 128;
+constexpr int kBwdSmemBytes = 6 * kTileBytes + 1024 + 4096;
+
+struct BwdParams {
+  const __nv_bfloat16* q;     // [S][Hq][128]
+  const __nv_bfloat16* dout;  // [S][Hq][128]
+  const float* lse2;          // [Hq][S]: the forward's lse times log2(e)
+  const float* dd;            // [Hq][S]: rowsum(dO * O)
+  int64_t S, w0, wlen;
+  int Hq, Hkv, G, B, nbp;
+  float scale_log2;  // log2(e) / sqrt(128)
+  float scale;       // 1 / sqrt(128)
+};
+
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait_group() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
+__device__ __forceinline__ float bwd_warp_sum(float v) {
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+// Row (t, h) of q / dO into row r of a 128-row tile in the 128-byte-swizzled
+// layout (two 64-column halves); a missing row (off < 0) is zero-filled.
+__device__ __forceinline__ void gather_row(uint32_t dst0, const __nv_bfloat16* base, int64_t off, int r) {
+  const bool valid = off >= 0;
+  const __nv_bfloat16* src = valid ? base + off : base;
+#pragma unroll
+  for (int c16 = 0; c16 < 16; ++c16) {
+    const int half = c16 >> 3, c = c16 & 7;
+    cp_async_16(dst0 + half * kHalfBytes + r * 128 + ((c ^ (r & 7)) << 4), src + (valid ? c16 * 8 : 0),
+                valid ? 16u : 0u);
+  }
+}
+
+// D = rowsum(dO * O) and lse * log2(e) per row. grid ceil(S*Hq/8), 256
+// threads: one warp per row (t, h); fixed-order shuffle sums.
+__global__ void __launch_bounds__(256) bwd_prep_kernel(const __nv_bfloat16* __restrict__ o,
+                                                       const __nv_bfloat16* __restrict__ dout,
+                                                       const float* __restrict__ lse, int64_t S, int Hq,
+                                                       float* __restrict__ lse2, float* __restrict__ dd) {
+  grid_dependency_sync();
+  const int lane = threadIdx.x & 31;
+  const int64_t row = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
+  if (row >= S * Hq) return;
+  const int64_t t = row / Hq;
+  const int h = (int)(row % Hq);
+  const uint2 a = __ldg(reinterpret_cast<const uint2*>(o + row * kHeadDim + lane * 4));
+  const uint2 b = __ldg(reinterpret_cast<const uint2*>(dout + row * kHeadDim + lane * 4));
+  const float2 a0 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&a.x));
+  const float2 a1 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&a.y));
+  const float2 b0 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&b.x));
+  const float2 b1 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&b.y));
+  float s = a0.x * b0.x;
+  s = fmaf(a0.y, b0.y, s);
+  s = fmaf(a1.x, b1.x, s);
+  s = fmaf(a1.y, b1.y, s);
+  s = bwd_warp_sum(s);
+  if (lane == 0) {
+    dd[(int64_t)h * S + t] = s;
+    lse2[(int64_t)h * S + t] = lse[(int64_t)h * S + t] * 1.4426950408889634f;
+  }
+}
+
+// n float4 zeros (the dK / dV accumulators before the first window).
+__global__ void __launch_bounds__(256) bwd_zero_kernel(float4* __restrict__ p, int64_t n) {
+  grid_dependency_sync();
+  for (int64_t i = (int64_t)blockIdx.x * 256 + threadIdx.x; i < n; i += (int64_t)gridDim.x * 256)
+    p[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+}
+
+// fp32 accumulators to bf16 outputs (n groups of four values).
+__global__ void __launch_bounds__(256) bwd_cast_kernel(const float4* __restrict__ a, __nv_bfloat16* __restrict__ out,
+                                                       int64_t n) {
+  grid_dependency_sync();
+  for (int64_t i = (int64_t)blockIdx.x * 256 + threadIdx.x; i < n; i += (int64_t)gridDim.x * 256) {
+    const float4 v = a[i];
+    *reinterpret_cast<uint2*>(out + i * 4) = make_uint2(pack_bf16x2(v.x, v.y), pack_bf16x2(v.z, v.w));
+  }
+}
+
+struct BwdShared {
+  uint64_t kv_full[2];
+  uint64_t s_done, x_done, drain;
+  uint32_t tmem_base;
+  int abort_flag;
+};
+
+// dS = P * (dP - D) for 128 columns of one TMEM lane: S at tS, dP at tP.
+// Column e is a key (dq kernel: kTransposed false, the lane is a query row
+// with lse2_row / dd_row) or a query row (dkdv kernel: kTransposed, the lane
+// is a key; per-column lse2 / dd / token from shared memory). P (kept only
+// when kTransposed) goes over the first 64 columns at tS, dS over the first 64 at tP (dkdv) or
+// over tS (dq). Masked entries: keys beyond `lim` (dq), or keys above the
+// column's token (dkdv).
+template <bool kTransposed>
+__device__ __forceinline__ void bwd_softmax_grad(uint32_t tS, uint32_t tP, float c2, float lse2_row, float dd_row,
+                                                 int lim, const float* s_lse2, const float* s_dd, const int* s_tok,
+                                                 int key) {
+#pragma unroll
+  for (int ch = 0; ch < 4; ++ch) {
+    uint32_t sr[32], pr[32];
+    tmem_ld32(tS + ch * 32, sr);
+    tmem_ld32(tP + ch * 32, pr);
+    tmem_ld_wait();
+    uint32_t pk[16], dk[16];
+#pragma unroll
+    for (int e = 0; e < 32; e += 2) {
+      float pv[2], dv[2];
+#pragma unroll
+      for (int u = 0; u < 2; ++u) {
+        const int col = ch * 32 + e + u;
+        const float l2 = kTransposed ? s_lse2[col] : lse2_row;
+        const float d = kTransposed ? s_dd[col] : dd_row;
+        float pe = ex2_approx(fmaf(__uint_as_float(sr[e + u]), c2, -l2));
+        const bool masked = kTransposed ? (key > s_tok[col]) : (col > lim);
+        if (masked) pe = 0.f;
+        pv[u] = pe;
+        dv[u] = pe * (__uint_as_float(pr[e + u]) - d);
+      }
+      pk[e >> 1] = pack_bf16x2(pv[0], pv[1]);
+      dk[e >> 1] = pack_bf16x2(dv[0], dv[1]);
+    }
+    if (kTransposed) {
+      tmem_st16(tS + ch * 16, pk);
+      tmem_st16(tP + ch * 16, dk);
+    } else {
+      tmem_st16(tS + ch * 16, dk);
+    }
+  }
+}
+
+// grid = number of SMs, 128 threads (thread = query row = TMEM lane), items
+// (unit, tile) taken with a fixed stride. TMEM: S 0..127 (then dS as bf16
+// over 0..63), dP 128..255, dQ 256..383.
+__global__ void __launch_bounds__(kBwdThreads, 1)
+    bwd_dq_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant__ CUtensorMap tmap_v,
+                  AttnParams ap, BwdParams p) {
+  grid_dependency_sync();
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sQ = smem;
+  uint8_t* sdO = sQ + kTileBytes;
+  uint8_t* sK = sdO + kTileBytes;         // 2 stages
+  uint8_t* sV = sK + 2 * kTileBytes;      // 2 stages
+  BwdShared* sh = reinterpret_cast<BwdShared*>(sV + 2 * kTileBytes);
+  const int warp = threadIdx.x >> 5;
+  const int row = threadIdx.x;
+  if (threadIdx.x == 0) {
+    mbar_init(&sh->kv_full[0], 1);
+    mbar_init(&sh->kv_full[1], 1);
+    mbar_init(&sh->s_done, 1);
+    mbar_init(&sh->x_done, 1);
+    mbar_init(&sh->drain, 1);
+    sh->abort_flag = 0;
+    fence_barrier_init();
+    prefetch_tmap(&tmap_k);
+    prefetch_tmap(&tmap_v);
+  }
+  if (warp == 0) {
+    tmem_alloc(&sh->tmem_base, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = sh->tmem_base;
+  const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+  volatile int* ab = &sh->abort_flag;
+  const uint32_t idesc_s = idesc_bf16_f32(128, 128, false);
+  const uint32_t idesc_o = idesc_bf16_f32(128, 128, true);
+  const uint64_t dQd = sdesc_sw128(smem_u32(sQ), 16, 1024);
+  const uint64_t ddOd = sdesc_sw128(smem_u32(sdO), 16, 1024);
+  const uint64_t dK = sdesc_sw128(smem_u32(sK), 16, 1024);
+  const uint64_t dV = sdesc_sw128(smem_u32(sV), 16, 1024);
+  const uint64_t dKmn = sdesc_sw128(smem_u32(sK), kHalfBytes, 1024);
+  const float c2 = p.scale_log2;
+  const int n_units = ap.hdr[1];
+  uint32_t kv_it = 0;   // K/V loads issued before this item
+  uint32_t mma_it = 0;  // steps done (phase of s_done / x_done)
+  uint32_t loaded = 0;    // K/V loads issued in total (thread 0)
+  uint32_t consumed = 0;  // K/V loads waited for
+  auto load_kv = [&](uint32_t L, const UnitInfo& u, int s) {  // thread 0
+    const int st = L & 1;
+    const int key = (int)(u.key0 + (int64_t)s * kTile);
+    mbar_arrive_expect_tx(&sh->kv_full[st], 2 * kTileBytes);
+    tma_load_3d(sK + st * kTileBytes, &tmap_k, &sh->kv_full[st], 0, u.g, key);
+    tma_load_3d(sK + st * kTileBytes + kHalfBytes, &tmap_k, &sh->kv_full[st], 64, u.g, key);
+    tma_load_3d(sV + st * kTileBytes, &tmap_v, &sh->kv_full[st], 0, u.g, key);
+    tma_load_3d(sV + st * kTileBytes + kHalfBytes, &tmap_v, &sh->kv_full[st], 64, u.g, key);
+    loaded = L + 1;
+  };
+  for (int item = blockIdx.x; item < 2 * n_units; item += gridDim.x) {
+    const UnitInfo u = decode_unit(ap, item >> 1);
+    const int x = item & 1;
+    if (x == 1 && !u.has_b) continue;
+    // this thread's query row
+    int64_t t = -1;
+    int h = 0;
+    if (row < u.rows[x]) {
+      if (u.own) {
+        t = u.tq[x] + row;
+        h = u.h[x];
+      } else {
+        const int rr = __ldg(ap.list + u.list0[x] + row);
+        t = p.w0 + rr / p.G;
+        h = u.g * p.G + rr % p.G;
+      }
+    }
+    const int64_t off = t >= 0 ? (t * p.Hq + h) * kHeadDim : -1;
+    gather_row(smem_u32(sQ), p.q, off, row);
+    gather_row(smem_u32(sdO), p.dout, off, row);
+    float lse2_r = INFINITY, dd_r = 0.f;  // a missing row gets P = 0
+    if (t >= 0) {
+      lse2_r = __ldg(p.lse2 + (int64_t)h * p.S + t);
+      dd_r = __ldg(p.dd + (int64_t)h * p.S + t);
+    }
+    if (threadIdx.x == 0) {
+      load_kv(kv_it, u, 0);
+      if (u.nsteps > 1) load_kv(kv_it + 1, u, 1);
+    }
+    cp_async_wait_all();
+    fence_proxy_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const int dstep = u.own ? u.diag[x] : u.nsteps;
+    for (int s = 0; s < u.nsteps; ++s) {
+      const uint32_t L = kv_it + s;
+      const int st = L & 1;
+      if (!mbar_wait(&sh->kv_full[st], (L >> 1) & 1, ab)) goto done;
+      consumed = L + 1;
+      tc_fence_after();
+      if (warp == 0) {
+        if (elect_one()) {
+          const uint64_t k0 = dK + ((st * kTileBytes) >> 4), v0 = dV + ((st * kTileBytes) >> 4);
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk) {
+            const uint32_t o = ((kk >> 2) * kHalfBytes + (kk & 3) * 32) >> 4;
+            mma_bf16_ss(tmem, dQd + o, k0 + o, idesc_s, kk > 0 ? 1u : 0u);
+          }
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk) {
+            const uint32_t o = ((kk >> 2) * kHalfBytes + (kk & 3) * 32) >> 4;
+            mma_bf16_ss(tmem + 128, ddOd + o, v0 + o, idesc_s, kk > 0 ? 1u : 0u);
+          }
+          mma_commit(&sh->s_done);
+        }
+        __syncwarp();
+      }
+      if (!mbar_wait(&sh->s_done, mma_it & 1, ab)) goto done;
+      __syncwarp();
+      tc_fence_after();
+      {
+        // keys e > lim are masked on and after the diagonal step
+        const int lim = s >= dstep ? row - (s - dstep) * kTile : kTile;
+        bwd_softmax_grad<false>(tmem + lane_off, tmem + lane_off + 128, c2, lse2_r, dd_r, lim, nullptr, nullptr,
+                                nullptr, 0);
+      }
+      tmem_st_wait();
+      tc_fence_before();
+      __syncthreads();
+      tc_fence_after();
+      if (warp == 0) {
+        if (elect_one()) {
+          const uint64_t k0 = dKmn + ((st * kTileBytes) >> 4);
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk)
+            mma_bf16_ts(tmem + 256, tmem + kk * 8, k0 + ((kk * 2048) >> 4), idesc_o, (s > 0 || kk > 0) ? 1u : 0u);
+          mma_commit(&sh->x_done);
+        }
+        __syncwarp();
+      }
+      if (!mbar_wait(&sh->x_done, mma_it & 1, ab)) goto done;
+      tc_fence_after();
+      ++mma_it;
+      // K/V stage st is free again
+      if (threadIdx.x == 0 && s + 2 < u.nsteps) load_kv(L + 2, u, s + 2);
+    }
+    kv_it += u.nsteps;
+    {
+      // the item's c * dQ as an fp16 partial
+      __half* dst = nullptr;
+      if (t >= 0)
+        dst = u.own ? ap.own_o + ((t - p.w0) * p.Hq + h) * kHeadDim
+                    : ap.part_o + ((int64_t)u.list0[x] + row) * kHeadDim;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        uint32_t o[32];
+        tmem_ld32(tmem + lane_off + 256 + c * 32, o);
+        tmem_ld_wait();
+        if (dst) {
+#pragma unroll
+          for (int e = 0; e < 32; e += 8) {
+            uint4 hv;
+            hv.x = pack_half2(__uint_as_float(o[e]) * p.scale, __uint_as_float(o[e + 1]) * p.scale);
+            hv.y = pack_half2(__uint_as_float(o[e + 2]) * p.scale, __uint_as_float(o[e + 3]) * p.scale);
+            hv.z = pack_half2(__uint_as_float(o[e + 4]) * p.scale, __uint_as_float(o[e + 5]) * p.scale);
+            hv.w = pack_half2(__uint_as_float(o[e + 6]) * p.scale, __uint_as_float(o[e + 7]) * p.scale);
+            *reinterpret_cast<uint4*>(dst + c * 32 + e) = hv;
+          }
+        }
+      }
+      // the next item's MMAs overwrite TMEM and shared memory
+      tc_fence_before();
+      __syncthreads();
+      tc_fence_after();
+    }
+  }
+done:
+  if (*ab) {
+    // after a timeout: let issued copies and products land first (bounded)
+    volatile int keep = 0;
+    if (threadIdx.x == 0)
+      for (uint32_t L = consumed; L < loaded; ++L) mbar_wait(&sh->kv_full[L & 1], (L >> 1) & 1, &keep, (1ull << 28));
+    if (warp == 0) {
+      if (elect_one()) mma_commit(&sh->drain);
+      __syncwarp();
+      mbar_wait(&sh->drain, 0, &keep, (1ull << 28));
+    }
+  }
+  cp_async_wait_all();
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// dQ of the window's rows: the sum of each row's fp16 partials in a fixed
+// order (selected past blocks ascending, own block last), already scaled by
+// c. grid ceil(wlen*Hq/8), 256 threads: one warp per row (t, h).
+__global__ void __launch_bounds__(256) bwd_dq_reduce_kernel(const int32_t* __restrict__ sel,
+                                                            const uint32_t* __restrict__ flags,
+                                                            const int32_t* __restrict__ wordbase,
+                                                            const __half* __restrict__ part_o,
+                                                            const __half* __restrict__ own_o, WindowGeom w,
+                                                            __nv_bfloat16* __restrict__ dq) {
+  grid_dependency_sync();
+  const int lane = threadIdx.x & 31;
+  const int64_t row = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
+  if (row >= w.wlen * w.Hq) return;
+  const int64_t tl = row / w.Hq;
+  const int h = (int)(row % w.Hq);
+  const int64_t t = w.w0 + tl;
+  const int g = h / w.G, hl = h % w.G;
+  const int bt = (int)(t / w.B);
+  const int64_t rr = tl * w.G + hl;
+  const int64_t word = rr >> 5;
+  const uint32_t below = (1u << (rr & 31)) - 1u;
+  const int32_t* srow = sel + ((int64_t)h * w.S + t) * w.k_eff;
+  const int P = w.k_eff - 1;
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int i = 0; i < P; ++i) {
+    const int j = __ldg(srow + i);
+    if (j < 0 || j >= bt) continue;
+    const int64_t f = ((int64_t)g * w.nbp + j) * w.wwords + word;
+    const int64_t pos = (int64_t)__ldg(wordbase + f) + __popc(__ldg(flags + f) & below);
+    const float4 o = load_half4(part_o + pos * kHeadDim + lane * 4);
+    acc.x += o.x;
+    acc.y += o.y;
+    acc.z += o.z;
+    acc.w += o.w;
+  }
+  const float4 o = load_half4(own_o + (tl * w.Hq + h) * kHeadDim + lane * 4);
+  acc.x += o.x;
+  acc.y += o.y;
+  acc.z += o.z;
+  acc.w += o.w;
+  *reinterpret_cast<uint2*>(dq + (t * w.Hq + h) * kHeadDim + lane * 4) =
+      make_uint2(pack_bf16x2(acc.x, acc.y), pack_bf16x2(acc.z, acc.w));
+}
+
+struct DkdvParams {
+  const int32_t* list;    // the window's router lists (group-rows)
+  const int32_t* cnt;     // [Hkv][nbp] routed rows per bucket (valid when routed)
+  const int32_t* loff;    // [Hkv][nbp] first list slot per bucket
+  float* dk_acc;          // [S][Hkv][128] fp32
+  float* dv_acc;          // [S][Hkv][128] fp32
+  int routed;             // the window has router lists
+};
+
+struct DkdvShared {
+  uint64_t kv_full;
+  uint64_t s_done, x_done, drain;
+  uint32_t tmem_base;
+  int abort_flag;
+  float lse2[2][kTile];
+  float dd[2][kTile];
+  int tok[2][kTile];
+};
+
+// grid (nblocks, B/128, Hkv), 128 threads (thread = key = TMEM lane for the
+// products; thread = row for the gathers). TMEM: S^T 0..127 (P^T as bf16 over
+// 0..63), dP^T 128..255 (dS^T over 128..191), dV 256..383, dK 384..511.
+__global__ void __launch_bounds__(kBwdThreads, 1)
+    bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant__ CUtensorMap tmap_v,
+                    BwdParams p, DkdvParams d) {
+  grid_dependency_sync();
+  const int j = blockIdx.x, kt = blockIdx.y, g = blockIdx.z;
+  const int64_t kstart = (int64_t)j * p.B + (int64_t)kt * kTile;
+  if (kstart >= p.S) return;
+  // the rows that attend these keys in this window: the bucket's routed rows,
+  // then the own block's rows from the tile's first key on (causal)
+  const int nr = (d.routed && j < p.nbp) ? __ldg(d.cnt + g * p.nbp + j) : 0;
+  const int lbase = (d.routed && j < p.nbp) ? __ldg(d.loff + g * p.nbp + j) : 0;
+  const int64_t t_lo = max(kstart, p.w0);
+  const int64_t t_hi = min(min((int64_t)(j + 1) * p.B, p.S), p.w0 + p.wlen);
+  const int64_t n_own = t_hi > t_lo ? (t_hi - t_lo) * p.G : 0;
+  const int64_t own_rr0 = (t_lo - p.w0) * p.G;
+  const int n_rt = (nr + kTile - 1) / kTile;
+  const int ntiles = n_rt + (int)((n_own + kTile - 1) / kTile);
+  if (ntiles == 0) return;
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sK = smem;
+  uint8_t* sV = sK + kTileBytes;
+  uint8_t* sQ = sV + kTileBytes;   // 2 stages
+  uint8_t* sdO = sQ + 2 * kTileBytes;  // 2 stages
+  DkdvShared* sh = reinterpret_cast<DkdvShared*>(sdO + 2 * kTileBytes);
+  const int warp = threadIdx.x >> 5;
+  if (threadIdx.x == 0) {
+    mbar_init(&sh->kv_full, 1);
+    mbar_init(&sh->s_done, 1);
+    mbar_init(&sh->x_done, 1);
+    mbar_init(&sh->drain, 1);
+    sh->abort_flag = 0;
+    fence_barrier_init();
+    mbar_arrive_expect_tx(&sh->kv_full, 2 * kTileBytes);
+    tma_load_3d(sK, &tmap_k, &sh->kv_full, 0, g, (int)kstart);
+    tma_load_3d(sK + kHalfBytes, &tmap_k, &sh->kv_full, 64, g, (int)kstart);
+    tma_load_3d(sV, &tmap_v, &sh->kv_full, 0, g, (int)kstart);
+    tma_load_3d(sV + kHalfBytes, &tmap_v, &sh->kv_full, 64, g, (int)kstart);
+  }
+  if (warp == 0) {
+    tmem_alloc(&sh->tmem_base, 512);
+    tmem_relinquish();
+  }
+  // rows of tile i into stage i & 1 (thread = row)
+  auto gather = [&](int i) {
+    const int st = i & 1;
+    const int r = threadIdx.x;
+    int64_t t = -1;
+    int h = 0;
+    if (i < n_rt) {
+      if (i * kTile + r < nr) {
+        const int rr = __ldg(d.list + lbase + i * kTile + r);
+        t = p.w0 + rr / p.G;
+        h = g * p.G + rr % p.G;
+      }
+    } else {
+      const int64_t k = (int64_t)(i - n_rt) * kTile + r;
+      if (k < n_own) {
+        const int64_t rr = own_rr0 + k;
+        t = p.w0 + rr / p.G;
+        h = g * p.G + (int)(rr % p.G);
+      }
+    }
+    const int64_t off = t >= 0 ? (t * p.Hq + h) * kHeadDim : -1;
+    gather_row(smem_u32(sQ + st * kTileBytes), p.q, off, r);
+    gather_row(smem_u32(sdO + st * kTileBytes), p.dout, off, r);
+    cp_async_commit();
+    sh->lse2[st][r] = t >= 0 ? __ldg(p.lse2 + (int64_t)h * p.S + t) : INFINITY;
+    sh->dd[st][r] = t >= 0 ? __ldg(p.dd + (int64_t)h * p.S + t) : 0.f;
+    // routed rows lie past the block: no key of it is masked for them
+    sh->tok[st][r] = (t < 0 || i < n_rt) ? 0x7fffffff : (int)t;
+  };
+  gather(0);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = sh->tmem_base;
+  const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+  volatile int* ab = &sh->abort_flag;
+  const uint32_t idesc_s = idesc_bf16_f32(128, 128, false);
+  const uint32_t idesc_o = idesc_bf16_f32(128, 128, true);
+  const uint64_t dKd = sdesc_sw128(smem_u32(sK), 16, 1024);
+  const uint64_t dVd = sdesc_sw128(smem_u32(sV), 16, 1024);
+  const uint64_t dQk = sdesc_sw128(smem_u32(sQ), 16, 1024);
+  const uint64_t ddOk = sdesc_sw128(smem_u32(sdO), 16, 1024);
+  const uint64_t dQm = sdesc_sw128(smem_u32(sQ), kHalfBytes, 1024);
+  const uint64_t ddOm = sdesc_sw128(smem_u32(sdO), kHalfBytes, 1024);
+  const float c2 = p.scale_log2;
+  const int key = (int)kstart + threadIdx.x;
+  bool kv_ready = false;
+  for (int i = 0; i < ntiles; ++i) {
+    const int st = i & 1;
+    // the other stage was last read by tile i-1's products, which are done
+    if (i + 1 < ntiles) {
+      gather(i + 1);
+      cp_async_wait_group<1>();
+    } else {
+      cp_async_wait_group<0>();
+    }
+    fence_proxy_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (!kv_ready) {
+      if (!mbar_wait(&sh->kv_full, 0, ab)) goto done;
+      kv_ready = true;
+      tc_fence_after();
+    }
+    if (warp == 0) {
+      if (elect_one()) {
+        const uint64_t q0 = dQk + ((st * kTileBytes) >> 4), o0 = ddOk + ((st * kTileBytes) >> 4);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint32_t o = ((kk >> 2) * kHalfBytes + (kk & 3) * 32) >> 4;
+          mma_bf16_ss(tmem, dKd + o, q0 + o, idesc_s, kk > 0 ? 1u : 0u);
+        }
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint32_t o = ((kk >> 2) * kHalfBytes + (kk & 3) * 32) >> 4;
+          mma_bf16_ss(tmem + 128, dVd + o, o0 + o, idesc_s, kk > 0 ? 1u : 0u);
+        }
+        mma_commit(&sh->s_done);
+      }
+      __syncwarp();
+    }
+    if (!mbar_wait(&sh->s_done, i & 1, ab)) goto done;
+    __syncwarp();
+    tc_fence_after();
+    bwd_softmax_grad<true>(tmem + lane_off, tmem + lane_off + 128, c2, 0.f, 0.f, 0, sh->lse2[st], sh->dd[st],
+                           sh->tok[st], key);
+    tmem_st_wait();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 0) {
+      if (elect_one()) {
+        const uint64_t o0 = ddOm + ((st * kTileBytes) >> 4), q0 = dQm + ((st * kTileBytes) >> 4);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          mma_bf16_ts(tmem + 256, tmem + kk * 8, o0 + ((kk * 2048) >> 4), idesc_o, (i > 0 || kk > 0) ? 1u : 0u);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          mma_bf16_ts(tmem + 384, tmem + 128 + kk * 8, q0 + ((kk * 2048) >> 4), idesc_o,
+                      (i > 0 || kk > 0) ? 1u : 0u);
+        mma_commit(&sh->x_done);
+      }
+      __syncwarp();
+    }
+    if (!mbar_wait(&sh->x_done, i & 1, ab)) goto done;
+    tc_fence_after();
+  }
+  {
+    // dV and c * dK of this thread's key, added to the window's accumulators
+    const bool valid = key < p.S;
+    float* dv = d.dv_acc + ((int64_t)key * p.Hkv + g) * kHeadDim;
+    float* dk = d.dk_acc + ((int64_t)key * p.Hkv + g) * kHeadDim;
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      uint32_t a[32], b[32];
+      tmem_ld32(tmem + lane_off + 256 + c * 32, a);
+      tmem_ld32(tmem + lane_off + 384 + c * 32, b);
+      tmem_ld_wait();
+      if (valid) {
+#pragma unroll
+        for (int e = 0; e < 32; e += 4) {
+          float4 x = *reinterpret_cast<float4*>(dv + c * 32 + e);
+          x.x += __uint_as_float(a[e]);
+          x.y += __uint_as_float(a[e + 1]);
+          x.z += __uint_as_float(a[e + 2]);
+          x.w += __uint_as_float(a[e + 3]);
+          *reinterpret_cast<float4*>(dv + c * 32 + e) = x;
+          float4 y = *reinterpret_cast<float4*>(dk + c * 32 + e);
+          y.x = fmaf(__uint_as_float(b[e]), p.scale, y.x);
+          y.y = fmaf(__uint_as_float(b[e + 1]), p.scale, y.y);
+          y.z = fmaf(__uint_as_float(b[e + 2]), p.scale, y.z);
+          y.w = fmaf(__uint_as_float(b[e + 3]), p.scale, y.w);
+          *reinterpret_cast<float4*>(dk + c * 32 + e) = y;
+        }
+      }
+    }
+  }
+done:
+  if (*ab) {
+    volatile int keep = 0;
+    if (threadIdx.x == 0) mbar_wait(&sh->kv_full, 0, &keep, (1ull << 28));
+    if (warp == 0) {
+      if (elect_one()) mma_commit(&sh->drain);
+      __syncwarp();
+      mbar_wait(&sh->drain, 0, &keep, (1ull << 28));
+    }
+  }
+  cp_async_wait_all();
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+}  // namespace moba

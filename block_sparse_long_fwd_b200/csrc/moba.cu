@@ -16,6 +16,7 @@
 #include <vector>
 
 #include "attn.cuh"
+#include "bwd.cuh"
 #include "common.cuh"
 #include "gate_tc.cuh"
 #include "merge.cuh"
@@ -67,6 +68,10 @@ int device_info(DeviceInfo* out) {
     if (d.sm100) {
       MOBA_CUDA(cudaFuncSetAttribute(moba::attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      moba::kAttnSmemBytes));
+      MOBA_CUDA(cudaFuncSetAttribute(moba::bwd_dq_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     moba::kBwdSmemBytes));
+      MOBA_CUDA(cudaFuncSetAttribute(moba::bwd_dkdv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     moba::kBwdSmemBytes));
       MOBA_CUDA(cudaFuncSetAttribute(moba::gate_tc_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      moba::kGateSmemBytes));
       MOBA_CUDA(cudaFuncSetAttribute(moba::gate_tc_kernel<4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -372,7 +377,17 @@ void launch_pool(const Plan& p, const void* k, float* kmean, int splits, cudaStr
 // Optional per-stage device timing: an event after every stage, tagged with
 // the stage it closes (-1 opens a call); elapsed times between consecutive
 // events are summed per stage when the profile ends.
-enum Stage { kPool = 0, kGate = 1, kRoute = 2, kAttn = 3, kMerge = 4, kNumStages = 5 };
+enum Stage {
+  kPool = 0,
+  kGate = 1,
+  kRoute = 2,
+  kAttn = 3,
+  kMerge = 4,
+  kBwdPrep = 5,
+  kBwdDq = 6,
+  kBwdDkdv = 7,
+  kNumStages = 8
+};
 
 struct StageTimer {
   bool on = false;
@@ -413,6 +428,62 @@ struct StageTimer {
 
 thread_local StageTimer g_timer;
 
+moba::WindowGeom window_geom(const Plan& p, int64_t w0) {
+  moba::WindowGeom wg;
+  wg.S = p.S;
+  wg.Hq = p.Hq;
+  wg.Hkv = p.Hkv;
+  wg.G = p.G;
+  wg.B = p.B;
+  wg.k_eff = p.k_eff;
+  wg.nbp = p.nbp;
+  wg.w0 = w0;
+  wg.wlen = std::min(p.W, p.S - w0);
+  wg.q0 = p.q0;
+  wg.wwords = (wg.wlen * p.G + 31) / 32;
+  wg.pair_tokens = pair_tokens(p) ? 1 : 0;
+  return wg;
+}
+
+// Some row of the window can have a past block.
+bool window_routed(const Plan& p, const moba::WindowGeom& wg) {
+  return p.P > 0 && p.nbp > 0 && (wg.w0 + wg.wlen) > p.B;
+}
+
+// The router for one query window (flags, counts, scan, fill); returns the
+// number of kernels launched.
+int launch_route(const Plan& p, const moba::WindowGeom& wg, bool routed, uint8_t* ws, cudaStream_t st) {
+  const int32_t* sel = reinterpret_cast<const int32_t*>(ws + p.o_sel);
+  uint32_t* flags = reinterpret_cast<uint32_t*>(ws + p.o_flags);
+  int32_t* wordbase = reinterpret_cast<int32_t*>(ws + p.o_wordbase);
+  int32_t* cnt = reinterpret_cast<int32_t*>(ws + p.o_cnt);
+  int32_t* loff = reinterpret_cast<int32_t*>(ws + p.o_loff);
+  int32_t* toff = reinterpret_cast<int32_t*>(ws + p.o_toff);
+  int32_t* list = reinterpret_cast<int32_t*>(ws + p.o_list);
+  int4* tiles = reinterpret_cast<int4*>(ws + p.o_tiles);
+  int32_t* hdr = reinterpret_cast<int32_t*>(ws + p.o_hdr);
+  const int nbk = p.Hkv * p.nbp;
+  int n = 0;
+  if (routed) {
+    dim3 gf((unsigned)((wg.wwords + 7) / 8), p.Hkv);
+    launch_chained(moba::route_flags_kernel, gf, dim3(256), 0, st, sel, wg, flags);
+    dim3 gb(p.nbp, p.Hkv);
+    launch_chained(moba::route_count_kernel, gb, dim3(256), 0, st, static_cast<const uint32_t*>(flags), wg, cnt);
+    n += 2;
+  }
+  launch_chained(moba::route_scan_kernel, dim3(1), dim3(1024), 0, st, static_cast<const int32_t*>(cnt),
+                 routed ? nbk : 0, wg, loff, toff, tiles, hdr);
+  ++n;
+  if (routed) {
+    dim3 gb(p.nbp, p.Hkv);
+    launch_chained(moba::route_fill_kernel, gb, dim3(256), 0, st, static_cast<const uint32_t*>(flags),
+                   static_cast<const int32_t*>(cnt), static_cast<const int32_t*>(loff),
+                   static_cast<const int32_t*>(toff), wg, wordbase, list, tiles);
+    ++n;
+  }
+  return n;
+}
+
 int run_forward(const Plan& p, const DeviceInfo& dev, const void* q, const void* k, const void* v, void* out,
                 float* lse, uint8_t* ws, cudaStream_t st) {
   StageTimer* tm = &g_timer;
@@ -423,9 +494,6 @@ int run_forward(const Plan& p, const DeviceInfo& dev, const void* q, const void*
   int32_t* sel = reinterpret_cast<int32_t*>(ws + p.o_sel);
   uint32_t* flags = reinterpret_cast<uint32_t*>(ws + p.o_flags);
   int32_t* wordbase = reinterpret_cast<int32_t*>(ws + p.o_wordbase);
-  int32_t* cnt = reinterpret_cast<int32_t*>(ws + p.o_cnt);
-  int32_t* loff = reinterpret_cast<int32_t*>(ws + p.o_loff);
-  int32_t* toff = reinterpret_cast<int32_t*>(ws + p.o_toff);
   int32_t* list = reinterpret_cast<int32_t*>(ws + p.o_list);
   int4* tiles = reinterpret_cast<int4*>(ws + p.o_tiles);
   int32_t* hdr = reinterpret_cast<int32_t*>(ws + p.o_hdr);
@@ -454,7 +522,6 @@ int run_forward(const Plan& p, const DeviceInfo& dev, const void* q, const void*
   }
   tm->mark(kGate);
 
-  const int nbk = p.Hkv * p.nbp;
   moba::AttnParams ap;
   ap.q = static_cast<const __nv_bfloat16*>(q);
   ap.list = list;
@@ -472,37 +539,9 @@ int run_forward(const Plan& p, const DeviceInfo& dev, const void* q, const void*
   ap.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)moba::kHeadDim));
 
   for (int64_t w0 = p.wbase; w0 < p.S; w0 += p.W) {
-    moba::WindowGeom wg;
-    wg.S = p.S;
-    wg.Hq = p.Hq;
-    wg.Hkv = p.Hkv;
-    wg.G = p.G;
-    wg.B = p.B;
-    wg.k_eff = p.k_eff;
-    wg.nbp = p.nbp;
-    wg.w0 = w0;
-    wg.wlen = std::min(p.W, p.S - w0);
-    wg.q0 = p.q0;
-    wg.wwords = (wg.wlen * p.G + 31) / 32;
-    wg.pair_tokens = pair_tokens(p) ? 1 : 0;
-    const bool routed = p.P > 0 && p.nbp > 0 && (w0 + wg.wlen) > p.B;
-    if (routed) {
-      dim3 gf((unsigned)((wg.wwords + 7) / 8), p.Hkv);
-      launch_chained(moba::route_flags_kernel, gf, dim3(256), 0, st, static_cast<const int32_t*>(sel), wg, flags);
-      dim3 gb(p.nbp, p.Hkv);
-      launch_chained(moba::route_count_kernel, gb, dim3(256), 0, st, static_cast<const uint32_t*>(flags), wg, cnt);
-      tm->count(2);
-    }
-    launch_chained(moba::route_scan_kernel, dim3(1), dim3(1024), 0, st, static_cast<const int32_t*>(cnt), routed ? nbk : 0,
-                   wg, loff, toff, tiles, hdr);
-    tm->count(1);
-    if (routed) {
-      dim3 gb(p.nbp, p.Hkv);
-      launch_chained(moba::route_fill_kernel, gb, dim3(256), 0, st, static_cast<const uint32_t*>(flags),
-                     static_cast<const int32_t*>(cnt), static_cast<const int32_t*>(loff),
-                     static_cast<const int32_t*>(toff), wg, wordbase, list, tiles);
-      tm->count(1);
-    }
+    const moba::WindowGeom wg = window_geom(p, w0);
+    const bool routed = window_routed(p, wg);
+    tm->count(launch_route(p, wg, routed, ws, st));
     tm->mark(kRoute);
     ap.w0 = w0;
     launch_chained(moba::attn_kernel, dim3(dev.sms), dim3(moba::kAttnThreads), moba::kAttnSmemBytes, st, tmk, tmv, ap);
@@ -527,6 +566,142 @@ int run_forward(const Plan& p, const DeviceInfo& dev, const void* q, const void*
     else launch_chained(moba::merge_kernel<0>, mg, dim3(256), 0, st, mp);
     tm->count(1);
     tm->mark(kMerge);
+  }
+  MOBA_CUDA(cudaGetLastError());
+  return MOBA_OK;
+}
+
+// Scratch of the backward pass beyond the forward's layout: lse * log2(e)
+// and D = rowsum(dO * O) per row, and fp32 dK / dV accumulators.
+struct BwdLayout {
+  size_t o_lse2, o_dd, o_dk, o_dv, total;
+};
+
+BwdLayout bwd_layout(const Plan& p) {
+  BwdLayout b;
+  Carve c;
+  c.off = p.total;
+  b.o_lse2 = c.take((size_t)p.Hq * p.S * 4);
+  b.o_dd = c.take((size_t)p.Hq * p.S * 4);
+  b.o_dk = c.take((size_t)p.S * p.Hkv * moba::kHeadDim * 4);
+  b.o_dv = c.take((size_t)p.S * p.Hkv * moba::kHeadDim * 4);
+  b.total = c.off;
+  return b;
+}
+
+// The backward launch sequence: the forward's pool, gate and router (so the
+// selection is the forward's), then per query window the dQ partials, their
+// reduction and the window's dK / dV contributions; the fp32 accumulators are
+// cast to bf16 at the end.
+int run_backward(const Plan& p, const BwdLayout& bl, const DeviceInfo& dev, const void* q, const void* k,
+                 const void* v, const void* o, const float* lse, const void* dout, void* dq, void* dk, void* dv,
+                 uint8_t* ws, cudaStream_t st) {
+  StageTimer* tm = &g_timer;
+  tm->st = st;
+  if (tm->on) tm->calls++;
+  float* kmean = reinterpret_cast<float*>(ws + p.o_kmean);
+  int32_t* sel = reinterpret_cast<int32_t*>(ws + p.o_sel);
+  float* lse2 = reinterpret_cast<float*>(ws + bl.o_lse2);
+  float* dd = reinterpret_cast<float*>(ws + bl.o_dd);
+  float* dk_acc = reinterpret_cast<float*>(ws + bl.o_dk);
+  float* dv_acc = reinterpret_cast<float*>(ws + bl.o_dv);
+  CUtensorMap tmk, tmv;
+  int rc = make_kv_map(&tmk, k, p.S, p.Hkv);
+  if (rc) return rc;
+  rc = make_kv_map(&tmv, v, p.S, p.Hkv);
+  if (rc) return rc;
+
+  tm->mark(-1);
+  if (p.P > 0 && p.k_eff < p.nb && p.nbp > 0) {
+    launch_pool(p, k, kmean, p.splits, st);
+    tm->count(1);
+    tm->mark(kPool);
+  }
+  {
+    const int n = launch_gate(p, q, kmean, p.splits, reinterpret_cast<__nv_bfloat16*>(ws + p.o_khi),
+                              reinterpret_cast<__nv_bfloat16*>(ws + p.o_klo), sel, st);
+    if (n < 0) return -n;
+    tm->count(n);
+  }
+  tm->mark(kGate);
+  {
+    const int64_t rows = p.S * p.Hq;
+    launch_chained(moba::bwd_prep_kernel, dim3((unsigned)((rows + 7) / 8)), dim3(256), 0, st,
+                   static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dout), lse, p.S, p.Hq,
+                   lse2, dd);
+    const int64_t n4 = 2 * p.S * p.Hkv * moba::kHeadDim / 4;  // dK then dV accumulators, contiguous
+    launch_chained(moba::bwd_zero_kernel, dim3((unsigned)std::min<int64_t>((n4 + 255) / 256, dev.sms * 16)),
+                   dim3(256), 0, st, reinterpret_cast<float4*>(dk_acc), n4);
+    tm->count(2);
+  }
+  tm->mark(kBwdPrep);
+
+  moba::AttnParams ap;
+  ap.q = static_cast<const __nv_bfloat16*>(q);
+  ap.list = reinterpret_cast<const int32_t*>(ws + p.o_list);
+  ap.units = reinterpret_cast<const int4*>(ws + p.o_tiles);
+  ap.hdr = reinterpret_cast<int32_t*>(ws + p.o_hdr);
+  ap.part_o = reinterpret_cast<__half*>(ws + p.o_part_o);
+  ap.part_lse = reinterpret_cast<float*>(ws + p.o_part_lse);
+  ap.own_o = reinterpret_cast<__half*>(ws + p.o_own_o);
+  ap.own_lse = reinterpret_cast<float*>(ws + p.o_own_lse);
+  ap.S = p.S;
+  ap.q0 = 0;
+  ap.Hq = p.Hq;
+  ap.G = p.G;
+  ap.B = p.B;
+  ap.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)moba::kHeadDim));
+  moba::BwdParams bp;
+  bp.q = static_cast<const __nv_bfloat16*>(q);
+  bp.dout = static_cast<const __nv_bfloat16*>(dout);
+  bp.lse2 = lse2;
+  bp.dd = dd;
+  bp.S = p.S;
+  bp.Hq = p.Hq;
+  bp.Hkv = p.Hkv;
+  bp.G = p.G;
+  bp.B = p.B;
+  bp.nbp = p.nbp;
+  bp.scale_log2 = ap.scale_log2;
+  bp.scale = (float)(1.0 / std::sqrt((double)moba::kHeadDim));
+  moba::DkdvParams dp;
+  dp.list = ap.list;
+  dp.cnt = reinterpret_cast<const int32_t*>(ws + p.o_cnt);
+  dp.loff = reinterpret_cast<const int32_t*>(ws + p.o_loff);
+  dp.dk_acc = dk_acc;
+  dp.dv_acc = dv_acc;
+
+  for (int64_t w0 = 0; w0 < p.S; w0 += p.W) {
+    const moba::WindowGeom wg = window_geom(p, w0);
+    const bool routed = window_routed(p, wg);
+    tm->count(launch_route(p, wg, routed, ws, st));
+    tm->mark(kRoute);
+    ap.w0 = w0;
+    bp.w0 = w0;
+    bp.wlen = wg.wlen;
+    launch_chained(moba::bwd_dq_kernel, dim3(dev.sms), dim3(moba::kBwdThreads), moba::kBwdSmemBytes, st, tmk, tmv,
+                   ap, bp);
+    launch_chained(moba::bwd_dq_reduce_kernel, dim3((unsigned)((wg.wlen * p.Hq + 7) / 8)), dim3(256), 0, st,
+                   static_cast<const int32_t*>(sel), reinterpret_cast<const uint32_t*>(ws + p.o_flags),
+                   reinterpret_cast<const int32_t*>(ws + p.o_wordbase), static_cast<const __half*>(ap.part_o),
+                   static_cast<const __half*>(ap.own_o), wg, static_cast<__nv_bfloat16*>(dq));
+    tm->count(2);
+    tm->mark(kBwdDq);
+    dp.routed = routed ? 1 : 0;
+    launch_chained(moba::bwd_dkdv_kernel, dim3((unsigned)p.nb, (unsigned)(p.B / moba::kTile), (unsigned)p.Hkv),
+                   dim3(moba::kBwdThreads), moba::kBwdSmemBytes, st, tmk, tmv, bp, dp);
+    tm->count(1);
+    tm->mark(kBwdDkdv);
+  }
+  {
+    const int64_t n4 = p.S * p.Hkv * moba::kHeadDim / 4;
+    const dim3 gc((unsigned)std::min<int64_t>((n4 + 255) / 256, dev.sms * 16));
+    launch_chained(moba::bwd_cast_kernel, gc, dim3(256), 0, st, reinterpret_cast<const float4*>(dk_acc),
+                   static_cast<__nv_bfloat16*>(dk), n4);
+    launch_chained(moba::bwd_cast_kernel, gc, dim3(256), 0, st, reinterpret_cast<const float4*>(dv_acc),
+                   static_cast<__nv_bfloat16*>(dv), n4);
+    tm->count(2);
+    tm->mark(kBwdDkdv);
   }
   MOBA_CUDA(cudaGetLastError());
   return MOBA_OK;
@@ -768,6 +943,30 @@ int moba_fwd_varlen(const void* q, const void* k, const void* v, const int64_t* 
                     int heads_kv, int head_dim, int block_size, int topk, void* out, float* lse,
                     cudaStream_t stream) {
   return varlen_impl(q, k, v, cu_seqlens, batch, heads_q, heads_kv, head_dim, block_size, topk, out, lse, stream);
+}
+
+int moba_bwd(const void* q, const void* k, const void* v, const void* out, const float* lse, const void* dout,
+             int64_t seqlen, int heads_q, int heads_kv, int head_dim, int block_size, int topk, void* dq, void* dk,
+             void* dv, cudaStream_t stream) {
+  g_err.clear();
+  if (!q || !k || !v || !out || !lse || !dout || !dq || !dk || !dv)
+    return fail(MOBA_ERR_INVALID_ARG, "null pointer argument");
+  int rc = check_shape(seqlen, heads_q, heads_kv, head_dim, block_size, topk);
+  if (rc) return rc;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(lse) || !aligned16(dout) ||
+      !aligned16(dq) || !aligned16(dk) || !aligned16(dv))
+    return fail(MOBA_ERR_INVALID_ARG, "device buffers must be 16-byte aligned");
+  DeviceInfo dev;
+  rc = device_info(&dev);
+  if (rc) return rc;
+  Plan p;
+  rc = make_plan(&p, seqlen, 0, heads_q, heads_kv, block_size, topk);
+  if (rc) return rc;
+  const BwdLayout bl = bwd_layout(p);
+  const Runner run = [&](uint8_t* ws, cudaStream_t st) {
+    return run_backward(p, bl, dev, q, k, v, out, lse, dout, dq, dk, dv, ws, st);
+  };
+  return direct_run(bl.total, run, stream);
 }
 
 int moba_profile_begin(void) {

@@ -165,6 +165,33 @@ int moba_fwd_varlen(const void* q, const void* k, const void* v,
                     void* out, float* lse, cudaStream_t stream);
 
 /*
+ * moba_bwd - the gradient of moba_fwd: dq, dk, dv from the upstream gradient
+ * dout, with the gate's choice held fixed (the top-k choice is piecewise
+ * constant; the block means receive no gradient). Needed to train MoBA on
+ * from a full-attention model ("MoBA (Mixture of Block Attention)" project
+ * summary, "Key Features"; "Efficient Long-Context Attention with MoBA", "How
+ * MoBA Works"). Per q head h of kv head g, with P the forward's attention
+ * weights over the row's attended keys and c = 1/sqrt(head_dim):
+ *   dv = sum over g's q heads of P^T dout, dS = P * (dout v^T - rowsum(dout * out)),
+ *   dq = c dS k, dk = sum over g's q heads of c dS^T q.
+ * The pool, gate and router run again, so the selection is the forward's.
+ *
+ * q, k, v    device bf16, as passed to moba_fwd.
+ * out, lse   device, moba_fwd's outputs for them (bf16 [S][heads_q][128],
+ *            fp32 [heads_q][S]); P is rebuilt from lse.
+ * dout       device bf16 [S][heads_q][head_dim].
+ * dq         device bf16 output [S][heads_q][head_dim].
+ * dk, dv     device bf16 outputs [S][heads_kv][head_dim].
+ * Shapes and checks as moba_fwd; every pointer 16-byte aligned. Scratch is
+ * stream-ordered, as for moba_fwd (dK / dV accumulate in fp32 scratch).
+ * The result is deterministic: every sum runs in a fixed order.
+ */
+int moba_bwd(const void* q, const void* k, const void* v, const void* out,
+             const float* lse, const void* dout, int64_t seqlen, int heads_q,
+             int heads_kv, int head_dim, int block_size, int topk, void* dq,
+             void* dk, void* dv, cudaStream_t stream);
+
+/*
  * moba_fwd_host - moba_fwd on HOST buffers (same layouts): copies q, k, v to
  * the device, runs the forward pass and copies out and lse back, all on
  * `stream`, and synchronises the stream before returning. Host buffers that
@@ -199,9 +226,11 @@ int moba_gate(const void* q, const float* kmean, int64_t seqlen, int heads_q,
  * thread. After moba_profile_begin(), every moba_fwd call also records CUDA
  * events on its stream between its stages (no extra synchronisation).
  * moba_profile_end() waits for the last recorded event, writes the summed
- * milliseconds per stage to stage_ms[0..4] = {pool, gate, route, attention,
- * merge}, the number of kernels launched to *launches and the number of
- * forward calls to *calls, then turns the timing off. Returns a moba_status.
+ * milliseconds per stage to stage_ms[0..7] = {pool, gate, route, attention,
+ * merge, bwd_prep, bwd_dq, bwd_dkdv} (the last three for moba_bwd calls),
+ * the number of kernels launched to *launches and the number of forward and
+ * backward calls to *calls, then turns the timing off. Returns a
+ * moba_status.
  */
 int moba_profile_begin(void);
 int moba_profile_end(float* stage_ms, int* launches, int* calls);
