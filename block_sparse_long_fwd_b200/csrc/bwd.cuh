@@ -40,6 +40,7 @@
 namespace moba {
 
 constexpr int kBwdThreads = 128;
+constexpr int kDkdvThreads = 256;
 constexpr int kBwdSmemBytes = 6 * kTileBytes + 1024 + 4096;
 
 struct BwdParams {
@@ -149,21 +150,34 @@ __device__ __forceinline__ void bwd_softmax_grad(uint32_t tS, uint32_t tP, float
     tmem_ld_wait();
     uint32_t pk[16], dk[16];
 #pragma unroll
-    for (int e = 0; e < 32; e += 2) {
-      float pv[2], dv[2];
+    for (int e4 = 0; e4 < 32; e4 += 4) {
+      // per-column values, four at a time (shared-memory broadcasts)
+      float l2[4], dd4[4];
+      int tk[4];
+      if (kTransposed) {
+        const float4 a = *reinterpret_cast<const float4*>(s_lse2 + ch * 32 + e4);
+        const float4 b = *reinterpret_cast<const float4*>(s_dd + ch * 32 + e4);
+        const int4 c = *reinterpret_cast<const int4*>(s_tok + ch * 32 + e4);
+        l2[0] = a.x, l2[1] = a.y, l2[2] = a.z, l2[3] = a.w;
+        dd4[0] = b.x, dd4[1] = b.y, dd4[2] = b.z, dd4[3] = b.w;
+        tk[0] = c.x, tk[1] = c.y, tk[2] = c.z, tk[3] = c.w;
+      }
+      float pv[4], dv[4];
 #pragma unroll
-      for (int u = 0; u < 2; ++u) {
-        const int col = ch * 32 + e + u;
-        const float l2 = kTransposed ? s_lse2[col] : lse2_row;
-        const float d = kTransposed ? s_dd[col] : dd_row;
-        float pe = ex2_approx(fmaf(__uint_as_float(sr[e + u]), c2, -l2));
-        const bool masked = kTransposed ? (key > s_tok[col]) : (col > lim);
+      for (int u = 0; u < 4; ++u) {
+        const int col = ch * 32 + e4 + u;
+        const float l = kTransposed ? l2[u] : lse2_row;
+        const float d = kTransposed ? dd4[u] : dd_row;
+        float pe = ex2_approx(fmaf(__uint_as_float(sr[e4 + u]), c2, -l));
+        const bool masked = kTransposed ? (key > tk[u]) : (col > lim);
         if (masked) pe = 0.f;
         pv[u] = pe;
-        dv[u] = pe * (__uint_as_float(pr[e + u]) - d);
+        dv[u] = pe * (__uint_as_float(pr[e4 + u]) - d);
       }
-      pk[e >> 1] = pack_bf16x2(pv[0], pv[1]);
-      dk[e >> 1] = pack_bf16x2(dv[0], dv[1]);
+      pk[e4 >> 1] = pack_bf16x2(pv[0], pv[1]);
+      pk[(e4 >> 1) + 1] = pack_bf16x2(pv[2], pv[3]);
+      dk[e4 >> 1] = pack_bf16x2(dv[0], dv[1]);
+      dk[(e4 >> 1) + 1] = pack_bf16x2(dv[2], dv[3]);
     }
     if (kTransposed) {
       tmem_st16(tS + ch * 16, pk);
@@ -430,19 +444,25 @@ struct DkdvShared {
   uint64_t s_done, x_done, drain;
   uint32_t tmem_base;
   int abort_flag;
-  float lse2[2][kTile];
-  float dd[2][kTile];
-  int tok[2][kTile];
+  alignas(16) float lse2[2][kTile];
+  alignas(16) float dd[2][kTile];
+  alignas(16) int tok[2][kTile];
 };
 
-// grid (nblocks, B/128, Hkv), 128 threads (thread = key = TMEM lane for the
-// products; thread = row for the gathers). TMEM: S^T 0..127 (P^T as bf16 over
-// 0..63), dP^T 128..255 (dS^T over 128..191), dV 256..383, dK 384..511.
-__global__ void __launch_bounds__(kBwdThreads, 1)
+// grid (B/128 * nblocks * Hkv), key tile fastest, so the CTAs of one block
+// (which gather the same query rows) run together and share them in L2; 128
+// threads: two warps per TMEM lane quadrant (lane = key), each taking 64 of
+// the tile's 128 query columns; for the gathers, threads 0..127 copy Q rows
+// and 128..255 dO rows. TMEM: S^T 0..127 (P^T as bf16 over 0..63), dP^T
+// 128..255 (dS^T over 128..191), dV 256..383, dK 384..511.
+__global__ void __launch_bounds__(kDkdvThreads, 1)
     bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant__ CUtensorMap tmap_v,
                     BwdParams p, DkdvParams d) {
   grid_dependency_sync();
-  const int j = blockIdx.x, kt = blockIdx.y, g = blockIdx.z;
+  const int ntb = p.B / kTile;
+  const int kt = (int)(blockIdx.x % ntb);
+  const int j = (int)((blockIdx.x / ntb) % (p.nbp + 1));
+  const int g = (int)(blockIdx.x / ((int64_t)ntb * (p.nbp + 1)));
   const int64_t kstart = (int64_t)j * p.B + (int64_t)kt * kTile;
   if (kstart >= p.S) return;
   // the rows that attend these keys in this window: the bucket's routed rows,
@@ -482,17 +502,22 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     tmem_alloc(&sh->tmem_base, 512);
     tmem_relinquish();
   }
-  // rows of tile i into stage i & 1 (thread = row)
-  auto gather = [&](int i) {
-    const int st = i & 1;
-    const int r = threadIdx.x;
-    int64_t t = -1;
-    int h = 0;
+  // Row r (= this thread) of tile i: its (t, h) from the router list or the
+  // own range; t = -1 past the tile's rows. The list entry is read a tile
+  // ahead (list_ahead) so the gather never waits on it.
+  const int grow = threadIdx.x & (kTile - 1);  // the row this thread gathers
+  auto list_entry = [&](int i) -> int {
+    const int r = grow;
+    return (i < n_rt && i * kTile + r < nr) ? __ldg(d.list + lbase + i * kTile + r) : -1;
+  };
+  auto row_of = [&](int i, int lst, int64_t& t, int& h) {
+    const int r = grow;
+    t = -1;
+    h = 0;
     if (i < n_rt) {
-      if (i * kTile + r < nr) {
-        const int rr = __ldg(d.list + lbase + i * kTile + r);
-        t = p.w0 + rr / p.G;
-        h = g * p.G + rr % p.G;
+      if (lst >= 0) {
+        t = p.w0 + lst / p.G;
+        h = g * p.G + lst % p.G;
       }
     } else {
       const int64_t k = (int64_t)(i - n_rt) * kTile + r;
@@ -502,21 +527,43 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         h = g * p.G + (int)(rr % p.G);
       }
     }
-    const int64_t off = t >= 0 ? (t * p.Hq + h) * kHeadDim : -1;
-    gather_row(smem_u32(sQ + st * kTileBytes), p.q, off, r);
-    gather_row(smem_u32(sdO + st * kTileBytes), p.dout, off, r);
-    cp_async_commit();
-    sh->lse2[st][r] = t >= 0 ? __ldg(p.lse2 + (int64_t)h * p.S + t) : INFINITY;
-    sh->dd[st][r] = t >= 0 ? __ldg(p.dd + (int64_t)h * p.S + t) : 0.f;
-    // routed rows lie past the block: no key of it is masked for them
-    sh->tok[st][r] = (t < 0 || i < n_rt) ? 0x7fffffff : (int)t;
   };
-  gather(0);
+  // rows of tile i into stage i & 1 (cp.async, one commit group); its
+  // per-row values come back in registers and are stored later
+  auto gather = [&](int i, int lst, float& l2, float& dv, int& tk) {
+    const int st = i & 1;
+    int64_t t;
+    int h;
+    row_of(i, lst, t, h);
+    const int64_t off = t >= 0 ? (t * p.Hq + h) * kHeadDim : -1;
+    if (threadIdx.x < kTile)
+      gather_row(smem_u32(sQ + st * kTileBytes), p.q, off, grow);
+    else
+      gather_row(smem_u32(sdO + st * kTileBytes), p.dout, off, grow);
+    cp_async_commit();
+    l2 = t >= 0 ? __ldg(p.lse2 + (int64_t)h * p.S + t) : INFINITY;
+    dv = t >= 0 ? __ldg(p.dd + (int64_t)h * p.S + t) : 0.f;
+    // routed rows lie past the block: no key of it is masked for them
+    tk = (t < 0 || i < n_rt) ? 0x7fffffff : (int)t;
+  };
+  auto store_meta = [&](int i, float l2, float dv, int tk) {
+    if (threadIdx.x >= kTile) return;
+    const int st = i & 1;
+    sh->lse2[st][grow] = l2;
+    sh->dd[st][grow] = dv;
+    sh->tok[st][grow] = tk;
+  };
+  float m_l2, m_dd;
+  int m_tok;
+  gather(0, list_entry(0), m_l2, m_dd, m_tok);
+  store_meta(0, m_l2, m_dd, m_tok);
+  int list_ahead = list_entry(1);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = sh->tmem_base;
-  const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+  const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
+  const int hf = warp >> 2;  // this warp's half of the query columns / of the epilogue
   volatile int* ab = &sh->abort_flag;
   const uint32_t idesc_s = idesc_bf16_f32(128, 128, false);
   const uint32_t idesc_o = idesc_bf16_f32(128, 128, true);
@@ -527,17 +574,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   const uint64_t dQm = sdesc_sw128(smem_u32(sQ), kHalfBytes, 1024);
   const uint64_t ddOm = sdesc_sw128(smem_u32(sdO), kHalfBytes, 1024);
   const float c2 = p.scale_log2;
-  const int key = (int)kstart + threadIdx.x;
+  const int key = (int)kstart + (warp & 3) * 32 + (threadIdx.x & 31);
   bool kv_ready = false;
   for (int i = 0; i < ntiles; ++i) {
     const int st = i & 1;
-    // the other stage was last read by tile i-1's products, which are done
-    if (i + 1 < ntiles) {
-      gather(i + 1);
-      cp_async_wait_group<1>();
-    } else {
-      cp_async_wait_group<0>();
-    }
+    // tile i's rows (the only commit group in flight) and per-row values
+    cp_async_wait_group<0>();
     fence_proxy_async_smem();
     tc_fence_before();
     __syncthreads();
@@ -564,11 +606,57 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       }
       __syncwarp();
     }
+    // while the tensor core works: the next tile's rows into the other stage
+    // (its last readers, tile i-1's products, are done) and the list entries
+    // of the one after
+    const bool more = i + 1 < ntiles;
+    if (more) {
+      gather(i + 1, list_ahead, m_l2, m_dd, m_tok);
+      list_ahead = list_entry(i + 2);
+    }
     if (!mbar_wait(&sh->s_done, i & 1, ab)) goto done;
     __syncwarp();
     tc_fence_after();
-    bwd_softmax_grad<true>(tmem + lane_off, tmem + lane_off + 128, c2, 0.f, 0.f, 0, sh->lse2[st], sh->dd[st],
-                           sh->tok[st], key);
+    {
+      // this warp's 64 columns of S^T and dP^T into registers, then (once
+      // every warp has read its columns) P^T and dS^T back as bf16
+      uint32_t sr[64], pr[64];
+      tmem_ld32(tmem + lane_off + hf * 64, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
+      tmem_ld32(tmem + lane_off + hf * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
+      tmem_ld32(tmem + lane_off + 128 + hf * 64, *reinterpret_cast<uint32_t(*)[32]>(&pr[0]));
+      tmem_ld32(tmem + lane_off + 128 + hf * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&pr[32]));
+      tmem_ld_wait();
+      uint32_t pk[32], dk[32];
+      const float* cl2 = sh->lse2[st] + hf * 64;
+      const float* cdd = sh->dd[st] + hf * 64;
+      const int* ctk = sh->tok[st] + hf * 64;
+#pragma unroll
+      for (int e4 = 0; e4 < 64; e4 += 4) {
+        const float4 a = *reinterpret_cast<const float4*>(cl2 + e4);
+        const float4 b = *reinterpret_cast<const float4*>(cdd + e4);
+        const int4 c = *reinterpret_cast<const int4*>(ctk + e4);
+        const float l2[4] = {a.x, a.y, a.z, a.w}, dd4[4] = {b.x, b.y, b.z, b.w};
+        const int tk[4] = {c.x, c.y, c.z, c.w};
+        float pv[4], dv[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          float pe = ex2_approx(fmaf(__uint_as_float(sr[e4 + u]), c2, -l2[u]));
+          if (key > tk[u]) pe = 0.f;
+          pv[u] = pe;
+          dv[u] = pe * (__uint_as_float(pr[e4 + u]) - dd4[u]);
+        }
+        pk[e4 >> 1] = pack_bf16x2(pv[0], pv[1]);
+        pk[(e4 >> 1) + 1] = pack_bf16x2(pv[2], pv[3]);
+        dk[e4 >> 1] = pack_bf16x2(dv[0], dv[1]);
+        dk[(e4 >> 1) + 1] = pack_bf16x2(dv[2], dv[3]);
+      }
+      if (more) store_meta(i + 1, m_l2, m_dd, m_tok);
+      __syncthreads();  // every warp has read its S^T / dP^T columns
+      tmem_st16(tmem + lane_off + hf * 32, pk);
+      tmem_st16(tmem + lane_off + hf * 32 + 16, pk + 16);
+      tmem_st16(tmem + lane_off + 128 + hf * 32, dk);
+      tmem_st16(tmem + lane_off + 128 + hf * 32 + 16, dk + 16);
+    }
     tmem_st_wait();
     tc_fence_before();
     __syncthreads();
@@ -592,30 +680,24 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   }
   {
     // dV and c * dK of this thread's key, added to the window's accumulators
+    // warps 0-3 take dV, warps 4-7 c * dK
     const bool valid = key < p.S;
-    float* dv = d.dv_acc + ((int64_t)key * p.Hkv + g) * kHeadDim;
-    float* dk = d.dk_acc + ((int64_t)key * p.Hkv + g) * kHeadDim;
+    float* dst = (hf ? d.dk_acc : d.dv_acc) + ((int64_t)key * p.Hkv + g) * kHeadDim;
+    const float mul = hf ? p.scale : 1.f;
 #pragma unroll
     for (int c = 0; c < 4; ++c) {
-      uint32_t a[32], b[32];
-      tmem_ld32(tmem + lane_off + 256 + c * 32, a);
-      tmem_ld32(tmem + lane_off + 384 + c * 32, b);
+      uint32_t a[32];
+      tmem_ld32(tmem + lane_off + 256 + hf * 128 + c * 32, a);
       tmem_ld_wait();
       if (valid) {
 #pragma unroll
         for (int e = 0; e < 32; e += 4) {
-          float4 x = *reinterpret_cast<float4*>(dv + c * 32 + e);
-          x.x += __uint_as_float(a[e]);
-          x.y += __uint_as_float(a[e + 1]);
-          x.z += __uint_as_float(a[e + 2]);
-          x.w += __uint_as_float(a[e + 3]);
-          *reinterpret_cast<float4*>(dv + c * 32 + e) = x;
-          float4 y = *reinterpret_cast<float4*>(dk + c * 32 + e);
-          y.x = fmaf(__uint_as_float(b[e]), p.scale, y.x);
-          y.y = fmaf(__uint_as_float(b[e + 1]), p.scale, y.y);
-          y.z = fmaf(__uint_as_float(b[e + 2]), p.scale, y.z);
-          y.w = fmaf(__uint_as_float(b[e + 3]), p.scale, y.w);
-          *reinterpret_cast<float4*>(dk + c * 32 + e) = y;
+          float4 x = *reinterpret_cast<float4*>(dst + c * 32 + e);
+          x.x = fmaf(__uint_as_float(a[e]), mul, x.x);
+          x.y = fmaf(__uint_as_float(a[e + 1]), mul, x.y);
+          x.z = fmaf(__uint_as_float(a[e + 2]), mul, x.z);
+          x.w = fmaf(__uint_as_float(a[e + 3]), mul, x.w);
+          *reinterpret_cast<float4*>(dst + c * 32 + e) = x;
         }
       }
     }

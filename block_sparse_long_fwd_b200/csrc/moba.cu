@@ -688,8 +688,8 @@ int run_backward(const Plan& p, const BwdLayout& bl, const DeviceInfo& dev, cons
     tm->count(2);
     tm->mark(kBwdDq);
     dp.routed = routed ? 1 : 0;
-    launch_chained(moba::bwd_dkdv_kernel, dim3((unsigned)p.nb, (unsigned)(p.B / moba::kTile), (unsigned)p.Hkv),
-                   dim3(moba::kBwdThreads), moba::kBwdSmemBytes, st, tmk, tmv, bp, dp);
+    launch_chained(moba::bwd_dkdv_kernel, dim3((unsigned)((int64_t)(p.B / moba::kTile) * p.nb * p.Hkv)),
+                   dim3(moba::kDkdvThreads), moba::kBwdSmemBytes, st, tmk, tmv, bp, dp);
     tm->count(1);
     tm->mark(kBwdDkdv);
   }
