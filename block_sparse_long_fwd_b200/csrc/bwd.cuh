@@ -40,7 +40,6 @@
 namespace moba {
 
 constexpr int kBwdThreads = 128;
-constexpr int kDkdvThreads = 256;
 constexpr int kBwdSmemBytes = 6 * kTileBytes + 1024 + 4096;
 
 struct BwdParams {
@@ -439,22 +438,56 @@ struct DkdvParams {
   int routed;             // the window has router lists
 };
 
+// dK / dV pipeline: query rows come in 64-row slices through a 4-stage
+// shared-memory ring; TMEM holds two slice buffers (S^T and dP^T, 64
+// columns each) beside the dV and dK accumulators, so the products of one
+// slice run while the element-wise step of the other is under way.
+constexpr int kSlice = 64;
+constexpr uint32_t kSliceHalf = kSlice * 128;    // one 64-channel half of a slice: 8 KB
+constexpr uint32_t kSliceBytes = 2 * kSliceHalf;  // 16 KB
+constexpr int kDkdvStages = 4;
+constexpr int kDkdvThreads = 352;  // warps 0-7 element-wise, 8 MMA + TMA, 9-10 gather
+
 struct DkdvShared {
-  uint64_t kv_full;
-  uint64_t s_done, x_done, drain;
+  uint64_t kv_full, drain, all_done;
+  uint64_t q_full[kDkdvStages], q_empty[kDkdvStages];
+  uint64_t s_full[2], p_full[2], x_done[2];
   uint32_t tmem_base;
   int abort_flag;
-  alignas(16) float lse2[2][kTile];
-  alignas(16) float dd[2][kTile];
-  alignas(16) int tok[2][kTile];
+  alignas(16) float lse2[kDkdvStages][kSlice];
+  alignas(16) float dd[kDkdvStages][kSlice];
+  alignas(16) int tok[kDkdvStages][kSlice];
 };
 
+// Row (t, h) of q / dO into row r of a 64-row slice (two 8 KB halves,
+// 128-byte swizzle); a missing row (off < 0) is zero-filled.
+__device__ __forceinline__ void gather_slice_row(uint32_t dst0, const __nv_bfloat16* base, int64_t off, int r) {
+  const bool valid = off >= 0;
+  const __nv_bfloat16* src = valid ? base + off : base;
+#pragma unroll
+  for (int c16 = 0; c16 < 16; ++c16) {
+    const int half = c16 >> 3, c = c16 & 7;
+    cp_async_16(dst0 + half * kSliceHalf + r * 128 + ((c ^ (r & 7)) << 4), src + (valid ? c16 * 8 : 0),
+                valid ? 16u : 0u);
+  }
+}
+
 // grid (B/128 * nblocks * Hkv), key tile fastest, so the CTAs of one block
-// (which gather the same query rows) run together and share them in L2; 128
-// threads: two warps per TMEM lane quadrant (lane = key), each taking 64 of
-// the tile's 128 query columns; for the gathers, threads 0..127 copy Q rows
-// and 128..255 dO rows. TMEM: S^T 0..127 (P^T as bf16 over 0..63), dP^T
-// 128..255 (dS^T over 128..191), dV 256..383, dK 384..511.
+// (which gather the same query rows) run together and share them in L2.
+// One CTA owns 128 keys (TMEM lane = key) and loops over 64-row slices of
+// the rows that attend them in this window: the bucket's router list, then
+// the own block's rows from the tile's first key on (causal). Per slice m
+// (TMEM buffer b = m & 1, ring stage m % 4):
+//   warp 8      S^T = K Q^T and dP^T = V dO^T (N = 64) into buffer b; once
+//               the slice's P^T and dS^T are back, dV += P^T dO and
+//               dK += dS^T Q (TS MMAs, dO and Q as MN-major B operands),
+//               which also free the ring stage and the buffer
+//   warps 0-3 / 4-7 (even / odd slices): P^T = 2^(S^T c - lse2) (0 where
+//               masked), dS^T = P^T (dP^T - D), both back as bf16 over the
+//               first half of S^T and of dP^T
+//   warps 9-10  gather the slice's Q and dO rows (cp.async) and per-row
+//               values, two slices in flight.
+// TMEM: buffer b at 128b (S^T 0..63, dP^T 64..127), dV 256..383, dK 384..511.
 __global__ void __launch_bounds__(kDkdvThreads, 1)
     bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant__ CUtensorMap tmap_v,
                     BwdParams p, DkdvParams d) {
@@ -465,257 +498,267 @@ __global__ void __launch_bounds__(kDkdvThreads, 1)
   const int g = (int)(blockIdx.x / ((int64_t)ntb * (p.nbp + 1)));
   const int64_t kstart = (int64_t)j * p.B + (int64_t)kt * kTile;
   if (kstart >= p.S) return;
-  // the rows that attend these keys in this window: the bucket's routed rows,
-  // then the own block's rows from the tile's first key on (causal)
   const int nr = (d.routed && j < p.nbp) ? __ldg(d.cnt + g * p.nbp + j) : 0;
   const int lbase = (d.routed && j < p.nbp) ? __ldg(d.loff + g * p.nbp + j) : 0;
   const int64_t t_lo = max(kstart, p.w0);
   const int64_t t_hi = min(min((int64_t)(j + 1) * p.B, p.S), p.w0 + p.wlen);
   const int64_t n_own = t_hi > t_lo ? (t_hi - t_lo) * p.G : 0;
   const int64_t own_rr0 = (t_lo - p.w0) * p.G;
-  const int n_rt = (nr + kTile - 1) / kTile;
-  const int ntiles = n_rt + (int)((n_own + kTile - 1) / kTile);
-  if (ntiles == 0) return;
+  const int n_rs = (nr + kSlice - 1) / kSlice;
+  const int ns = n_rs + (int)((n_own + kSlice - 1) / kSlice);
+  if (ns == 0) return;
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sK = smem;
   uint8_t* sV = sK + kTileBytes;
-  uint8_t* sQ = sV + kTileBytes;   // 2 stages
-  uint8_t* sdO = sQ + 2 * kTileBytes;  // 2 stages
-  DkdvShared* sh = reinterpret_cast<DkdvShared*>(sdO + 2 * kTileBytes);
-  const int warp = threadIdx.x >> 5;
+  uint8_t* sQ = sV + kTileBytes;                      // kDkdvStages slices
+  uint8_t* sdO = sQ + kDkdvStages * kSliceBytes;      // kDkdvStages slices
+  DkdvShared* sh = reinterpret_cast<DkdvShared*>(sdO + kDkdvStages * kSliceBytes);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
     mbar_init(&sh->kv_full, 1);
-    mbar_init(&sh->s_done, 1);
-    mbar_init(&sh->x_done, 1);
     mbar_init(&sh->drain, 1);
+    mbar_init(&sh->all_done, 1);
+    for (int i = 0; i < kDkdvStages; ++i) {
+      mbar_init(&sh->q_full[i], 64);
+      mbar_init(&sh->q_empty[i], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&sh->s_full[b], 1);
+      mbar_init(&sh->p_full[b], 128);
+      mbar_init(&sh->x_done[b], 1);
+    }
     sh->abort_flag = 0;
     fence_barrier_init();
-    mbar_arrive_expect_tx(&sh->kv_full, 2 * kTileBytes);
-    tma_load_3d(sK, &tmap_k, &sh->kv_full, 0, g, (int)kstart);
-    tma_load_3d(sK + kHalfBytes, &tmap_k, &sh->kv_full, 64, g, (int)kstart);
-    tma_load_3d(sV, &tmap_v, &sh->kv_full, 0, g, (int)kstart);
-    tma_load_3d(sV + kHalfBytes, &tmap_v, &sh->kv_full, 64, g, (int)kstart);
   }
-  if (warp == 0) {
+  if (warp == 8) {
     tmem_alloc(&sh->tmem_base, 512);
     tmem_relinquish();
   }
-  // Row r (= this thread) of tile i: its (t, h) from the router list or the
-  // own range; t = -1 past the tile's rows. The list entry is read a tile
-  // ahead (list_ahead) so the gather never waits on it.
-  const int grow = threadIdx.x & (kTile - 1);  // the row this thread gathers
-  auto list_entry = [&](int i) -> int {
-    const int r = grow;
-    return (i < n_rt && i * kTile + r < nr) ? __ldg(d.list + lbase + i * kTile + r) : -1;
-  };
-  auto row_of = [&](int i, int lst, int64_t& t, int& h) {
-    const int r = grow;
-    t = -1;
-    h = 0;
-    if (i < n_rt) {
-      if (lst >= 0) {
-        t = p.w0 + lst / p.G;
-        h = g * p.G + lst % p.G;
-      }
-    } else {
-      const int64_t k = (int64_t)(i - n_rt) * kTile + r;
-      if (k < n_own) {
-        const int64_t rr = own_rr0 + k;
-        t = p.w0 + rr / p.G;
-        h = g * p.G + (int)(rr % p.G);
-      }
-    }
-  };
-  // rows of tile i into stage i & 1 (cp.async, one commit group); its
-  // per-row values come back in registers and are stored later
-  auto gather = [&](int i, int lst, float& l2, float& dv, int& tk) {
-    const int st = i & 1;
-    int64_t t;
-    int h;
-    row_of(i, lst, t, h);
-    const int64_t off = t >= 0 ? (t * p.Hq + h) * kHeadDim : -1;
-    if (threadIdx.x < kTile)
-      gather_row(smem_u32(sQ + st * kTileBytes), p.q, off, grow);
-    else
-      gather_row(smem_u32(sdO + st * kTileBytes), p.dout, off, grow);
-    cp_async_commit();
-    l2 = t >= 0 ? __ldg(p.lse2 + (int64_t)h * p.S + t) : INFINITY;
-    dv = t >= 0 ? __ldg(p.dd + (int64_t)h * p.S + t) : 0.f;
-    // routed rows lie past the block: no key of it is masked for them
-    tk = (t < 0 || i < n_rt) ? 0x7fffffff : (int)t;
-  };
-  auto store_meta = [&](int i, float l2, float dv, int tk) {
-    if (threadIdx.x >= kTile) return;
-    const int st = i & 1;
-    sh->lse2[st][grow] = l2;
-    sh->dd[st][grow] = dv;
-    sh->tok[st][grow] = tk;
-  };
-  float m_l2, m_dd;
-  int m_tok;
-  gather(0, list_entry(0), m_l2, m_dd, m_tok);
-  store_meta(0, m_l2, m_dd, m_tok);
-  int list_ahead = list_entry(1);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = sh->tmem_base;
-  const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
-  const int hf = warp >> 2;  // this warp's half of the query columns / of the epilogue
   volatile int* ab = &sh->abort_flag;
-  const uint32_t idesc_s = idesc_bf16_f32(128, 128, false);
-  const uint32_t idesc_o = idesc_bf16_f32(128, 128, true);
-  const uint64_t dKd = sdesc_sw128(smem_u32(sK), 16, 1024);
-  const uint64_t dVd = sdesc_sw128(smem_u32(sV), 16, 1024);
-  const uint64_t dQk = sdesc_sw128(smem_u32(sQ), 16, 1024);
-  const uint64_t ddOk = sdesc_sw128(smem_u32(sdO), 16, 1024);
-  const uint64_t dQm = sdesc_sw128(smem_u32(sQ), kHalfBytes, 1024);
-  const uint64_t ddOm = sdesc_sw128(smem_u32(sdO), kHalfBytes, 1024);
-  const float c2 = p.scale_log2;
-  const int key = (int)kstart + (warp & 3) * 32 + (threadIdx.x & 31);
-  bool kv_ready = false;
-  for (int i = 0; i < ntiles; ++i) {
-    const int st = i & 1;
-    // tile i's rows (the only commit group in flight) and per-row values
-    cp_async_wait_group<0>();
-    fence_proxy_async_smem();
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-    if (!kv_ready) {
-      if (!mbar_wait(&sh->kv_full, 0, ab)) goto done;
-      kv_ready = true;
+
+  if (warp < 8) {
+    // ------------------------------------------------ element-wise, then the epilogue
+    const int X = warp >> 2;  // slices m with m % 2 == X, TMEM buffer X
+    const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
+    const uint32_t tb = tmem + lane_off + 128 * X;
+    const int key = (int)kstart + (warp & 3) * 32 + lane;
+    const float c2 = p.scale_log2;
+    for (int m = X; m < ns; m += 2) {
+      const int st = m % kDkdvStages;
+      if (!mbar_wait(&sh->s_full[X], (m >> 1) & 1, ab)) goto ew_done;
+      if (!mbar_wait(&sh->q_full[st], (m / kDkdvStages) & 1, ab)) goto ew_done;  // per-row values
+      __syncwarp();
       tc_fence_after();
-    }
-    if (warp == 0) {
-      if (elect_one()) {
-        const uint64_t q0 = dQk + ((st * kTileBytes) >> 4), o0 = ddOk + ((st * kTileBytes) >> 4);
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          const uint32_t o = ((kk >> 2) * kHalfBytes + (kk & 3) * 32) >> 4;
-          mma_bf16_ss(tmem, dKd + o, q0 + o, idesc_s, kk > 0 ? 1u : 0u);
-        }
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          const uint32_t o = ((kk >> 2) * kHalfBytes + (kk & 3) * 32) >> 4;
-          mma_bf16_ss(tmem + 128, dVd + o, o0 + o, idesc_s, kk > 0 ? 1u : 0u);
-        }
-        mma_commit(&sh->s_done);
-      }
-      __syncwarp();
-    }
-    // while the tensor core works: the next tile's rows into the other stage
-    // (its last readers, tile i-1's products, are done) and the list entries
-    // of the one after
-    const bool more = i + 1 < ntiles;
-    if (more) {
-      gather(i + 1, list_ahead, m_l2, m_dd, m_tok);
-      list_ahead = list_entry(i + 2);
-    }
-    if (!mbar_wait(&sh->s_done, i & 1, ab)) goto done;
-    __syncwarp();
-    tc_fence_after();
-    {
-      // this warp's 64 columns of S^T and dP^T into registers, then (once
-      // every warp has read its columns) P^T and dS^T back as bf16
       uint32_t sr[64], pr[64];
-      tmem_ld32(tmem + lane_off + hf * 64, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
-      tmem_ld32(tmem + lane_off + hf * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
-      tmem_ld32(tmem + lane_off + 128 + hf * 64, *reinterpret_cast<uint32_t(*)[32]>(&pr[0]));
-      tmem_ld32(tmem + lane_off + 128 + hf * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&pr[32]));
+      tmem_ld32(tb, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
+      tmem_ld32(tb + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
+      tmem_ld32(tb + 64, *reinterpret_cast<uint32_t(*)[32]>(&pr[0]));
+      tmem_ld32(tb + 96, *reinterpret_cast<uint32_t(*)[32]>(&pr[32]));
       tmem_ld_wait();
-      uint32_t pk[32], dk[32];
-      const float* cl2 = sh->lse2[st] + hf * 64;
-      const float* cdd = sh->dd[st] + hf * 64;
-      const int* ctk = sh->tok[st] + hf * 64;
 #pragma unroll
-      for (int e4 = 0; e4 < 64; e4 += 4) {
-        const float4 a = *reinterpret_cast<const float4*>(cl2 + e4);
-        const float4 b = *reinterpret_cast<const float4*>(cdd + e4);
-        const int4 c = *reinterpret_cast<const int4*>(ctk + e4);
-        const float l2[4] = {a.x, a.y, a.z, a.w}, dd4[4] = {b.x, b.y, b.z, b.w};
-        const int tk[4] = {c.x, c.y, c.z, c.w};
-        float pv[4], dv[4];
+      for (int ch = 0; ch < 2; ++ch) {
+        // columns 32*ch.. (slice rows); their bf16 pairs go to columns 16*ch..,
+        // which this thread has already read
+        uint32_t pk[16], dk[16];
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          float pe = ex2_approx(fmaf(__uint_as_float(sr[e4 + u]), c2, -l2[u]));
-          if (key > tk[u]) pe = 0.f;
-          pv[u] = pe;
-          dv[u] = pe * (__uint_as_float(pr[e4 + u]) - dd4[u]);
+        for (int e4 = 0; e4 < 32; e4 += 4) {
+          const int col = ch * 32 + e4;
+          const float4 a = *reinterpret_cast<const float4*>(&sh->lse2[st][col]);
+          const float4 bq = *reinterpret_cast<const float4*>(&sh->dd[st][col]);
+          const int4 c = *reinterpret_cast<const int4*>(&sh->tok[st][col]);
+          const float l2[4] = {a.x, a.y, a.z, a.w}, dd4[4] = {bq.x, bq.y, bq.z, bq.w};
+          const int tk[4] = {c.x, c.y, c.z, c.w};
+          float pv[4], dv[4];
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            float pe = ex2_approx(fmaf(__uint_as_float(sr[col + u]), c2, -l2[u]));
+            if (key > tk[u]) pe = 0.f;
+            pv[u] = pe;
+            dv[u] = pe * (__uint_as_float(pr[col + u]) - dd4[u]);
+          }
+          pk[e4 >> 1] = pack_bf16x2(pv[0], pv[1]);
+          pk[(e4 >> 1) + 1] = pack_bf16x2(pv[2], pv[3]);
+          dk[e4 >> 1] = pack_bf16x2(dv[0], dv[1]);
+          dk[(e4 >> 1) + 1] = pack_bf16x2(dv[2], dv[3]);
         }
-        pk[e4 >> 1] = pack_bf16x2(pv[0], pv[1]);
-        pk[(e4 >> 1) + 1] = pack_bf16x2(pv[2], pv[3]);
-        dk[e4 >> 1] = pack_bf16x2(dv[0], dv[1]);
-        dk[(e4 >> 1) + 1] = pack_bf16x2(dv[2], dv[3]);
+        tmem_st16(tb + ch * 16, pk);
+        tmem_st16(tb + 64 + ch * 16, dk);
       }
-      if (more) store_meta(i + 1, m_l2, m_dd, m_tok);
-      __syncthreads();  // every warp has read its S^T / dP^T columns
-      tmem_st16(tmem + lane_off + hf * 32, pk);
-      tmem_st16(tmem + lane_off + hf * 32 + 16, pk + 16);
-      tmem_st16(tmem + lane_off + 128 + hf * 32, dk);
-      tmem_st16(tmem + lane_off + 128 + hf * 32 + 16, dk + 16);
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(&sh->p_full[X]);
     }
-    tmem_st_wait();
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-    if (warp == 0) {
+    {
+      // all_done is committed once, after the last slice's dV / dK (a
+      // parity wait on x_done could match an older phase for the warpgroup
+      // that did not take the last slice); warps 0-3 add dV, warps 4-7
+      // c * dK to the window's accumulators
+      if (!mbar_wait(&sh->all_done, 0, ab)) goto ew_done;
+      __syncwarp();
+      tc_fence_after();
+      const bool valid = key < p.S;
+      float* dst = (X ? d.dk_acc : d.dv_acc) + ((int64_t)key * p.Hkv + g) * kHeadDim;
+      const float mul = X ? p.scale : 1.f;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        uint32_t a[32];
+        tmem_ld32(tmem + lane_off + 256 + X * 128 + c * 32, a);
+        tmem_ld_wait();
+        if (valid) {
+#pragma unroll
+          for (int e = 0; e < 32; e += 4) {
+            float4 x = *reinterpret_cast<float4*>(dst + c * 32 + e);
+            x.x = fmaf(__uint_as_float(a[e]), mul, x.x);
+            x.y = fmaf(__uint_as_float(a[e + 1]), mul, x.y);
+            x.z = fmaf(__uint_as_float(a[e + 2]), mul, x.z);
+            x.w = fmaf(__uint_as_float(a[e + 3]), mul, x.w);
+            *reinterpret_cast<float4*>(dst + c * 32 + e) = x;
+          }
+        }
+      }
+    }
+  ew_done:;
+  } else if (warp == 8) {
+    // ------------------------------------------------ K/V load and MMA issue
+    const uint32_t idesc_s = idesc_bf16_f32(128, kSlice, false);
+    const uint32_t idesc_o = idesc_bf16_f32(128, 128, true);
+    const uint64_t dKd = sdesc_sw128(smem_u32(sK), 16, 1024);
+    const uint64_t dVd = sdesc_sw128(smem_u32(sV), 16, 1024);
+    const uint64_t dQk = sdesc_sw128(smem_u32(sQ), 16, 1024);
+    const uint64_t ddOk = sdesc_sw128(smem_u32(sdO), 16, 1024);
+    const uint64_t dQm = sdesc_sw128(smem_u32(sQ), kSliceHalf, 1024);
+    const uint64_t ddOm = sdesc_sw128(smem_u32(sdO), kSliceHalf, 1024);
+    if (lane == 0) {
+      prefetch_tmap(&tmap_k);
+      prefetch_tmap(&tmap_v);
+      mbar_arrive_expect_tx(&sh->kv_full, 2 * kTileBytes);
+      tma_load_3d(sK, &tmap_k, &sh->kv_full, 0, g, (int)kstart);
+      tma_load_3d(sK + kHalfBytes, &tmap_k, &sh->kv_full, 64, g, (int)kstart);
+      tma_load_3d(sV, &tmap_v, &sh->kv_full, 0, g, (int)kstart);
+      tma_load_3d(sV + kHalfBytes, &tmap_v, &sh->kv_full, 64, g, (int)kstart);
+    }
+    __syncwarp();
+    // S^T and dP^T of slice m into buffer m & 1
+    auto issue_s = [&](int m) -> bool {
+      const int st = m % kDkdvStages, b = m & 1;
+      if (!mbar_wait(&sh->q_full[st], (m / kDkdvStages) & 1, ab)) return false;
+      tc_fence_after();
       if (elect_one()) {
-        const uint64_t o0 = ddOm + ((st * kTileBytes) >> 4), q0 = dQm + ((st * kTileBytes) >> 4);
+        const uint32_t so = (st * kSliceBytes) >> 4;
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          mma_bf16_ts(tmem + 256, tmem + kk * 8, o0 + ((kk * 2048) >> 4), idesc_o, (i > 0 || kk > 0) ? 1u : 0u);
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint32_t ao = ((kk >> 2) * kHalfBytes + (kk & 3) * 32) >> 4;
+          const uint32_t bo = ((kk >> 2) * kSliceHalf + (kk & 3) * 32) >> 4;
+          mma_bf16_ss(tmem + 128 * b, dKd + ao, dQk + so + bo, idesc_s, kk > 0 ? 1u : 0u);
+        }
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          mma_bf16_ts(tmem + 384, tmem + 128 + kk * 8, q0 + ((kk * 2048) >> 4), idesc_o,
-                      (i > 0 || kk > 0) ? 1u : 0u);
-        mma_commit(&sh->x_done);
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint32_t ao = ((kk >> 2) * kHalfBytes + (kk & 3) * 32) >> 4;
+          const uint32_t bo = ((kk >> 2) * kSliceHalf + (kk & 3) * 32) >> 4;
+          mma_bf16_ss(tmem + 128 * b + 64, dVd + ao, ddOk + so + bo, idesc_s, kk > 0 ? 1u : 0u);
+        }
+        mma_commit(&sh->s_full[b]);
       }
       __syncwarp();
-    }
-    if (!mbar_wait(&sh->x_done, i & 1, ab)) goto done;
+      return true;
+    };
+    if (!mbar_wait(&sh->kv_full, 0, ab)) goto mma_done;
     tc_fence_after();
-  }
-  {
-    // dV and c * dK of this thread's key, added to the window's accumulators
-    // warps 0-3 take dV, warps 4-7 c * dK
-    const bool valid = key < p.S;
-    float* dst = (hf ? d.dk_acc : d.dv_acc) + ((int64_t)key * p.Hkv + g) * kHeadDim;
-    const float mul = hf ? p.scale : 1.f;
+    if (!issue_s(0)) goto mma_done;
+    if (ns > 1 && !issue_s(1)) goto mma_done;
+    for (int m = 0; m < ns; ++m) {
+      const int st = m % kDkdvStages, b = m & 1;
+      if (!mbar_wait(&sh->p_full[b], (m >> 1) & 1, ab)) goto mma_done;
+      tc_fence_after();
+      if (elect_one()) {
+        const uint32_t so = (st * kSliceBytes) >> 4;
 #pragma unroll
-    for (int c = 0; c < 4; ++c) {
-      uint32_t a[32];
-      tmem_ld32(tmem + lane_off + 256 + hf * 128 + c * 32, a);
-      tmem_ld_wait();
-      if (valid) {
+        for (int kk = 0; kk < kSlice / 16; ++kk)
+          mma_bf16_ts(tmem + 256, tmem + 128 * b + kk * 8, ddOm + so + ((kk * 2048) >> 4), idesc_o,
+                      (m > 0 || kk > 0) ? 1u : 0u);
 #pragma unroll
-        for (int e = 0; e < 32; e += 4) {
-          float4 x = *reinterpret_cast<float4*>(dst + c * 32 + e);
-          x.x = fmaf(__uint_as_float(a[e]), mul, x.x);
-          x.y = fmaf(__uint_as_float(a[e + 1]), mul, x.y);
-          x.z = fmaf(__uint_as_float(a[e + 2]), mul, x.z);
-          x.w = fmaf(__uint_as_float(a[e + 3]), mul, x.w);
-          *reinterpret_cast<float4*>(dst + c * 32 + e) = x;
-        }
+        for (int kk = 0; kk < kSlice / 16; ++kk)
+          mma_bf16_ts(tmem + 384, tmem + 128 * b + 64 + kk * 8, dQm + so + ((kk * 2048) >> 4), idesc_o,
+                      (m > 0 || kk > 0) ? 1u : 0u);
+        mma_commit(&sh->q_empty[st]);
+        mma_commit(&sh->x_done[b]);
+        if (m == ns - 1) mma_commit(&sh->all_done);
+      }
+      __syncwarp();
+      if (m + 2 < ns) {
+        // buffer b is rewritten only after this slice's products have read it
+        if (!mbar_wait(&sh->x_done[b], (m >> 1) & 1, ab)) goto mma_done;
+        tc_fence_after();
+        if (!issue_s(m + 2)) goto mma_done;
       }
     }
-  }
-done:
-  if (*ab) {
-    volatile int keep = 0;
-    if (threadIdx.x == 0) mbar_wait(&sh->kv_full, 0, &keep, (1ull << 28));
-    if (warp == 0) {
+  mma_done:
+    __syncwarp();
+    if (*ab) {
+      // after a timeout: let the K/V load and every issued product land
+      volatile int keep = 0;
+      if (lane == 0) mbar_wait(&sh->kv_full, 0, &keep, (1ull << 28));
       if (elect_one()) mma_commit(&sh->drain);
       __syncwarp();
       mbar_wait(&sh->drain, 0, &keep, (1ull << 28));
     }
+  } else {
+    // ------------------------------------------------ row gather (64 threads)
+    const int r = threadIdx.x - 9 * 32;  // row of the slice
+    auto list_entry = [&](int m) -> int {
+      return (m < n_rs && m * kSlice + r < nr) ? __ldg(d.list + lbase + m * kSlice + r) : -1;
+    };
+    int lst_next = list_entry(0);
+    for (int m = 0; m < ns; ++m) {
+      const int st = m % kDkdvStages;
+      const int lst = lst_next;
+      lst_next = list_entry(m + 1);
+      if (!mbar_wait(&sh->q_empty[st], ((m / kDkdvStages) & 1) ^ 1, ab)) goto gather_done;
+      int64_t t = -1;
+      int h = 0;
+      if (m < n_rs) {
+        if (lst >= 0) {
+          t = p.w0 + lst / p.G;
+          h = g * p.G + lst % p.G;
+        }
+      } else {
+        const int64_t k = (int64_t)(m - n_rs) * kSlice + r;
+        if (k < n_own) {
+          const int64_t rr = own_rr0 + k;
+          t = p.w0 + rr / p.G;
+          h = g * p.G + (int)(rr % p.G);
+        }
+      }
+      const int64_t off = t >= 0 ? (t * p.Hq + h) * kHeadDim : -1;
+      gather_slice_row(smem_u32(sQ + st * kSliceBytes), p.q, off, r);
+      gather_slice_row(smem_u32(sdO + st * kSliceBytes), p.dout, off, r);
+      cp_async_commit();
+      sh->lse2[st][r] = t >= 0 ? __ldg(p.lse2 + (int64_t)h * p.S + t) : INFINITY;
+      sh->dd[st][r] = t >= 0 ? __ldg(p.dd + (int64_t)h * p.S + t) : 0.f;
+      // routed rows lie past the block: no key of it is masked for them
+      sh->tok[st][r] = (t < 0 || m < n_rs) ? 0x7fffffff : (int)t;
+      if (m > 0) {
+        // the previous slice's copies have landed
+        cp_async_wait_group<1>();
+        fence_proxy_async_smem();
+        mbar_arrive(&sh->q_full[(m - 1) % kDkdvStages]);
+      }
+    }
+    cp_async_wait_group<0>();
+    fence_proxy_async_smem();
+    mbar_arrive(&sh->q_full[(ns - 1) % kDkdvStages]);
+  gather_done:
+    cp_async_wait_all();
   }
-  cp_async_wait_all();
   tc_fence_before();
   __syncthreads();
-  if (warp == 0) {
+  if (warp == 8) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
