@@ -125,3 +125,12 @@ def test_varlen_checks_each_sequence_shape_and_pointers(lib):
     rc = lib.moba_fwd_varlen(FAKE, FAKE, FAKE, ctypes.cast(arr, ctypes.c_void_p), batch, 3, 2, 128, 512, 3, FAKE,
                              FAKE + 4, None)
     assert rc == moba.MOBA_ERR_INVALID_ARG and "multiple" in moba.last_error()
+
+
+def test_backward_rejects_bad_arguments_before_launch(lib):
+    rc = lib.moba_bwd(FAKE, FAKE, FAKE, FAKE, None, FAKE, 4096, 1, 1, 128, 512, 3, FAKE, FAKE, FAKE, None)
+    assert rc == moba.MOBA_ERR_INVALID_ARG and "null" in moba.last_error()
+    rc = lib.moba_bwd(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 4096, 1, 1, 64, 512, 3, FAKE, FAKE, FAKE, None)
+    assert rc == moba.MOBA_ERR_INVALID_ARG and "head_dim" in moba.last_error()
+    rc = lib.moba_bwd(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE + 8, 4096, 1, 1, 128, 512, 3, FAKE, FAKE, FAKE, None)
+    assert rc == moba.MOBA_ERR_INVALID_ARG and "aligned" in moba.last_error()
