@@ -123,8 +123,12 @@ __global__ void __launch_bounds__(256) bwd_cast_kernel(const float4* __restrict_
   }
 }
 
+constexpr int kDqThreads = 256;  // two warps per TMEM lane quadrant
+constexpr int kDqKStages = 3;    // K is read by S(s) and dQ(s): three stages in flight
+constexpr int kDqSmemBytes = (2 + kDqKStages + 2) * kTileBytes + 1024 + 512;
+
 struct BwdShared {
-  uint64_t kv_full[2];
+  uint64_t k_full[kDqKStages], v_full[2];
   uint64_t s_done, x_done, drain;
   uint32_t tmem_base;
   int abort_flag;
@@ -187,10 +191,19 @@ __device__ __forceinline__ void bwd_softmax_grad(uint32_t tS, uint32_t tP, float
   }
 }
 
-// grid = number of SMs, 128 threads (thread = query row = TMEM lane), items
-// (unit, tile) taken with a fixed stride. TMEM: S 0..127 (then dS as bf16
-// over 0..63), dP 128..255, dQ 256..383.
-__global__ void __launch_bounds__(kBwdThreads, 1)
+// grid = number of SMs, 256 threads: two warps per TMEM lane quadrant (lane =
+// query row), each taking 64 of a step's 128 key columns and 64 of dQ's
+// columns; threads 0..127 gather Q rows, 128..255 dO rows. Items (unit,
+// tile) are taken with a fixed stride. Per 128-key step s:
+//   S(s) = Q K^T, dP(s) = dO V^T   (SS MMAs into TMEM 0..127, 128..255)
+//   every warp loads its S / dP columns, then S(s+1), dP(s+1) are issued
+//   into the same columns while the warps compute dS(s) = P (dP - D)
+//   dS(s) goes to TMEM 384..447 (bf16) once dQ(s-1) has read the previous
+//   one, and dQ += dS(s) K (TS MMA, K as an MN-major B operand) into
+//   256..383.
+// K sits in a 3-stage ring (read by S(s) and by dQ(s)), V in 2 stages; the
+// loads for step s+2 go out once dQ(s-1) is done.
+__global__ void __launch_bounds__(kDqThreads, 1)
     bwd_dq_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant__ CUtensorMap tmap_v,
                   AttnParams ap, BwdParams p) {
   grid_dependency_sync();
@@ -198,14 +211,16 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sQ = smem;
   uint8_t* sdO = sQ + kTileBytes;
-  uint8_t* sK = sdO + kTileBytes;         // 2 stages
-  uint8_t* sV = sK + 2 * kTileBytes;      // 2 stages
+  uint8_t* sK = sdO + kTileBytes;             // kDqKStages stages
+  uint8_t* sV = sK + kDqKStages * kTileBytes;  // 2 stages
   BwdShared* sh = reinterpret_cast<BwdShared*>(sV + 2 * kTileBytes);
   const int warp = threadIdx.x >> 5;
-  const int row = threadIdx.x;
+  const int row = threadIdx.x & (kTile - 1);  // query row (TMEM lane) and gathered row
+  const int hf = warp >> 2;                   // this warp's half of the columns
   if (threadIdx.x == 0) {
-    mbar_init(&sh->kv_full[0], 1);
-    mbar_init(&sh->kv_full[1], 1);
+    for (int i = 0; i < kDqKStages; ++i) mbar_init(&sh->k_full[i], 1);
+    mbar_init(&sh->v_full[0], 1);
+    mbar_init(&sh->v_full[1], 1);
     mbar_init(&sh->s_done, 1);
     mbar_init(&sh->x_done, 1);
     mbar_init(&sh->drain, 1);
@@ -222,7 +237,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = sh->tmem_base;
-  const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+  const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
   volatile int* ab = &sh->abort_flag;
   const uint32_t idesc_s = idesc_bf16_f32(128, 128, false);
   const uint32_t idesc_o = idesc_bf16_f32(128, 128, true);
@@ -233,19 +248,45 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   const uint64_t dKmn = sdesc_sw128(smem_u32(sK), kHalfBytes, 1024);
   const float c2 = p.scale_log2;
   const int n_units = ap.hdr[1];
-  uint32_t kv_it = 0;   // K/V loads issued before this item
-  uint32_t mma_it = 0;  // steps done (phase of s_done / x_done)
-  uint32_t loaded = 0;    // K/V loads issued in total (thread 0)
-  uint32_t consumed = 0;  // K/V loads waited for
+  uint32_t L0 = 0;      // global index of this item's first step
+  uint32_t loaded = 0;  // K/V step loads issued (thread 0)
+  uint32_t waited = 0;  // K/V step loads waited for (thread 0)
   auto load_kv = [&](uint32_t L, const UnitInfo& u, int s) {  // thread 0
-    const int st = L & 1;
+    const int ks = L % kDqKStages, vs = L & 1;
     const int key = (int)(u.key0 + (int64_t)s * kTile);
-    mbar_arrive_expect_tx(&sh->kv_full[st], 2 * kTileBytes);
-    tma_load_3d(sK + st * kTileBytes, &tmap_k, &sh->kv_full[st], 0, u.g, key);
-    tma_load_3d(sK + st * kTileBytes + kHalfBytes, &tmap_k, &sh->kv_full[st], 64, u.g, key);
-    tma_load_3d(sV + st * kTileBytes, &tmap_v, &sh->kv_full[st], 0, u.g, key);
-    tma_load_3d(sV + st * kTileBytes + kHalfBytes, &tmap_v, &sh->kv_full[st], 64, u.g, key);
+    mbar_arrive_expect_tx(&sh->k_full[ks], kTileBytes);
+    tma_load_3d(sK + ks * kTileBytes, &tmap_k, &sh->k_full[ks], 0, u.g, key);
+    tma_load_3d(sK + ks * kTileBytes + kHalfBytes, &tmap_k, &sh->k_full[ks], 64, u.g, key);
+    mbar_arrive_expect_tx(&sh->v_full[vs], kTileBytes);
+    tma_load_3d(sV + vs * kTileBytes, &tmap_v, &sh->v_full[vs], 0, u.g, key);
+    tma_load_3d(sV + vs * kTileBytes + kHalfBytes, &tmap_v, &sh->v_full[vs], 64, u.g, key);
     loaded = L + 1;
+  };
+  // S(L) and dP(L) (thread 0's warp; K / V of step L must have landed)
+  auto issue_s = [&](uint32_t L) -> bool {
+    if (threadIdx.x == 0) {
+      if (!mbar_wait(&sh->k_full[L % kDqKStages], (L / kDqKStages) & 1, ab)) return false;
+      if (!mbar_wait(&sh->v_full[L & 1], (L >> 1) & 1, ab)) return false;
+      waited = L + 1;
+    }
+    __syncwarp();
+    tc_fence_after();
+    if (elect_one()) {
+      const uint64_t k0 = dK + (((L % kDqKStages) * kTileBytes) >> 4), v0 = dV + (((L & 1) * kTileBytes) >> 4);
+#pragma unroll
+      for (int kk = 0; kk < 8; ++kk) {
+        const uint32_t o = ((kk >> 2) * kHalfBytes + (kk & 3) * 32) >> 4;
+        mma_bf16_ss(tmem, dQd + o, k0 + o, idesc_s, kk > 0 ? 1u : 0u);
+      }
+#pragma unroll
+      for (int kk = 0; kk < 8; ++kk) {
+        const uint32_t o = ((kk >> 2) * kHalfBytes + (kk & 3) * 32) >> 4;
+        mma_bf16_ss(tmem + 128, ddOd + o, v0 + o, idesc_s, kk > 0 ? 1u : 0u);
+      }
+      mma_commit(&sh->s_done);
+    }
+    __syncwarp();
+    return !*ab;
   };
   for (int item = blockIdx.x; item < 2 * n_units; item += gridDim.x) {
     const UnitInfo u = decode_unit(ap, item >> 1);
@@ -265,16 +306,19 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       }
     }
     const int64_t off = t >= 0 ? (t * p.Hq + h) * kHeadDim : -1;
-    gather_row(smem_u32(sQ), p.q, off, row);
-    gather_row(smem_u32(sdO), p.dout, off, row);
+    if (threadIdx.x < kTile)
+      gather_row(smem_u32(sQ), p.q, off, row);
+    else
+      gather_row(smem_u32(sdO), p.dout, off, row);
     float lse2_r = INFINITY, dd_r = 0.f;  // a missing row gets P = 0
     if (t >= 0) {
       lse2_r = __ldg(p.lse2 + (int64_t)h * p.S + t);
       dd_r = __ldg(p.dd + (int64_t)h * p.S + t);
     }
     if (threadIdx.x == 0) {
-      load_kv(kv_it, u, 0);
-      if (u.nsteps > 1) load_kv(kv_it + 1, u, 1);
+      // the previous item's products are all done: every stage is free
+      load_kv(L0, u, 0);
+      if (u.nsteps > 1) load_kv(L0 + 1, u, 1);
     }
     cp_async_wait_all();
     fence_proxy_async_smem();
@@ -282,67 +326,73 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     __syncthreads();
     tc_fence_after();
     const int dstep = u.own ? u.diag[x] : u.nsteps;
+    if (warp == 0 && !issue_s(L0)) goto done;
     for (int s = 0; s < u.nsteps; ++s) {
-      const uint32_t L = kv_it + s;
-      const int st = L & 1;
-      if (!mbar_wait(&sh->kv_full[st], (L >> 1) & 1, ab)) goto done;
-      consumed = L + 1;
-      tc_fence_after();
-      if (warp == 0) {
-        if (elect_one()) {
-          const uint64_t k0 = dK + ((st * kTileBytes) >> 4), v0 = dV + ((st * kTileBytes) >> 4);
-#pragma unroll
-          for (int kk = 0; kk < 8; ++kk) {
-            const uint32_t o = ((kk >> 2) * kHalfBytes + (kk & 3) * 32) >> 4;
-            mma_bf16_ss(tmem, dQd + o, k0 + o, idesc_s, kk > 0 ? 1u : 0u);
-          }
-#pragma unroll
-          for (int kk = 0; kk < 8; ++kk) {
-            const uint32_t o = ((kk >> 2) * kHalfBytes + (kk & 3) * 32) >> 4;
-            mma_bf16_ss(tmem + 128, ddOd + o, v0 + o, idesc_s, kk > 0 ? 1u : 0u);
-          }
-          mma_commit(&sh->s_done);
-        }
-        __syncwarp();
-      }
-      if (!mbar_wait(&sh->s_done, mma_it & 1, ab)) goto done;
+      const uint32_t L = L0 + s;
+      if (!mbar_wait(&sh->s_done, L & 1, ab)) goto done;
       __syncwarp();
       tc_fence_after();
+      uint32_t sr[64], pr[64];
+      tmem_ld32(tmem + lane_off + hf * 64, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
+      tmem_ld32(tmem + lane_off + hf * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
+      tmem_ld32(tmem + lane_off + 128 + hf * 64, *reinterpret_cast<uint32_t(*)[32]>(&pr[0]));
+      tmem_ld32(tmem + lane_off + 128 + hf * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&pr[32]));
+      tmem_ld_wait();
+      tc_fence_before();
+      __syncthreads();  // every warp holds its S(s) / dP(s) columns
+      tc_fence_after();
+      if (warp == 0 && s + 1 < u.nsteps && !issue_s(L + 1)) goto done;
+      // dS(s), keys e > lim masked on and after the diagonal step
+      uint32_t dk[32];
       {
-        // keys e > lim are masked on and after the diagonal step
         const int lim = s >= dstep ? row - (s - dstep) * kTile : kTile;
-        bwd_softmax_grad<false>(tmem + lane_off, tmem + lane_off + 128, c2, lse2_r, dd_r, lim, nullptr, nullptr,
-                                nullptr, 0);
+#pragma unroll
+        for (int e = 0; e < 64; e += 2) {
+          float dv[2];
+#pragma unroll
+          for (int v2 = 0; v2 < 2; ++v2) {
+            float pe = ex2_approx(fmaf(__uint_as_float(sr[e + v2]), c2, -lse2_r));
+            if (hf * 64 + e + v2 > lim) pe = 0.f;
+            dv[v2] = pe * (__uint_as_float(pr[e + v2]) - dd_r);
+          }
+          dk[e >> 1] = pack_bf16x2(dv[0], dv[1]);
+        }
       }
+      // dQ(s-1) has read the previous dS; its K stage is then free, and V's
+      // stage was freed by dP(s): load step s+2
+      if (s > 0 && !mbar_wait(&sh->x_done, (L - 1) & 1, ab)) goto done;
+      if (threadIdx.x == 0 && s + 2 < u.nsteps) load_kv(L + 2, u, s + 2);
+      tc_fence_after();
+      tmem_st16(tmem + lane_off + 384 + hf * 32, dk);
+      tmem_st16(tmem + lane_off + 384 + hf * 32 + 16, dk + 16);
       tmem_st_wait();
       tc_fence_before();
       __syncthreads();
       tc_fence_after();
       if (warp == 0) {
         if (elect_one()) {
-          const uint64_t k0 = dKmn + ((st * kTileBytes) >> 4);
+          const uint64_t k0 = dKmn + (((L % kDqKStages) * kTileBytes) >> 4);
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk)
-            mma_bf16_ts(tmem + 256, tmem + kk * 8, k0 + ((kk * 2048) >> 4), idesc_o, (s > 0 || kk > 0) ? 1u : 0u);
+            mma_bf16_ts(tmem + 256, tmem + 384 + kk * 8, k0 + ((kk * 2048) >> 4), idesc_o,
+                        (s > 0 || kk > 0) ? 1u : 0u);
           mma_commit(&sh->x_done);
         }
         __syncwarp();
       }
-      if (!mbar_wait(&sh->x_done, mma_it & 1, ab)) goto done;
-      tc_fence_after();
-      ++mma_it;
-      // K/V stage st is free again
-      if (threadIdx.x == 0 && s + 2 < u.nsteps) load_kv(L + 2, u, s + 2);
     }
-    kv_it += u.nsteps;
+    L0 += u.nsteps;
+    // the item's last dQ product, then c * dQ as an fp16 partial
+    if (!mbar_wait(&sh->x_done, (L0 - 1) & 1, ab)) goto done;
+    __syncwarp();
+    tc_fence_after();
     {
-      // the item's c * dQ as an fp16 partial
       __half* dst = nullptr;
       if (t >= 0)
         dst = u.own ? ap.own_o + ((t - p.w0) * p.Hq + h) * kHeadDim
                     : ap.part_o + ((int64_t)u.list0[x] + row) * kHeadDim;
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
+      for (int c = 2 * hf; c < 2 * hf + 2; ++c) {
         uint32_t o[32];
         tmem_ld32(tmem + lane_off + 256 + c * 32, o);
         tmem_ld_wait();
@@ -358,7 +408,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           }
         }
       }
-      // the next item's MMAs overwrite TMEM and shared memory
+      // the next item's gather and products overwrite shared memory and TMEM
       tc_fence_before();
       __syncthreads();
       tc_fence_after();
@@ -369,7 +419,10 @@ done:
     // after a timeout: let issued copies and products land first (bounded)
     volatile int keep = 0;
     if (threadIdx.x == 0)
-      for (uint32_t L = consumed; L < loaded; ++L) mbar_wait(&sh->kv_full[L & 1], (L >> 1) & 1, &keep, (1ull << 28));
+      for (uint32_t L = waited; L < loaded; ++L) {
+        mbar_wait(&sh->k_full[L % kDqKStages], (L / kDqKStages) & 1, &keep, (1ull << 28));
+        mbar_wait(&sh->v_full[L & 1], (L >> 1) & 1, &keep, (1ull << 28));
+      }
     if (warp == 0) {
       if (elect_one()) mma_commit(&sh->drain);
       __syncwarp();

@@ -69,7 +69,7 @@ int device_info(DeviceInfo* out) {
       MOBA_CUDA(cudaFuncSetAttribute(moba::attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      moba::kAttnSmemBytes));
       MOBA_CUDA(cudaFuncSetAttribute(moba::bwd_dq_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                     moba::kBwdSmemBytes));
+                                     moba::kDqSmemBytes));
       MOBA_CUDA(cudaFuncSetAttribute(moba::bwd_dkdv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      moba::kBwdSmemBytes));
       MOBA_CUDA(cudaFuncSetAttribute(moba::gate_tc_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -679,7 +679,7 @@ int run_backward(const Plan& p, const BwdLayout& bl, const DeviceInfo& dev, cons
     ap.w0 = w0;
     bp.w0 = w0;
     bp.wlen = wg.wlen;
-    launch_chained(moba::bwd_dq_kernel, dim3(dev.sms), dim3(moba::kBwdThreads), moba::kBwdSmemBytes, st, tmk, tmv,
+    launch_chained(moba::bwd_dq_kernel, dim3(dev.sms), dim3(moba::kDqThreads), moba::kDqSmemBytes, st, tmk, tmv,
                    ap, bp);
     launch_chained(moba::bwd_dq_reduce_kernel, dim3((unsigned)((wg.wlen * p.Hq + 7) / 8)), dim3(256), 0, st,
                    static_cast<const int32_t*>(sel), reinterpret_cast<const uint32_t*>(ws + p.o_flags),
