@@ -315,7 +315,7 @@ def run_chunk(args, w):
         "config": dict(workload_config(w, 1), mode="decode" if n == 1 else "chunked prefill", q_start=q0, chunk=n,
                        block_means="cached (pooled once)" if args.cached_means else "pooled every call"),
         "eff_tflops": flops * args.steps / (total_ms / 1e3) / 1e12,
-        "stage_ms_per_step": {kk: vv / max(calls, 1) for kk, vv in stages.items()},
+        "stage_ms_per_step": {kk: vv / max(calls, 1) for kk, vv in stages.items() if not kk.startswith("bwd_")},
         "roofline": {"bound": "tensor", "kernel": "attn_kernel", "achieved": achieved,
                      "peak": peaks["bf16_tflops"], "unit": "TFLOP/s", "frac": achieved / peaks["bf16_tflops"],
                      "traffic": None, "peak_source": f"{peaks_src} bf16 burst",
@@ -395,7 +395,7 @@ def run_backward(args, w):
     e2e_ms = 1e3 * (time.perf_counter() - t0)
     peaks, peaks_src = load_peaks()
     fwd_flops = chunk_flops(w, 0)
-    per = {kk: vv / max(calls, 1) for kk, vv in stages.items()}
+    per = {kk: vv / max(calls, 1) for kk, vv in stages.items() if kk not in ("attention", "merge")}
     dkdv_flops = 2.0 * fwd_flops  # S^T, dP^T, dV, dK
     achieved = dkdv_flops / (per["bwd_dkdv"] / 1e3) / 1e12
     line = {
@@ -503,7 +503,7 @@ def run_varlen(args, w):
         "config": dict(workload_config(w, 1), mode="packed batch", batch_per_gpu=int(args.varlen),
                        lengths=[int(x) for x in lengths]),
         "eff_tflops": flops * args.steps / (total_ms / 1e3) / 1e12,
-        "stage_ms_per_step": {kk: vv / args.steps for kk, vv in stages.items()},
+        "stage_ms_per_step": {kk: vv / args.steps for kk, vv in stages.items() if not kk.startswith("bwd_")},
         "roofline": {"bound": "tensor", "kernel": "attn_kernel", "achieved": achieved,
                      "peak": peaks["bf16_tflops"], "unit": "TFLOP/s", "frac": achieved / peaks["bf16_tflops"],
                      "traffic": None, "peak_source": f"{peaks_src} bf16 burst",
@@ -650,7 +650,7 @@ def run_ours(args, w):
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
             "config": workload_config(wr, world),
             "eff_tflops": world * flops * args.steps / (total_ms / 1e3) / 1e12,
-            "stage_ms_per_step": {kk: vv / max(calls, 1) for kk, vv in stages.items()},
+            "stage_ms_per_step": {kk: vv / max(calls, 1) for kk, vv in stages.items() if not kk.startswith("bwd_")},
             "ms_per_step_kernel_by_kernel": prof_ms,
             "roofline": {"bound": "tensor", "kernel": "attn_kernel", "achieved": achieved, "peak": peak,
                          "unit": "TFLOP/s", "frac": achieved / peak, "traffic": attn_traffic(wr.name),
