@@ -261,6 +261,30 @@ __global__ void __launch_bounds__(kGateTcThreads)
           if (i < jn && __uint_as_float(sc[e]) > thr) cand |= 1ull << i;
         }
       }
+      if (KP >= 8 && KP <= 24 && c == 0 && jn > KP) {
+        // First chunk, where every column beats an empty list (short lists
+        // insert cheaply and skip this): split the
+        // row's jn columns into KP strided groups; the smallest group
+        // maximum tau0 is met by KP distinct columns, so a column strictly
+        // below it cannot reach the top KP (a tie with it still can: ties go
+        // to the lower block). Columns below tau0 leave the candidate set.
+        float gm[KP > 24 ? 1 : KP];
+#pragma unroll
+        for (int g = 0; g < (KP > 24 ? 1 : KP); ++g) gm[g] = -INFINITY;
+#pragma unroll
+        for (int i = 0; i < kGateBlkChunk; ++i) {
+          const float sv = i < jn ? stage[(((i >> 2) ^ (row & 15)) << 2) | (i & 3)] : -INFINITY;
+          gm[i % (KP > 24 ? 1 : KP)] = fmaxf(gm[i % (KP > 24 ? 1 : KP)], sv);
+        }
+        float tau0 = gm[0];
+#pragma unroll
+        for (int g = 1; g < (KP > 24 ? 1 : KP); ++g) tau0 = fminf(tau0, gm[g]);
+        uint64_t keep = 0;
+#pragma unroll
+        for (int i = 0; i < kGateBlkChunk; ++i)
+          if (stage[(((i >> 2) ^ (row & 15)) << 2) | (i & 3)] >= tau0) keep |= 1ull << i;
+        cand &= keep;
+      }
       while (cand) {
         const int i = __ffsll((long long)cand) - 1;
         cand &= cand - 1;
