@@ -15,19 +15,22 @@
 // so the selection is the forward's):
 //   bwd_dq_kernel    per forward work unit and tile of 128 query rows:
 //                    S = Q K^T and dP = dO V^T on the tensor cores for each
-//                    128-key step of the unit's block, dS written back over
-//                    S in TMEM as bf16, dQ += dS K accumulated in TMEM; the
-//                    unit's c*dQ goes out as an fp16 partial into the slot
-//                    the forward uses for its partial output.
+//                    128-key step of the unit's block (the next step's
+//                    issued while this step's element-wise work runs), dS to
+//                    TMEM as bf16, dQ += dS K accumulated in TMEM; the unit's
+//                    c*dQ goes out as an fp16 partial into the slot the
+//                    forward uses for its partial output.
 //   bwd_dq_reduce    dQ = sum of a row's partials in a fixed order (its
 //                    selected past blocks ascending, its own block last).
 //   bwd_dkdv_kernel  per (kv head, block, 128-key tile): the transposed
 //                    products S^T = K Q^T and dP^T = V dO^T for every
-//                    128-row tile of the rows that attend the block (its
+//                    64-row slice of the rows that attend the block (its
 //                    router list, then its own causal rows), P^T and dS^T
 //                    written back as bf16, dV += P^T dO and dK += dS^T Q
-//                    accumulated in TMEM over all of them; one fp32
-//                    read-add-write per key row and query window.
+//                    accumulated in TMEM over all of them (two slice
+//                    buffers, so one slice's element-wise step overlaps the
+//                    other's products); one fp32 read-add-write per key row
+//                    and query window.
 // Both tensor-core kernels take K, V, Q and dO tiles in the 128-byte-swizzled
 // layout, read K-major for S / dP and MN-major for the dQ / dK / dV products.
 // Every mbarrier wait is bounded and sets the device status on a timeout.
@@ -39,7 +42,7 @@
 
 namespace moba {
 
-constexpr int kBwdThreads = 128;
+// dK / dV kernel: K, V, four 64-row Q and dO slices, its shared state
 constexpr int kBwdSmemBytes = 6 * kTileBytes + 1024 + 4096;
 
 struct BwdParams {
@@ -133,63 +136,6 @@ struct BwdShared {
   uint32_t tmem_base;
   int abort_flag;
 };
-
-// dS = P * (dP - D) for 128 columns of one TMEM lane: S at tS, dP at tP.
-// Column e is a key (dq kernel: kTransposed false, the lane is a query row
-// with lse2_row / dd_row) or a query row (dkdv kernel: kTransposed, the lane
-// is a key; per-column lse2 / dd / token from shared memory). P (kept only
-// when kTransposed) goes over the first 64 columns at tS, dS over the first 64 at tP (dkdv) or
-// over tS (dq). Masked entries: keys beyond `lim` (dq), or keys above the
-// column's token (dkdv).
-template <bool kTransposed>
-__device__ __forceinline__ void bwd_softmax_grad(uint32_t tS, uint32_t tP, float c2, float lse2_row, float dd_row,
-                                                 int lim, const float* s_lse2, const float* s_dd, const int* s_tok,
-                                                 int key) {
-#pragma unroll
-  for (int ch = 0; ch < 4; ++ch) {
-    uint32_t sr[32], pr[32];
-    tmem_ld32(tS + ch * 32, sr);
-    tmem_ld32(tP + ch * 32, pr);
-    tmem_ld_wait();
-    uint32_t pk[16], dk[16];
-#pragma unroll
-    for (int e4 = 0; e4 < 32; e4 += 4) {
-      // per-column values, four at a time (shared-memory broadcasts)
-      float l2[4], dd4[4];
-      int tk[4];
-      if (kTransposed) {
-        const float4 a = *reinterpret_cast<const float4*>(s_lse2 + ch * 32 + e4);
-        const float4 b = *reinterpret_cast<const float4*>(s_dd + ch * 32 + e4);
-        const int4 c = *reinterpret_cast<const int4*>(s_tok + ch * 32 + e4);
-        l2[0] = a.x, l2[1] = a.y, l2[2] = a.z, l2[3] = a.w;
-        dd4[0] = b.x, dd4[1] = b.y, dd4[2] = b.z, dd4[3] = b.w;
-        tk[0] = c.x, tk[1] = c.y, tk[2] = c.z, tk[3] = c.w;
-      }
-      float pv[4], dv[4];
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int col = ch * 32 + e4 + u;
-        const float l = kTransposed ? l2[u] : lse2_row;
-        const float d = kTransposed ? dd4[u] : dd_row;
-        float pe = ex2_approx(fmaf(__uint_as_float(sr[e4 + u]), c2, -l));
-        const bool masked = kTransposed ? (key > tk[u]) : (col > lim);
-        if (masked) pe = 0.f;
-        pv[u] = pe;
-        dv[u] = pe * (__uint_as_float(pr[e4 + u]) - d);
-      }
-      pk[e4 >> 1] = pack_bf16x2(pv[0], pv[1]);
-      pk[(e4 >> 1) + 1] = pack_bf16x2(pv[2], pv[3]);
-      dk[e4 >> 1] = pack_bf16x2(dv[0], dv[1]);
-      dk[(e4 >> 1) + 1] = pack_bf16x2(dv[2], dv[3]);
-    }
-    if (kTransposed) {
-      tmem_st16(tS + ch * 16, pk);
-      tmem_st16(tP + ch * 16, dk);
-    } else {
-      tmem_st16(tS + ch * 16, dk);
-    }
-  }
-}
 
 // grid = number of SMs, 256 threads: two warps per TMEM lane quadrant (lane =
 // query row), each taking 64 of a step's 128 key columns and 64 of dQ's
