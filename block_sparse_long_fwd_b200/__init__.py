@@ -45,6 +45,7 @@ SIGNATURES = {
     "moba_last_error": (ctypes.c_char_p, []),
     "moba_device_status": (_i32, [_vp]),
     "moba_selftest_bounded_wait": (_i32, [_i32, _vp]),
+    "moba_selftest_bounded_wait_async": (_i32, [_i32, _vp]),
 }
 
 

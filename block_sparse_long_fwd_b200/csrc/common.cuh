@@ -19,8 +19,17 @@ constexpr int kTile = 128;  // query rows per attention tile and keys per step
 
 // First device-side error of the calls since the last read (0 = none).
 __device__ int g_status;
+// Device address of a host-mapped copy of the status (set by the host when it
+// first uses the device; null before): the next call on the host sees an
+// error there without reading device memory. A plain store (no atomics on
+// host memory), taken only when something has failed.
+__device__ int* g_status_mirror;
 
-__device__ __forceinline__ void record_status(int code) { atomicCAS(&g_status, 0, code); }
+__device__ __forceinline__ void record_status(int code) {
+  atomicCAS(&g_status, 0, code);
+  int* m = g_status_mirror;
+  if (m) *reinterpret_cast<volatile int*>(m) = code;
+}
 
 __device__ __forceinline__ uint64_t globaltimer_ns() {
   uint64_t t;

@@ -47,6 +47,7 @@ struct DeviceInfo {
   bool ready = false;
   bool sm100 = false;
   int sms = 0;
+  int* status_host = nullptr;  // host-mapped copy of the device status word
 };
 
 std::mutex g_dev_mu;
@@ -90,6 +91,15 @@ int device_info(DeviceInfo* out) {
                                      moba::kGateSmemBytes));
       MOBA_CUDA(cudaFuncSetAttribute(moba::gate_tc_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      moba::kGateSmemBytes));
+      // host-mapped copy of the status word (kernels store an error code
+      // there too, so a later call sees it without a device read)
+      int* h = nullptr;
+      MOBA_CUDA(cudaHostAlloc(reinterpret_cast<void**>(&h), sizeof(int), cudaHostAllocMapped | cudaHostAllocPortable));
+      *h = 0;
+      int* hd = nullptr;
+      MOBA_CUDA(cudaHostGetDevicePointer(reinterpret_cast<void**>(&hd), h, 0));
+      MOBA_CUDA(cudaMemcpyToSymbol(moba::g_status_mirror, &hd, sizeof(hd)));
+      d.status_host = h;
       // keep freed scratch in the stream-ordered pool between calls
       cudaMemPool_t pool;
       MOBA_CUDA(cudaDeviceGetDefaultMemPool(&pool, dev));
@@ -126,6 +136,35 @@ int make_kv_map(CUtensorMap* map, const void* base, int64_t S, int H) {
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
+
+// An error code a kernel of an earlier call left in the host-mapped status
+// word: this call reports it (once) instead of launching, and clears it and
+// the device word, so the call after starts clean.
+int take_pending_status(const DeviceInfo& dev, cudaStream_t st) {
+  if (!dev.status_host) return MOBA_OK;
+  volatile int* h = dev.status_host;
+  const int s = *h;
+  if (!s) return MOBA_OK;
+  *h = 0;
+  static const int zero = 0;
+  cudaMemcpyToSymbolAsync(moba::g_status, &zero, sizeof(int), 0, cudaMemcpyHostToDevice, st);
+  return fail(s, "a kernel of an earlier call on this device reported status %d (a bounded wait ran out or a "
+              "check failed); its results are not valid", s);
+}
+
+// MOBA_SYNC=1: every call synchronises its stream and returns the kernels'
+// status itself.
+bool sync_mode() {
+  const char* e = getenv("MOBA_SYNC");
+  return e && e[0] == '1';
+}
+
+// A call's result: under MOBA_SYNC=1 a successful launch waits for its stream
+// and returns the kernels' status.
+int finish_call(int rc, cudaStream_t st) {
+  if (rc == MOBA_OK && sync_mode()) return moba_device_status(st);
+  return rc;
+}
 
 int check_shape(int64_t S, int Hq, int Hkv, int d, int B, int topk) {
   if (S < 1) return fail(MOBA_ERR_INVALID_ARG, "seqlen must be >= 1 (got %lld)", (long long)S);
@@ -845,6 +884,8 @@ int fwd_impl(const void* q, const void* k, const void* v, int64_t seqlen, int64_
   DeviceInfo dev;
   rc = device_info(&dev);
   if (rc) return rc;
+  rc = take_pending_status(dev, stream);
+  if (rc) return rc;
   Plan p;
   rc = make_plan(&p, seqlen, q_start, heads_q, heads_kv, block_size, topk);
   if (rc) return rc;
@@ -854,9 +895,9 @@ int fwd_impl(const void* q, const void* k, const void* v, int64_t seqlen, int64_
   if (use_graph && !g_timer.on) {
     GraphKey key{0, q, k, v, out, lse, p.means, p.S, p.q0, p.W, p.lse_ld, p.Hq, p.Hkv, p.B, p.topk, {}};
     const int g = graph_run(std::move(key), p.total, run, stream);
-    if (g >= 0) return g;  // negative: no graph for this call, launch directly
+    if (g >= 0) return finish_call(g, stream);  // negative: no graph for this call, launch directly
   }
-  return direct_run(p.total, run, stream);
+  return finish_call(direct_run(p.total, run, stream), stream);
 }
 
 // A packed batch of independent sequences: sequence b holds tokens
@@ -897,6 +938,8 @@ int varlen_impl(const void* q, const void* k, const void* v, const int64_t* cu, 
   DeviceInfo dev;
   int rc = device_info(&dev);
   if (rc) return rc;
+  rc = take_pending_status(dev, stream);
+  if (rc) return rc;
   const size_t qrow = (size_t)heads_q * head_dim * 2, kvrow = (size_t)heads_kv * head_dim * 2;
   const Runner run = [&](uint8_t* ws, cudaStream_t st) {
     for (size_t i = 0; i < plans.size(); ++i) {
@@ -912,9 +955,9 @@ int varlen_impl(const void* q, const void* k, const void* v, const int64_t* cu, 
     GraphKey key{0, q, k, v, out, lse, nullptr, T, 0, 0, T, heads_q, heads_kv, block_size, topk,
                  std::vector<int64_t>(cu, cu + batch + 1)};
     const int g = graph_run(std::move(key), total, run, stream);
-    if (g >= 0) return g;
+    if (g >= 0) return finish_call(g, stream);
   }
-  return direct_run(total, run, stream);
+  return finish_call(direct_run(total, run, stream), stream);
 }
 
 }  // namespace
@@ -959,6 +1002,8 @@ int moba_bwd(const void* q, const void* k, const void* v, const void* out, const
   DeviceInfo dev;
   rc = device_info(&dev);
   if (rc) return rc;
+  rc = take_pending_status(dev, stream);
+  if (rc) return rc;
   Plan p;
   rc = make_plan(&p, seqlen, 0, heads_q, heads_kv, block_size, topk);
   if (rc) return rc;
@@ -966,7 +1011,7 @@ int moba_bwd(const void* q, const void* k, const void* v, const void* out, const
   const Runner run = [&](uint8_t* ws, cudaStream_t st) {
     return run_backward(p, bl, dev, q, k, v, out, lse, dout, dq, dk, dv, ws, st);
   };
-  return direct_run(bl.total, run, stream);
+  return finish_call(direct_run(bl.total, run, stream), stream);
 }
 
 int moba_profile_begin(void) {
@@ -1036,6 +1081,8 @@ int moba_pool(const void* k, int64_t seqlen, int heads_kv, int head_dim, int blo
   DeviceInfo dev;
   rc = device_info(&dev);
   if (rc) return rc;
+  rc = take_pending_status(dev, stream);
+  if (rc) return rc;
   Plan p;
   p.S = seqlen;
   p.Hkv = heads_kv;
@@ -1044,7 +1091,7 @@ int moba_pool(const void* k, int64_t seqlen, int heads_kv, int head_dim, int blo
   p.nbp = p.nb - 1;
   launch_pool(p, k, kmean, 1, stream);
   MOBA_CUDA(cudaGetLastError());
-  return MOBA_OK;
+  return finish_call(MOBA_OK, stream);
 }
 
 int moba_gate(const void* q, const float* kmean, int64_t seqlen, int heads_q, int heads_kv, int head_dim,
@@ -1059,6 +1106,8 @@ int moba_gate(const void* q, const float* kmean, int64_t seqlen, int heads_q, in
   if (!aligned16(q)) return fail(MOBA_ERR_INVALID_ARG, "device buffers must be 16-byte aligned");
   DeviceInfo dev;
   rc = device_info(&dev);
+  if (rc) return rc;
+  rc = take_pending_status(dev, stream);
   if (rc) return rc;
   Plan p;
   p.S = seqlen;
@@ -1084,7 +1133,7 @@ int moba_gate(const void* q, const float* kmean, int64_t seqlen, int heads_q, in
   if (n < 0) return -n;
   MOBA_CUDA(cudaGetLastError());
   if (ef != cudaSuccess) return fail(MOBA_ERR_CUDA, "cudaFreeAsync failed: %s", cudaGetErrorString(ef));
-  return MOBA_OK;
+  return finish_call(MOBA_OK, stream);
 }
 
 int moba_device_status(cudaStream_t stream) {
@@ -1094,6 +1143,9 @@ int moba_device_status(cudaStream_t stream) {
   MOBA_CUDA(cudaMemcpyFromSymbol(&s, moba::g_status, sizeof(int)));
   const int zero = 0;
   MOBA_CUDA(cudaMemcpyToSymbol(moba::g_status, &zero, sizeof(int)));
+  DeviceInfo dev;
+  if (device_info(&dev) == MOBA_OK && dev.status_host) *reinterpret_cast<volatile int*>(dev.status_host) = 0;
+  g_err.clear();
   if (s) fail(s, "a kernel reported device status %d", s);
   return s;
 }
@@ -1128,6 +1180,17 @@ extern "C" int moba_selftest_bounded_wait(int timeout_us, cudaStream_t stream) {
   moba::selftest_wait_kernel<<<1, 32, 0, stream>>>((uint64_t)timeout_us * 2000ull);
   MOBA_CUDA(cudaGetLastError());
   return moba_device_status(stream);
+}
+
+extern "C" int moba_selftest_bounded_wait_async(int timeout_us, cudaStream_t stream) {
+  g_err.clear();
+  if (timeout_us < 1 || timeout_us > 2000000) return fail(MOBA_ERR_INVALID_ARG, "timeout_us must be in [1, 2e6]");
+  DeviceInfo dev;
+  int rc = device_info(&dev);
+  if (rc) return rc;
+  moba::selftest_wait_kernel<<<1, 32, 0, stream>>>((uint64_t)timeout_us * 2000ull);
+  MOBA_CUDA(cudaGetLastError());
+  return finish_call(MOBA_OK, stream);
 }
 
 // ------------------------------------------------------------ no allocation
@@ -1205,5 +1268,7 @@ extern "C" int moba_fwd_noalloc(const void* q, const void* k, const void* v, int
   void* scratch = nullptr;
   rc = noalloc_scratch(&scratch);
   if (rc) return rc;
-  return run_forward(p, dev, q, k, v, out, lse, static_cast<uint8_t*>(scratch), stream);
+  rc = take_pending_status(dev, stream);
+  if (rc) return rc;
+  return finish_call(run_forward(p, dev, q, k, v, out, lse, static_cast<uint8_t*>(scratch), stream), stream);
 }

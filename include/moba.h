@@ -39,7 +39,11 @@
  * moba_status; moba_last_error() then gives a message (thread-local). Device
  * side faults that the kernels detect (a bounded wait that ran out, an index
  * check) are recorded in a per-device status word that moba_device_status()
- * reads after synchronising the stream.
+ * reads after synchronising the stream. The kernels also store the code in a
+ * host-mapped copy, so the next call on the device (any entry point that
+ * launches) returns it before launching anything, once, and clears it. With
+ * the environment variable MOBA_SYNC=1, every call synchronises its stream
+ * and returns that status itself.
  */
 #ifndef MOBA_B200_H
 #define MOBA_B200_H
@@ -279,6 +283,13 @@ int moba_device_status(cudaStream_t stream);
  * bounded-wait helper the attention kernel uses, without faulting the GPU.
  */
 int moba_selftest_bounded_wait(int timeout_us, cudaStream_t stream);
+
+/*
+ * The same kernel, launched without reading the status afterwards: the next
+ * call on the device reports MOBA_ERR_DEVICE_TIMEOUT (or this call does, with
+ * MOBA_SYNC=1). Exercises the error reporting of the other entry points.
+ */
+int moba_selftest_bounded_wait_async(int timeout_us, cudaStream_t stream);
 
 #ifdef __cplusplus
 }

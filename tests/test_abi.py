@@ -134,3 +134,8 @@ def test_backward_rejects_bad_arguments_before_launch(lib):
     assert rc == moba.MOBA_ERR_INVALID_ARG and "head_dim" in moba.last_error()
     rc = lib.moba_bwd(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE + 8, 4096, 1, 1, 128, 512, 3, FAKE, FAKE, FAKE, None)
     assert rc == moba.MOBA_ERR_INVALID_ARG and "aligned" in moba.last_error()
+
+
+def test_async_selftest_checks_its_bound_before_launch(lib):
+    assert lib.moba_selftest_bounded_wait_async(0, None) == moba.MOBA_ERR_INVALID_ARG
+    assert lib.moba_selftest_bounded_wait_async(3000000, None) == moba.MOBA_ERR_INVALID_ARG

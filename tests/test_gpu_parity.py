@@ -149,6 +149,37 @@ def test_bounded_wait_reports_timeout():
     assert moba.device_status() == 0  # cleared by the read
 
 
+def test_an_earlier_device_error_is_reported_by_the_next_call():
+    # a kernel whose bounded wait runs out, launched without reading the
+    # status: the next call returns that code before launching, once
+    import block_sparse_long_fwd_b200 as moba
+    S, Hq, Hkv, B, topk = 1000, 2, 1, 256, 3
+    _, q, k, v = make_inputs(S, Hq, Hkv, B, topk, 5)
+    qd, kd, vd = (torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).cuda() for a in (q, k, v))
+    stream = torch.cuda.current_stream().cuda_stream
+    assert moba.lib().moba_selftest_bounded_wait_async(20000, stream) == moba.MOBA_OK
+    torch.cuda.synchronize()
+    with pytest.raises(moba.MobaError) as err:
+        moba.fwd(qd, kd, vd, B, topk)
+    assert err.value.code == moba.MOBA_ERR_DEVICE_TIMEOUT
+    out, lse = moba.fwd(qd, kd, vd, B, topk)  # reported once: this call runs
+    torch.cuda.synchronize()
+    assert moba.device_status() == moba.MOBA_OK
+    assert torch.isfinite(lse).all()
+
+
+def test_sync_mode_returns_the_device_status_from_the_call(monkeypatch):
+    import block_sparse_long_fwd_b200 as moba
+    monkeypatch.setenv("MOBA_SYNC", "1")
+    stream = torch.cuda.current_stream().cuda_stream
+    assert moba.lib().moba_selftest_bounded_wait_async(20000, stream) == moba.MOBA_ERR_DEVICE_TIMEOUT
+    S, Hq, Hkv, B, topk = 1000, 2, 1, 256, 3
+    _, q, k, v = make_inputs(S, Hq, Hkv, B, topk, 6)
+    qd, kd, vd = (torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).cuda() for a in (q, k, v))
+    moba.fwd(qd, kd, vd, B, topk)  # a clean call returns MOBA_OK after synchronising
+    assert moba.device_status() == moba.MOBA_OK
+
+
 def test_host_entry_point_matches_device_entry_point():
     import block_sparse_long_fwd_b200 as moba
     S, Hq, Hkv, B, topk = 3000, 4, 2, 256, 3
