@@ -708,19 +708,22 @@ def main():
     if args.seqlen:
         w = si.Workload(f"{w.name}_s{args.seqlen}", args.seqlen, w.heads_q, w.heads_kv, w.head_dim, w.block_size,
                         w.topk, w.seed)
+    # one timed mode at a time, checked before any GPU work
+    if sum(bool(x) for x in (args.chunk, args.varlen, args.backward)) > 1:
+        ap.error("--chunk, --varlen and --backward are separate modes: give at most one")
+    if args.cached_means and not args.chunk:
+        ap.error("--cached-means applies to --chunk")
+    if args.chunk and not 1 <= args.chunk <= w.seqlen:
+        ap.error("--chunk must be in [1, seqlen]")
+    if args.varlen and not 1 <= args.varlen <= w.seqlen:
+        ap.error("--varlen must be in [1, seqlen]")
     if args.impl == "reference":
         return run_reference(args, w)
     if args.chunk:
-        if not 1 <= args.chunk <= w.seqlen:
-            ap.error("--chunk must be in [1, seqlen]")
         return run_chunk(args, w)
     if args.backward:
-        if args.chunk or args.varlen:
-            ap.error("--backward does not combine with --chunk or --varlen")
         return run_backward(args, w)
     if args.varlen:
-        if not 1 <= args.varlen <= w.seqlen or args.chunk:
-            ap.error("--varlen must be in [1, seqlen] and not combined with --chunk")
         return run_varlen(args, w)
     return run_ours(args, w)
 
