@@ -37,7 +37,7 @@ def test_chunk_flops_of_the_whole_sequence_match_the_library_count():
     ["--varlen", "3", "--chunk", "2"],
     ["--warmup", "2"],
     ["--cached-means"],
-    ["--chunk", "0", "--backward"],
+    ["--chunk", "-1"],
 ])
 def test_incompatible_modes_are_rejected_before_any_gpu_work(args):
     r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py")] + args, capture_output=True, text=True,
