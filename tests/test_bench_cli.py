@@ -44,3 +44,18 @@ def test_incompatible_modes_are_rejected_before_any_gpu_work(args):
                        timeout=300, cwd=ROOT)
     assert r.returncode == 2, r.stderr[-500:]
     assert "error" in r.stderr
+
+
+@pytest.mark.parametrize("name,shape,flops", [
+    ("4k", (4096, 1, 1, 512, 3), 2.28e9),
+    ("32k", (32768, 1, 1, 2048, 3), 7.95e10),
+    ("128k", (131072, 32, 8, 4096, 12), 8.30e13),
+    ("1m", (1048576, 32, 8, 4096, 12), 7.91e14),
+    ("10m", (10485760, 1, 1, 8192, 12), 5.04e14),
+])
+def test_workloads_and_their_flops_match_the_config_table(name, shape, flops):
+    # the five configurations and their effective (selected-block) FLOPs:
+    # 4*d*Hq per unmasked (query, key) pair, own block causal
+    w = si.WORKLOADS[name]
+    assert (w.seqlen, w.heads_q, w.heads_kv, w.block_size, w.topk) == shape and w.head_dim == 128
+    assert bench.chunk_flops(w, 0) == pytest.approx(flops, rel=5e-3)
