@@ -1,9 +1,11 @@
 #!/usr/bin/env python
 """Benchmark of the B200 MoBA causal prefill forward pass.
 
-`python bench.py --gpus N --steps K --warmup W [--config 32k]` prints one JSON
+`python bench.py --gpus N --steps K --warmup W [--config 1m]` prints one JSON
 line. A step is one whole forward pass (pool, gate, router, attention, merge)
-over one synthetic sequence resident in HBM. With N > 1 (launched by
+over one synthetic sequence resident in HBM. The default workload is the
+1M-token one (32 q / 8 kv heads, block 4096, top-12): the largest single-GPU
+configuration, with the most work of the five. With N > 1 (launched by
 torch.distributed.run) every rank runs its own independent sequence: weak
 scaling, no collective on the data path (a MAX all-reduce of the timings
 only).
@@ -208,7 +210,7 @@ def run_reference(args, w):
     rank, world, _ = dist_env()
     if rank != 0:
         return 0
-    per_step = 3.0
+    per_step = 2.0
     q, k, v, m, t_pool, run, n, threads = oracle_sample(w, per_step, w.seed + 4242)
     for _ in range(args.warmup):
         run(max(n // 8, 1))
@@ -688,7 +690,7 @@ def main():
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--config", choices=sorted(si.WORKLOADS), default="32k")
+    ap.add_argument("--config", choices=sorted(si.WORKLOADS), default="1m")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--seqlen", type=int, default=0, help="override the workload's seqlen (profiling cases)")

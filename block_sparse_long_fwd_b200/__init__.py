@@ -46,6 +46,7 @@ SIGNATURES = {
     "moba_device_status": (_i32, [_vp]),
     "moba_selftest_bounded_wait": (_i32, [_i32, _vp]),
     "moba_selftest_bounded_wait_async": (_i32, [_i32, _vp]),
+    "moba_selftest_device_check": (_i32, [_vp]),
 }
 
 

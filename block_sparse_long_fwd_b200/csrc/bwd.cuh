@@ -413,6 +413,7 @@ __global__ void __launch_bounds__(256) bwd_dq_reduce_kernel(const int32_t* __res
     if (j < 0 || j >= bt) continue;
     const int64_t f = ((int64_t)g * w.nbp + j) * w.wwords + word;
     const int64_t pos = (int64_t)__ldg(wordbase + f) + __popc(__ldg(flags + f) & below);
+    if (!slot_ok(w, pos)) continue;
     const float4 o = load_half4(part_o + pos * kHeadDim + lane * 4);
     acc.x += o.x;
     acc.y += o.y;

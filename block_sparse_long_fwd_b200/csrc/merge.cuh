@@ -83,6 +83,7 @@ __global__ void __launch_bounds__(256) merge_kernel(MergeParams m) {
     if (j < 0 || j >= bt) return -1;
     const int64_t f = ((int64_t)g * w.nbp + j) * w.wwords + word;
     const int64_t pos = (int64_t)__ldg(m.wordbase + f) + __popc(__ldg(m.flags + f) & below);
+    if (!slot_ok(w, pos)) return -1;
     li = __ldg(m.part_lse + pos);
     return pos;
   };

@@ -100,11 +100,6 @@ int device_info(DeviceInfo* out) {
       MOBA_CUDA(cudaHostGetDevicePointer(reinterpret_cast<void**>(&hd), h, 0));
       MOBA_CUDA(cudaMemcpyToSymbol(moba::g_status_mirror, &hd, sizeof(hd)));
       d.status_host = h;
-      // keep freed scratch in the stream-ordered pool between calls
-      cudaMemPool_t pool;
-      MOBA_CUDA(cudaDeviceGetDefaultMemPool(&pool, dev));
-      uint64_t thr = UINT64_MAX;
-      MOBA_CUDA(cudaMemPoolSetAttribute(pool, cudaMemPoolAttrReleaseThreshold, &thr));
     }
     if (!g_encode) {
       cudaDriverEntryPointQueryResult q;
@@ -481,6 +476,7 @@ moba::WindowGeom window_geom(const Plan& p, int64_t w0) {
   wg.q0 = p.q0;
   wg.wwords = (wg.wlen * p.G + 31) / 32;
   wg.pair_tokens = pair_tokens(p) ? 1 : 0;
+  wg.list_cap = std::max<int64_t>(p.list_cap, 1);
   return wg;
 }
 
@@ -755,9 +751,42 @@ namespace {
 // A launch sequence over one scratch buffer of `total` bytes.
 using Runner = std::function<int(uint8_t* ws, cudaStream_t st)>;
 
+bool g_pool_kept[64] = {};
+
+// The entry points that take stream-ordered scratch raise the release
+// threshold of the device's default pool once, so scratch freed at the end
+// of a call stays reserved for the next one. (moba_fwd_noalloc never gets
+// here: it leaves the caller's allocator alone.)
+void keep_freed_scratch() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
+    cudaGetLastError();
+    return;
+  }
+  std::lock_guard<std::mutex> lk(g_dev_mu);
+  if (g_pool_kept[dev]) return;
+  cudaMemPool_t pool;
+  if (cudaDeviceGetDefaultMemPool(&pool, dev) == cudaSuccess) {
+    uint64_t thr = UINT64_MAX;
+    cudaMemPoolSetAttribute(pool, cudaMemPoolAttrReleaseThreshold, &thr);
+  }
+  cudaGetLastError();
+  g_pool_kept[dev] = true;
+}
+
+// Bytes to request for `total` bytes of scratch. MOBA_TEST_SCRATCH_PAD=<n>
+// adds n bytes to every request: a test hook that makes the stream-ordered
+// allocation fail on purpose, so the MOBA_ERR_OOM path can be exercised.
+size_t scratch_request(size_t total) {
+  const char* e = getenv("MOBA_TEST_SCRATCH_PAD");
+  return e ? total + (size_t)strtoull(e, nullptr, 10) : total;
+}
+
 // The launch sequence with stream-ordered scratch, issued on `stream`.
 int direct_run(size_t total, const Runner& run, cudaStream_t stream) {
+  keep_freed_scratch();
   void* ws = nullptr;
+  total = scratch_request(total);
   cudaError_t e = cudaMallocAsync(&ws, total, stream);
   if (e != cudaSuccess) {
     cudaGetLastError();
@@ -811,7 +840,8 @@ bool graphs_enabled() {
 // MOBA_OK / error after launching a graph; -1 when the caller should launch
 // directly. key.dev is filled in here.
 int graph_run(GraphKey key, size_t total, const Runner& run, cudaStream_t stream) {
-  if (!graphs_enabled()) return -1;
+  if (!graphs_enabled() || getenv("MOBA_TEST_SCRATCH_PAD")) return -1;
+  keep_freed_scratch();
   int d = 0;
   if (cudaGetDevice(&d) != cudaSuccess || d < 0 || d >= 64) return -1;
   key.dev = d;
@@ -1047,6 +1077,7 @@ int moba_fwd_host(const void* q_host, const void* k_host, const void* v_host, in
   const size_t lb = (size_t)seqlen * heads_q * 4;
   Carve c;
   const size_t oq = c.take(qb), ok = c.take(kb), ov = c.take(kb), oo = c.take(qb), ol = c.take(lb);
+  keep_freed_scratch();
   void* buf = nullptr;
   cudaError_t e = cudaMallocAsync(&buf, c.off, stream);
   if (e != cudaSuccess) {
@@ -1121,6 +1152,7 @@ int moba_gate(const void* q, const float* kmean, int64_t seqlen, int heads_q, in
   p.P = p.k_eff - 1;
   // bf16 hi/lo parts of the means: stream-ordered scratch for this call
   const size_t part = (size_t)heads_kv * moba::gate_rows_padded(std::max(p.nbp, 1)) * moba::kHeadDim * 2;
+  keep_freed_scratch();
   void* parts = nullptr;
   cudaError_t e = cudaMallocAsync(&parts, 2 * part, stream);
   if (e != cudaSuccess) {
@@ -1180,6 +1212,72 @@ extern "C" int moba_selftest_bounded_wait(int timeout_us, cudaStream_t stream) {
   moba::selftest_wait_kernel<<<1, 32, 0, stream>>>((uint64_t)timeout_us * 2000ull);
   MOBA_CUDA(cudaGetLastError());
   return moba_device_status(stream);
+}
+
+// A tiny merge whose router tables are inconsistent on purpose: rows
+// 128..255 of a 256-token, 2-block problem route to past block 0, but the
+// flag words' list slots start at 2^20 while the list holds one entry. The
+// merge kernel must record MOBA_ERR_DEVICE_CHECK and skip those reads (it
+// never touches memory outside the buffers allocated here).
+extern "C" int moba_selftest_device_check(cudaStream_t stream) {
+  g_err.clear();
+  DeviceInfo dev;
+  int rc = device_info(&dev);
+  if (rc) return rc;
+  rc = moba_device_status(stream);  // clear earlier state
+  if (rc) return rc;
+  constexpr int S = 256, K = 2, WW = 8;
+  std::vector<int32_t> sel(S * K), wordbase(WW, 1 << 20);
+  std::vector<uint32_t> flags(WW, 0u);
+  for (int t = 0; t < S; ++t) {  // t < 128: own block 0 only; else past block 0, own block 1
+    sel[t * K] = 0;
+    sel[t * K + 1] = t < 128 ? -1 : 1;
+  }
+  for (int w = 4; w < WW; ++w) flags[w] = 0xFFFFFFFFu;
+  Carve c;
+  const size_t o_sel = c.take(sel.size() * 4), o_flags = c.take(WW * 4), o_wb = c.take(WW * 4),
+               o_po = c.take(moba::kHeadDim * 2), o_pl = c.take(4), o_oo = c.take((size_t)S * moba::kHeadDim * 2),
+               o_ol = c.take(S * 4), o_out = c.take((size_t)S * moba::kHeadDim * 2), o_lse = c.take(S * 4);
+  uint8_t* b = nullptr;
+  MOBA_CUDA(cudaMalloc(reinterpret_cast<void**>(&b), c.off));
+  rc = MOBA_OK;
+  if (cudaMemsetAsync(b, 0, c.off, stream) != cudaSuccess ||
+      cudaMemcpyAsync(b + o_sel, sel.data(), sel.size() * 4, cudaMemcpyHostToDevice, stream) != cudaSuccess ||
+      cudaMemcpyAsync(b + o_flags, flags.data(), WW * 4, cudaMemcpyHostToDevice, stream) != cudaSuccess ||
+      cudaMemcpyAsync(b + o_wb, wordbase.data(), WW * 4, cudaMemcpyHostToDevice, stream) != cudaSuccess)
+    rc = fail(MOBA_ERR_CUDA, "self-test set-up failed: %s", cudaGetErrorString(cudaGetLastError()));
+  if (!rc) {
+    moba::MergeParams mp;
+    mp.sel = reinterpret_cast<const int32_t*>(b + o_sel);
+    mp.flags = reinterpret_cast<const uint32_t*>(b + o_flags);
+    mp.wordbase = reinterpret_cast<const int32_t*>(b + o_wb);
+    mp.part_o = reinterpret_cast<const __half*>(b + o_po);
+    mp.part_lse = reinterpret_cast<const float*>(b + o_pl);
+    mp.own_o = reinterpret_cast<const __half*>(b + o_oo);
+    mp.own_lse = reinterpret_cast<const float*>(b + o_ol);
+    mp.out = reinterpret_cast<__nv_bfloat16*>(b + o_out);
+    mp.lse = reinterpret_cast<float*>(b + o_lse);
+    mp.lse_ld = S;
+    moba::WindowGeom& w = mp.w;
+    w.S = S;
+    w.Hq = w.Hkv = w.G = 1;
+    w.B = 128;
+    w.k_eff = K;
+    w.nbp = 1;
+    w.w0 = 0;
+    w.wlen = S;
+    w.wwords = WW;
+    w.pair_tokens = 0;
+    w.q0 = 0;
+    w.list_cap = 1;
+    moba::merge_kernel<0><<<S / 8, 256, 0, stream>>>(mp);
+    if (cudaGetLastError() != cudaSuccess) rc = fail(MOBA_ERR_CUDA, "self-test launch failed");
+  }
+  const int st = moba_device_status(stream);
+  cudaFree(b);
+  if (rc) return rc;
+  if (st) fail(st, "the merge kernel reported device status %d", st);
+  return st;
 }
 
 extern "C" int moba_selftest_bounded_wait_async(int timeout_us, cudaStream_t stream) {

@@ -32,7 +32,17 @@ struct WindowGeom {
   int64_t wwords;    // flag words per bucket: ceil(wlen * G / 32)
   int pair_tokens;   // own units pair consecutive 128-token tiles of one head
   int64_t q0;        // first token with a query (0 for a whole prefill); sel rows start there
+  int64_t list_cap;  // routed list slots the scratch holds (every slot index is checked against it)
 };
+
+// A list slot outside [0, list_cap) means the router's tables are
+// inconsistent: the kernel records MOBA_ERR_DEVICE_CHECK and skips the
+// access instead of touching memory outside the scratch.
+__device__ __forceinline__ bool slot_ok(const WindowGeom& w, int64_t pos, int64_t n = 1) {
+  if (pos >= 0 && pos + n <= w.list_cap) return true;
+  record_status(MOBA_ERR_DEVICE_CHECK);
+  return false;
+}
 
 // First flag word of bucket j that can hold a set bit: rows with t >= (j+1)B.
 __device__ __forceinline__ int64_t bucket_word_begin(const WindowGeom& w, int j) {
@@ -264,6 +274,7 @@ __global__ void __launch_bounds__(256) route_fill_kernel(const uint32_t* __restr
     if (i < w.wwords) {
       int pos = base + running + before + incl - c;
       wordbase[foff + i] = pos;
+      if (!slot_ok(w, pos, c)) word = 0u;
       while (word) {
         const int bit = __ffs(word) - 1;
         word &= word - 1;

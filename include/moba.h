@@ -37,13 +37,21 @@
  *
  * Errors: argument checks run before any launch and return a nonzero
  * moba_status; moba_last_error() then gives a message (thread-local). Device
- * side faults that the kernels detect (a bounded wait that ran out, an index
- * check) are recorded in a per-device status word that moba_device_status()
- * reads after synchronising the stream. The kernels also store the code in a
- * host-mapped copy, so the next call on the device (any entry point that
- * launches) returns it before launching anything, once, and clears it. With
- * the environment variable MOBA_SYNC=1, every call synchronises its stream
- * and returns that status itself.
+ * side faults that the kernels detect are recorded in a per-device status
+ * word that moba_device_status() reads after synchronising the stream: a
+ * bounded wait that ran out (MOBA_ERR_DEVICE_TIMEOUT), or a router list slot
+ * outside the scratch's list (MOBA_ERR_DEVICE_CHECK; the kernel skips that
+ * access). The kernels also store the code in a host-mapped copy, so the next
+ * call on the device (any entry point that launches) returns it before
+ * launching anything, once, and clears it. With the environment variable
+ * MOBA_SYNC=1, every call synchronises its stream and returns that status
+ * itself. A failed scratch allocation returns MOBA_ERR_OOM; the environment
+ * variable MOBA_TEST_SCRATCH_PAD=<bytes> (a test hook) adds that many bytes
+ * to every scratch request so that this path can be exercised.
+ *
+ * Value range: routed and own-block partial outputs are kept in fp16 between
+ * the attention and merge stages, so v must hold finite values of magnitude
+ * below 65504 (each partial output is a convex combination of v rows).
  */
 #ifndef MOBA_B200_H
 #define MOBA_B200_H
@@ -62,7 +70,7 @@ typedef enum {
     MOBA_ERR_OOM = 3,            /* scratch allocation failed              */
     MOBA_ERR_CUDA = 4,           /* a CUDA runtime call failed             */
     MOBA_ERR_DEVICE_TIMEOUT = 5, /* a kernel's bounded wait ran out        */
-    MOBA_ERR_DEVICE_CHECK = 6    /* a kernel's index check failed          */
+    MOBA_ERR_DEVICE_CHECK = 6    /* a kernel found a list slot out of range */
 } moba_status;
 
 /* Limits checked before launch. */
@@ -210,8 +218,13 @@ int moba_fwd_host(const void* q_host, const void* k_host, const void* v_host,
 /*
  * moba_pool - the first stage alone: kmean[g][j][:] = mean of k[t][g][:]
  * over the tokens t of block j, for j < nblocks - 1 (fp32 accumulation, fixed
- * order). kmean is a device fp32 buffer [heads_kv][nblocks-1][head_dim].
- * Does nothing when nblocks == 1.
+ * order). The blocks are the method's partition of the context into
+ * block_size consecutive tokens ("MoBA (Mixture of Block Attention)" project
+ * summary, "How It Works"); the mean is what the gate scores a query
+ * against (the pages call the gate parameter-less without printing its
+ * score; this library takes the inner product with the block's mean key).
+ * kmean is a device fp32 buffer [heads_kv][nblocks-1][head_dim]. Does
+ * nothing when nblocks == 1. Errors as moba_fwd.
  */
 int moba_pool(const void* k, int64_t seqlen, int heads_kv, int head_dim,
               int block_size, float* kmean, cudaStream_t stream);
@@ -219,7 +232,13 @@ int moba_pool(const void* k, int64_t seqlen, int heads_kv, int head_dim,
 /*
  * moba_gate - the second stage alone: gate scores q . kmean over past blocks
  * and the per-row top-(k-1) with the own block forced, written as `sel`
- * (layout above). kmean as produced by moba_pool.
+ * (layout above): the parameter-less top-k gate of "MoBA (Mixture of Block
+ * Attention)" project summary, "How It Works", with the causal rules of
+ * "MoBA - Moonshot AIが提案した新しいアテンションメカニズム",
+ * "MoBAの技術的原則" (no future block; the own block always chosen). Ties go
+ * to the lower block index. kmean as produced by moba_pool (it may be NULL
+ * when no row chooses: topk 1, or topk >= nblocks). sel is a device int32
+ * buffer the caller owns. Errors as moba_fwd.
  */
 int moba_gate(const void* q, const float* kmean, int64_t seqlen, int heads_q,
               int heads_kv, int head_dim, int block_size, int topk,
@@ -252,12 +271,18 @@ int moba_profile_end(float* stage_ms, int* launches, int* calls);
  * allocating library routine. Problems whose scratch would not fit in the
  * array (the selection table and at least a 128-token query window) are
  * rejected with MOBA_ERR_UNSUPPORTED before any launch; moba_fwd handles
- * them. The first call on a device looks up the array's device address
- * (cudaGetSymbolAddress) with that device current; make that first call
- * before any stream capture. Every call shares the one array: calls that
- * overlap on the GPU (different streams, or threads) race on it and must be
- * serialised by the caller. Nothing in the array needs to start at zero;
- * every call writes each part before reading it.
+ * them. The first call on a device (of this or any other entry point) does
+ * the library's one-time set-up for that device: it reads device attributes,
+ * sets the kernels' shared-memory limits, pins one 4-byte host word
+ * (cudaHostAlloc, mapped) that mirrors the device status, loads the module
+ * (which maps the 64 MiB array) and looks up the array's device address
+ * (cudaGetSymbolAddress) with that device current. A caller that must not
+ * allocate at all at run time makes that first call during its own set-up,
+ * and before any stream capture. This entry point never changes the
+ * stream-ordered allocator's settings. Every call shares the one array:
+ * calls that overlap on the GPU (different streams, or threads) race on it
+ * and must be serialised by the caller. Nothing in the array needs to start
+ * at zero; every call writes each part before reading it.
  */
 int moba_fwd_noalloc(const void* q, const void* k, const void* v,
                      int64_t seqlen, int heads_q, int heads_kv, int head_dim,
@@ -270,7 +295,7 @@ const char* moba_last_error(void);
 /*
  * Synchronises `stream`, then returns and clears the status word that the
  * kernels on the current device write when a bounded wait runs out
- * (MOBA_ERR_DEVICE_TIMEOUT) or an index check fails (MOBA_ERR_DEVICE_CHECK);
+ * (MOBA_ERR_DEVICE_TIMEOUT) or a list slot check fails (MOBA_ERR_DEVICE_CHECK);
  * MOBA_OK when neither happened. The word is shared by every call on the
  * device since the last read.
  */
@@ -283,6 +308,15 @@ int moba_device_status(cudaStream_t stream);
  * bounded-wait helper the attention kernel uses, without faulting the GPU.
  */
 int moba_selftest_bounded_wait(int timeout_us, cudaStream_t stream);
+
+/*
+ * Runs the merge kernel once on a tiny problem whose router tables point a
+ * routed partial outside the list (the scratch of this call is its own
+ * small cudaMalloc'd buffer), and returns the status it leaves:
+ * MOBA_ERR_DEVICE_CHECK when the kernel's slot check caught it and skipped
+ * the read. No access leaves the allocated buffers.
+ */
+int moba_selftest_device_check(cudaStream_t stream);
 
 /*
  * The same kernel, launched without reading the status afterwards: the next

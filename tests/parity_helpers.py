@@ -26,6 +26,12 @@ def to_dev(a: np.ndarray) -> torch.Tensor:
     return torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).cuda()
 
 
+def bf16_bits(x) -> np.ndarray:
+    """fp32 values rounded to nearest-even bf16, as uint16 bit patterns."""
+    u = np.ascontiguousarray(x, dtype=np.float32).view(np.uint32).astype(np.uint64)
+    return ((u + 0x7FFF + ((u >> 16) & 1)) >> 16).astype(np.uint16)
+
+
 def make_inputs(S, Hq, Hkv, B, topk, seed):
     w = si.Workload("case", S, Hq, Hkv, 128, B, topk, seed)
     q, k, v = si.make_qkv(w)

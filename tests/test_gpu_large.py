@@ -1,0 +1,111 @@
+"""GPU parity on the three large workloads, in the configuration the benchmark
+times, on the slices the workload specification names.
+
+For each workload the whole forward pass runs on the GPU once, then:
+  - the selection table is compared with the oracle's gate on EVERY row and
+    head (bit-exact wherever the oracle's gap at the cut exceeds 1e-3
+    relative; below that the GPU's set must score within 1e-3 of the cut);
+  - outputs and lse are compared with the oracle on a slice:
+      128K: 4,096 uniformly drawn rows plus edge rows, the q head cycling
+            through all 32 heads;
+      1M:   every row of the first 65,536 tokens, for one q head per kv
+            group (head 4g + g mod 4 of group g, so every position in a
+            group is covered); by causality these rows depend on the prefix
+            alone ("MoBA - Moonshot AIが提案した新しいアテンションメカニズム",
+            "MoBAの技術的原則"), so the oracle runs on the prefix as its own
+            65,536-token problem; plus 2,048 rows drawn over the whole
+            sequence (all heads) and the last window's edge rows;
+      10M:  4,096 uniformly drawn rows plus the rows 0, B-1, B, 2B-1, S/2
+            and S-1.
+The 1M prefix check uses one q head per kv group (8 of 32 heads) to keep
+the oracle's share of the GPU test run to a few minutes.
+"""
+import numpy as np
+import pytest
+
+import oracle
+import synth_inputs as si
+from parity_helpers import check_sel_structure, check_selection, compare_outputs, run_gpu
+
+pytestmark = pytest.mark.gpu
+
+torch = pytest.importorskip("torch")
+if not torch.cuda.is_available():  # pragma: no cover
+    pytest.skip("no CUDA device", allow_module_level=True)
+
+
+def edge_rows(w):
+    S, B = w.seqlen, w.block_size
+    return np.array([0, B - 1, B, 2 * B - 1, S // 2, S - 1], dtype=np.int64)
+
+
+def drawn_rows(w, n, seed, heads="cycle"):
+    rng = np.random.default_rng(seed)
+    t = np.concatenate([edge_rows(w), rng.choice(w.seqlen, size=n, replace=False).astype(np.int64)])
+    h = (np.arange(t.size) % w.heads_q).astype(np.int32)
+    rng.shuffle(h)
+    return t, h
+
+
+def check_all_selections(q, k, sel_g, w, m):
+    """The GPU selection of every (token, head) row against the oracle's gate."""
+    S, Hq = w.seqlen, w.heads_q
+    rows_t = np.arange(S, dtype=np.int64)
+    near = 0
+    for h in range(Hq):
+        _, n = check_selection(q, k, sel_g[h], rows_t, np.full(S, h, dtype=np.int32), w.block_size, w.heads_kv,
+                               w.topk, m)
+        near += n
+    return near
+
+
+def check_rows(qo, ko, vo, w, out_g, lse_g, sel_g, rows_t, rows_h):
+    """Outputs of the given rows against the oracle run on (qo, ko, vo), which
+    hold the whole sequence or a prefix of it that contains every row."""
+    sel_rows = sel_g[rows_h, rows_t]  # already checked against the oracle's gate
+    out_o, lse_o, _ = oracle.attend(qo, ko, vo, w.block_size, w.topk, rows_t, rows_h, sel=sel_rows)
+    out_rows = out_g[torch.from_numpy(rows_t), torch.from_numpy(rows_h.astype(np.int64))].float().numpy()
+    return compare_outputs(out_rows, lse_g[rows_h, rows_t], out_o, lse_o)
+
+
+def run_workload(name):
+    w = si.WORKLOADS[name]
+    q, k, v = si.make_qkv(w)
+    out_g, lse_g, sel_g, kmean_g = run_gpu(q, k, v, w.block_size, w.topk)
+    m = oracle.kmean(k, w.block_size)
+    nbp = w.nblocks - 1
+    np.testing.assert_allclose(kmean_g, m[:, :nbp], rtol=1e-5, atol=1e-5)
+    check_sel_structure(sel_g, w.seqlen, w.block_size, w.topk)
+    near = check_all_selections(q, k, sel_g, w, m)
+    return w, q, k, v, out_g, lse_g, sel_g, near
+
+
+def test_128k_every_selection_and_4096_rows_over_all_heads():
+    w, q, k, v, out_g, lse_g, sel_g, near = run_workload("128k")
+    rows_t, rows_h = drawn_rows(w, 4096, w.seed + 1000)
+    assert set(rows_h.tolist()) == set(range(w.heads_q))
+    stats = check_rows(q, k, v, w, out_g, lse_g, sel_g, rows_t, rows_h)
+    print(dict(stats, near_ties=near, rows=int(rows_t.size)))
+
+
+def test_1m_every_selection_and_the_64k_prefix():
+    w, q, k, v, out_g, lse_g, sel_g, near = run_workload("1m")
+    P, G = 65536, w.heads_q // w.heads_kv
+    heads = np.array([g * G + g % G for g in range(w.heads_kv)], dtype=np.int32)
+    rows_t = np.repeat(np.arange(P, dtype=np.int64), heads.size)
+    rows_h = np.tile(heads, P)
+    pre = check_rows(q[:P], k[:P], v[:P], w, out_g, lse_g, sel_g, rows_t, rows_h)
+    # beyond the prefix: drawn rows over the whole sequence and the last tokens
+    dt, dh = drawn_rows(w, 2048, w.seed + 1000)
+    tail = np.arange(w.seqlen - 8, w.seqlen, dtype=np.int64)
+    dt = np.concatenate([dt, tail])
+    dh = np.concatenate([dh, (np.arange(tail.size) * 5 % w.heads_q).astype(np.int32)])
+    full = check_rows(q, k, v, w, out_g, lse_g, sel_g, dt, dh)
+    print({"prefix": pre, "drawn": full, "near_ties": near, "prefix_rows": int(rows_t.size)})
+
+
+def test_10m_every_selection_and_4096_rows():
+    w, q, k, v, out_g, lse_g, sel_g, near = run_workload("10m")
+    rows_t, rows_h = drawn_rows(w, 4096, w.seed + 1000)
+    stats = check_rows(q, k, v, w, out_g, lse_g, sel_g, rows_t, rows_h)
+    print(dict(stats, near_ties=near, rows=int(rows_t.size)))

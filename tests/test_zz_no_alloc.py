@@ -11,12 +11,12 @@ call finds the array holding the first call's contents).
 The file name sorts last so that a run that stops at the first failure has
 already run every other test.
 """
-import ctypes
-
 import numpy as np
 import pytest
 
-from parity_helpers import LSE_ABS, OUT_MAX_ABS, OUT_MEAN_ABS, make_inputs, to_dev
+import oracle
+from parity_helpers import (LSE_ABS, OUT_MAX_ABS, OUT_MEAN_ABS, check_selection, compare_outputs, make_inputs,
+                            to_dev)
 
 pytestmark = pytest.mark.gpu
 
@@ -72,12 +72,56 @@ def test_other_inputs_after_a_previous_call():
     got = call("moba_fwd_noalloc", q2d, k2d, v2d, 128, 3)
     ref = call("moba_fwd", q2d, k2d, v2d, 128, 3)
     torch.cuda.synchronize()
+    assert moba.device_status() == moba.MOBA_OK
     close(got, ref)
 
 
+def test_a_problem_that_needs_several_query_windows():
+    # The selection table (32768 x 16 x 8 x 4 B = 16.8 MB) fits in the fixed
+    # array but a whole-sequence query window (~0.9 GB of partial outputs)
+    # does not: the call must shrink its window and run several of them.
+    S, Hq, Hkv, B, topk = 32768, 16, 4, 2048, 8
+    _, q, k, v = make_inputs(S, Hq, Hkv, B, topk, 21)
+    qd, kd, vd = to_dev(q), to_dev(k), to_dev(v)
+    moba.profile_begin()
+    got = call("moba_fwd_noalloc", qd, kd, vd, B, topk)
+    _, launches, calls = moba.profile_end()
+    # pool and gate (3 kernels), then per window the router (1 kernel while the
+    # window holds no past block, else 4), attention and merge: one window
+    # would be at most 9 launches (1024-token windows here: 189)
+    assert calls == 1 and launches > 9, launches
+    again = call("moba_fwd_noalloc", qd, kd, vd, B, topk)
+    ref = call("moba_fwd", qd, kd, vd, B, topk)
+    torch.cuda.synchronize()
+    assert moba.device_status() == moba.MOBA_OK
+    close(got, ref)
+    close(again, ref)
+    # and against the oracle on drawn rows of every head
+    rng = np.random.default_rng(5)
+    rows_t = rng.choice(S, size=512, replace=False).astype(np.int64)
+    rows_h = (np.arange(512) % Hq).astype(np.int32)
+    sel = moba.gate(qd, moba.pool(kd, B), Hkv, B, topk).cpu().numpy()[rows_h, rows_t]
+    sel, _ = check_selection(q, k, sel, rows_t, rows_h, B, Hkv, topk)
+    out_o, lse_o, _ = oracle.attend(q, k, v, B, topk, rows_t, rows_h, sel=sel)
+    out, lse = got
+    compare_outputs(out[torch.from_numpy(rows_t), torch.from_numpy(rows_h.astype(np.int64))].float().cpu().numpy(),
+                    lse.cpu().numpy()[rows_h, rows_t], out_o, lse_o)
+
+
 def test_rejects_problems_beyond_the_fixed_scratch():
-    # 1M tokens x 32 heads needs a selection table far above the fixed array
-    fake = 0x1000
-    rc = moba.lib().moba_fwd_noalloc(fake, fake, fake, 1 << 20, 32, 8, 128, 4096, 12, fake, fake, None)
+    # 262144 tokens x 8 heads x top-8: the selection table alone (67 MB)
+    # exceeds the fixed array. Real, correctly sized buffers: were the check
+    # ever to let the call through, it would compute a valid result instead of
+    # touching memory it does not own, and fail the assertion below.
+    S, Hq, Hkv, B, topk = 262144, 8, 1, 128, 8
+    q = torch.zeros((S, Hq, 128), dtype=torch.bfloat16, device="cuda")
+    k = torch.zeros((S, Hkv, 128), dtype=torch.bfloat16, device="cuda")
+    v = torch.zeros_like(k)
+    out = torch.empty_like(q)
+    lse = torch.empty((Hq, S), dtype=torch.float32, device="cuda")
+    rc = moba.lib().moba_fwd_noalloc(q.data_ptr(), k.data_ptr(), v.data_ptr(), S, Hq, Hkv, 128, B, topk,
+                                     out.data_ptr(), lse.data_ptr(), torch.cuda.current_stream().cuda_stream)
     assert rc == moba.MOBA_ERR_UNSUPPORTED
     assert "too large for moba_fwd_noalloc" in moba.last_error()
+    torch.cuda.synchronize()
+    assert moba.device_status() == moba.MOBA_OK
