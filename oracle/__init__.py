@@ -104,14 +104,18 @@ def all_rows(S: int, Hq: int):
 
 def select(q: np.ndarray, m: np.ndarray, block_size: int, heads_kv: int, topk: int, rows_t, rows_h,
            nthreads: int | None = None):
-    """Selected blocks per row: (sel int32 [n][k_eff] ascending, -1 padded; info fp64 [n][3])."""
+    """Selected blocks per row: (sel int32 [n][k_eff] ascending, -1 padded; info fp64 [n][4]).
+
+    info[:, 0] is the gap at the cut relative to the row's largest |score|,
+    info[:, 1] the last chosen past score, info[:, 2] the first left out,
+    info[:, 3] the row's largest |score| over its past blocks."""
     q = _u16(q)
     S, Hq, d = q.shape
     m = np.ascontiguousarray(m, dtype=np.float64)
     rt, rh = _rows(rows_t, rows_h)
     k_eff = min(topk, nblocks(S, block_size))
     sel = np.empty((rt.size, k_eff), dtype=np.int32)
-    info = np.empty((rt.size, 3), dtype=np.float64)
+    info = np.empty((rt.size, 4), dtype=np.float64)
     lib().oracle_select(q.ctypes.data, m.ctypes.data, S, Hq, heads_kv, d, block_size, topk, rt.ctypes.data,
                         rh.ctypes.data, rt.size, sel.ctypes.data, info.ctypes.data, nthreads or threads())
     return sel, info

@@ -109,9 +109,13 @@ static int cmp_i32(const void* a, const void* b) {
  * descending, ties to the lower index). Written ascending into sel[0..k_eff),
  * padded with -1, k_eff = min(topk, nb).
  * info[0] = relative gap between the last selected and the first unselected
- *           past score, (s_a - s_b) / max(|s_a|, |s_b|); +inf when nothing
- *           was left out or nothing was chosen by score;
- * info[1] = s_a (the cut), info[2] = s_b. */
+ *           past score, (s_a - s_b) / max_j |s_j|, relative to the largest
+ *           score magnitude of the row's past blocks (a two-score
+ *           denominator max(|s_a|, |s_b|) vanishes as both approach zero,
+ *           where the gap says nothing about how well the ranking is
+ *           determined); +inf when nothing was left out or nothing was
+ *           chosen by score;
+ * info[1] = s_a (the cut), info[2] = s_b, info[3] = max_j |s_j|. */
 static void select_row(const uint16_t* q, const double* m, int64_t S, int Hq,
                        int Hkv, int d, int B, int topk, int64_t t, int h,
                        int32_t* sel, double* info, scored* work,
@@ -130,13 +134,15 @@ static void select_row(const uint16_t* q, const double* m, int64_t S, int Hq,
     for (int64_t i = 0; i < npast; ++i) sel[i] = (int32_t)work[i].j;
     qsort(sel, (size_t)npast, sizeof(int32_t), cmp_i32);
     sel[npast] = (int32_t)b;
+    double scale = 0.0;
+    for (int64_t j = 0; j < b; ++j) scale = fmax(scale, fabs(sbuf[j]));
     info[0] = INFINITY;
     info[1] = NAN;
     info[2] = NAN;
+    info[3] = scale;
     if (npast >= 1 && npast < b) {
         double sa = work[npast - 1].s, sb = work[npast].s;
-        double den = fmax(fabs(sa), fabs(sb));
-        info[0] = den > 0 ? (sa - sb) / den : 0.0;
+        info[0] = scale > 0 ? (sa - sb) / scale : 0.0;
         info[1] = sa;
         info[2] = sb;
     }
@@ -196,7 +202,7 @@ typedef struct {
     int64_t r0, r1;
     const int32_t* sel_in; /* [nrows][k_eff] or NULL */
     int32_t* sel_out;      /* [nrows][k_eff] or NULL */
-    double* info_out;      /* [nrows][3] or NULL */
+    double* info_out;      /* [nrows][4] or NULL */
     double* out;           /* [nrows][d] or NULL */
     double* lse;           /* [nrows] or NULL */
 } row_job;
@@ -213,7 +219,7 @@ static void* row_worker(void* arg) {
     int64_t* zu = (int64_t*)malloc(sizeof(int64_t) * (size_t)kmax);
     double* qd = (double*)malloc(sizeof(double) * (size_t)J->d);
     int32_t* selr = (int32_t*)malloc(sizeof(int32_t) * (size_t)k_eff);
-    double info[3];
+    double info[4];
     for (int64_t r = J->r0; r < J->r1; ++r) {
         int64_t t = J->rows_t[r];
         int h = J->rows_h[r];
@@ -225,7 +231,7 @@ static void* row_worker(void* arg) {
                        t, h, selr, info, work, sbuf);
             sel = selr;
             if (J->sel_out) memcpy(J->sel_out + r * k_eff, selr, sizeof(int32_t) * (size_t)k_eff);
-            if (J->info_out) memcpy(J->info_out + r * 3, info, sizeof(info));
+            if (J->info_out) memcpy(J->info_out + r * 4, info, sizeof(info));
         }
         if (J->out)
             attend_row(J->q, J->k, J->v, J->S, J->Hq, J->Hkv, J->d, J->B, t,

@@ -149,12 +149,15 @@ def test_select_gap_info():
     sel, info = oracle.select(q, m, B, Hkv, 3, rows_t, rows_h)
     for r, (t, h) in enumerate(zip(rows_t, rows_h)):
         b = t // B
-        s = np.sort(f64(q)[t, h] @ m[0, :b].T)[::-1]
+        raw = f64(q)[t, h] @ m[0, :b].T
+        s = np.sort(raw)[::-1]
+        scale = np.abs(raw).max() if b else 0.0
+        assert info[r, 3] == pytest.approx(scale, rel=1e-12, abs=1e-300)
         if 1 <= 2 < b:
             sa, sb = s[1], s[2]
             assert info[r, 1] == pytest.approx(sa, rel=1e-12)
             assert info[r, 2] == pytest.approx(sb, rel=1e-12)
-            assert info[r, 0] == pytest.approx((sa - sb) / max(abs(sa), abs(sb)), rel=1e-9, abs=1e-15)
+            assert info[r, 0] == pytest.approx((sa - sb) / scale, rel=1e-9, abs=1e-15)
         else:
             assert np.isinf(info[r, 0])
 
