@@ -16,21 +16,25 @@
 // natural-log lse_i; the merge stage combines them. The online softmax
 // (FlashAttention-style; the same page credits MoBA's speed to FlashAttention
 // plus MoE techniques) runs per 128-key step, per tile X in {A, B}:
-//   S_X = Q_X K^T      tcgen05.mma, Q and K from shared memory (128B
-//                      swizzle), fp32 accumulator in TMEM
+//   S_X = Q_X K^T      tcgen05.mma (M = N = 128), Q and K from shared memory
+//                      (128B swizzle), fp32 accumulator in TMEM
 //   P_X = 2^(S_X*c-m)  the tile's softmax warpgroup reads S_X from TMEM
-//                      (thread = row = TMEM lane) and writes bf16 P_X back
-//                      over the first 64 columns of S_X
+//                      (thread = row = TMEM lane) into registers and writes
+//                      bf16 P_X to its own TMEM columns
 //   O_X += P_X V       tcgen05.mma with A = P_X from TMEM, B = V (MN-major)
 //                      from shared memory, O_X in TMEM.
-// The tensor core alternates S_A, S_B, PV_A, PV_B, so each softmax
-// warpgroup works while the other tile's products run. The running max moves
-// (and O, l are rescaled) only when it grows by more than 8 in log2 units.
-// A quarter of the exponentials are evaluated on the FMA pipe (range
-// reduction 2^x = 2^n 2^f, |f| <= 1/2, and a minimax cubic for 2^f) to take
-// load off the MUFU unit.
+// One S buffer serves both tiles: S_A(s), S_B(s), S_A(s+1), ... each issued
+// as soon as the previous S has been read into the registers of its
+// softmax warpgroup. Because P has columns of its own, the next S never
+// waits for a P.V product, and both tiles' softmaxes run concurrently while
+// the tensor core works through S_A(s+1), PV_A(s), S_B(s+1), PV_B(s).
+// The running max moves (and O, l are rescaled) only when it grows by more
+// than 8 in log2 units. A quarter of the exponentials are evaluated on the
+// FMA pipe (range reduction 2^x = 2^n 2^f, |f| <= 1/2, and a minimax cubic
+// for 2^f) to take load off the MUFU unit.
 //
-// TMEM (512 columns): S_A 0..127, S_B 128..255, O_A 256..383, O_B 384..511.
+// TMEM (512 columns): S 0..127, P_A 128..191, P_B 192..255 (bf16 pairs),
+// O_A 256..383, O_B 384..511.
 // Warp roles (384 threads, one CTA per SM, persistent over the unit list):
 //   warps 0-3  softmax + epilogue of tile A     warps 4-7  same for tile B
 //   warp 8     TMA producer for K/V (3-D tensor maps, 128B swizzle)
@@ -53,6 +57,11 @@ constexpr int kAttnSmemBytes = (2 + 2 * kStages) * kTileBytes + 1024 + 512;
 constexpr uint32_t kNoHead = 0xFFFFu;
 constexpr uint32_t kNextTile = 0xFFFEu;  // own tile B: the next 128 tokens of tile A's head
 
+// TMEM columns
+constexpr uint32_t kTmemS = 0;
+constexpr uint32_t kTmemP = 128;  // + 64 * X
+constexpr uint32_t kTmemO = 256;  // + 128 * X
+
 struct AttnParams {
   const __nv_bfloat16* q;   // [S - q0][Hq][128]: the tokens with a query
   const int32_t* list;      // group-rows of the window, per bucket
@@ -63,6 +72,7 @@ struct AttnParams {
   __half* own_o;            // [wlen][Hq][128], fp16
   float* own_lse;           // [wlen][Hq]
   int64_t S, w0, q0;        // q0: first token with a query
+  int64_t wlen;             // tokens of the window
   int Hq, G, B;
   float scale_log2;         // log2(e) / sqrt(128)
 };
@@ -75,7 +85,7 @@ struct AttnShared {
   int ring[kRing];
   uint64_t q_full[2], q_empty[2];
   uint64_t k_full[kStages], k_empty[kStages], v_full[kStages], v_empty[kStages];
-  uint64_t s_full[2], p_full[2], pv_done[2], o_free[2];
+  uint64_t s_full[2], s_free, p_full[2], pv_done[2];
   uint64_t drain;
   uint32_t tmem_base;
   int abort_flag;
@@ -150,17 +160,16 @@ constexpr float kExp2C2 = 0.2426111251115799f;
 constexpr float kExp2C3 = 0.0551716685295105f;
 
 // P = 2^(s*c - m) for one 128-column row of S held as raw fp32 bits in r,
-// on column pairs with packed fp32 arithmetic; each 32-column chunk of P (16
-// TMEM columns of bf16 pairs) is stored to TMEM at tS as soon as it is
-// ready. Row sums accumulate into sum2 (four packed pairs). With kPoly, one
-// pair in four is evaluated on the FMA pipe (minimax cubic above) instead of
-// MUFU; columns masked to -inf must use the MUFU path (kPoly false).
+// on column pairs with packed fp32 arithmetic, into 64 registers of bf16
+// pairs (pk[i] = columns 2i, 2i+1). Row sums accumulate into sum2 (four
+// packed pairs). With kPoly, one pair in four is evaluated on the FMA pipe
+// (minimax cubic above) instead of MUFU; columns masked to -inf must use the
+// MUFU path (kPoly false).
 template <bool kPoly>
 __device__ __forceinline__ void exp_row(const uint32_t (&r)[128], uint64_t c2, uint64_t nm2, uint64_t (&sum2)[4],
-                                        uint32_t tS) {
+                                        uint32_t (&pk)[64]) {
 #pragma unroll
   for (int ch = 0; ch < 4; ++ch) {
-    uint32_t pk[16];
 #pragma unroll
     for (int e = ch * 32; e < ch * 32 + 32; e += 2) {
       const uint64_t x2 = f2_fma((uint64_t)r[e] | ((uint64_t)r[e + 1] << 32), c2, nm2);
@@ -180,9 +189,8 @@ __device__ __forceinline__ void exp_row(const uint32_t (&r)[128], uint64_t c2, u
         b = ex2_approx(f2_hi(x2));
       }
       sum2[(e >> 1) & 3] = f2_add(sum2[(e >> 1) & 3], f2_pack(a, b));
-      pk[(e >> 1) & 15] = pack_bf16x2(a, b);
+      pk[e >> 1] = pack_bf16x2(a, b);
     }
-    tmem_st16(tS + ch * 16, pk);
   }
 }
 
@@ -206,8 +214,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       mbar_init(&sh->s_full[x], 1);
       mbar_init(&sh->p_full[x], 128);
       mbar_init(&sh->pv_done[x], 1);
-      mbar_init(&sh->o_free[x], 128);
     }
+    mbar_init(&sh->s_free, 4);  // one lane of each warp of the consuming warpgroup
     for (int i = 0; i < kStages; ++i) {
       mbar_init(&sh->k_full[i], 1);
       mbar_init(&sh->k_empty[i], 1);
@@ -261,8 +269,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     const int X = warp >> 2;
     const int row = threadIdx.x & 127;  // TMEM lane
     const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
-    const uint32_t tS = tmem + X * 128 + lane_off;
-    const uint32_t tO = tmem + 256 + X * 128 + lane_off;
+    const uint32_t tS = tmem + kTmemS + lane_off;
+    const uint32_t tP = tmem + kTmemP + X * 64 + lane_off;
+    const uint32_t tO = tmem + kTmemO + X * 128 + lane_off;
     uint32_t sx = 0;  // steps done by tile X
     for (uint32_t un = 0;; ++un) {
       int ui;
@@ -289,6 +298,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           tmem_ld32(tS + 96, r3);
           tmem_ld_wait();
         }
+        // the S buffer is free for the next tile's product
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sh->s_free);
         // causal mask in an own unit from the step whose keys start at the
         // tile's first token: key > query (a later step is fully masked)
         const bool diag = s >= dstep;
@@ -319,25 +332,32 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           factor = ex2_approx(m_run - m_new);
           rescale = true;
         }
-        // p = 2^(s*c - m), stored into TMEM over the first 64 columns of S_X
+        // p = 2^(s*c - m), held in registers as bf16 pairs
+        uint32_t pk[64];
         {
           const uint64_t c2 = f2_pack(p.scale_log2, p.scale_log2);
           const uint64_t nm2 = f2_pack(-m_ref, -m_ref);
           uint64_t sum2[4] = {0ull, 0ull, 0ull, 0ull};
           if (diag) {
-            exp_row<false>(r, c2, nm2, sum2, tS);
+            exp_row<false>(r, c2, nm2, sum2, pk);
           } else {
-            exp_row<true>(r, c2, nm2, sum2, tS);
+            exp_row<true>(r, c2, nm2, sum2, pk);
           }
           const uint64_t s01 = f2_add(f2_add(sum2[0], sum2[1]), f2_add(sum2[2], sum2[3]));
           l_run = l_run * factor + (f2_lo(s01) + f2_hi(s01));
           m_run = m_ref;
         }
-        // O rescale: S_X(s) was issued after PV_X(s-1) completed, so O_X is
-        // settled here, and PV_X(s) waits for p_full below. The decision is
-        // per row, but tcgen05.ld/st are warp-collective: the whole warp
-        // takes the branch when any of its rows moves its reference (the
-        // others multiply by factor 1).
+        // PV_X(s-1) has completed: P_X's columns are free again and O_X is
+        // settled for a rescale. (This wait also keeps every thread's arrival
+        // on p_full for step s behind the completion of step s-1.)
+        if (s > 0) {
+          if (!mbar_wait(&sh->pv_done[X], (sx - 1) & 1, abort_flag)) goto done;
+          __syncwarp();
+          tc_fence_after();
+        }
+        // O rescale. The decision is per row, but tcgen05.ld/st are
+        // warp-collective: the whole warp takes the branch when any of its
+        // rows moves its reference (the others multiply by factor 1).
         if (__any_sync(0xffffffffu, rescale)) {
 #pragma unroll
           for (int c = 0; c < 4; ++c) {
@@ -349,12 +369,15 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             tmem_st32(tO + c * 32, o);
           }
         }
+#pragma unroll
+        for (int ch = 0; ch < 4; ++ch) tmem_st16(tP + ch * 16, pk + ch * 16);
         tmem_st_wait();
         tc_fence_before();
         mbar_arrive(&sh->p_full[X]);
       }
       {
-        // epilogue: O / l and lse for this tile's rows
+        // epilogue: O / l and lse for this tile's rows (the next unit's
+        // first P.V product waits for this tile's p_full, which comes after)
         if (!mbar_wait(&sh->pv_done[X], (sx - 1) & 1, abort_flag)) goto done;
         __syncwarp();
         tc_fence_after();
@@ -391,7 +414,6 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         }
         if (write) *dst_lse = lse;
         tc_fence_before();
-        mbar_arrive(&sh->o_free[X]);
       }
     }
   } else if (warp == 8) {
@@ -429,16 +451,13 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     }
   } else if (warp == 9) {
     // ------------------------------------------------ MMA issuer
-    // Per step s the tensor core runs, for each tile X in turn,
-    //   PV_X(s), then S_X(s+1) as two N = 64 halves: columns 64..127 first
-    //   (they do not hold P_X(s)), then, once PV_X(s) has completed,
-    //   columns 0..63.
-    // So tile A's softmax of step s+1 overlaps PV_B(s) and S_B(s+1), and
-    // tile B's overlaps PV_A(s+1) and S_A(s+2). The whole warp runs the loop
-    // (descriptors stay warp-uniform); lane 0 issues every MMA and commit.
-    // lane 0 (the lane elect.sync picks in a converged warp) issues every
-    // MMA and commit
-    const uint32_t idesc_s = idesc_bf16_f32(128, 64, false);
+    // Per unit: S_A(0), S_B(0); then per step s
+    //   S_A(s+1), PV_A(s), S_B(s+1), PV_B(s)
+    // Each S waits until the softmax warpgroup of the previous S has read it
+    // (s_free); each PV waits for its tile's P (p_full). The whole warp runs
+    // the loop (descriptors stay warp-uniform); one elected lane issues every
+    // MMA and commit.
+    const uint32_t idesc_s = idesc_bf16_f32(128, 128, false);
     const uint32_t idesc_o = idesc_bf16_f32(128, 128, true);
     // Descriptors are built once; moving the start address by b bytes adds
     // b >> 4 to the descriptor (the 14-bit start field cannot carry inside
@@ -447,25 +466,50 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     const uint64_t dK = sdesc_sw128(smem_u32(sK), 16, 1024);
     const uint64_t dV = sdesc_sw128(smem_u32(sV), kHalfBytes, 1024);
     uint32_t it = 0;          // K/V steps
-    uint32_t sx[2] = {0, 0};  // steps per tile
+    uint32_t ns = 0;          // products issued into the S buffer
+    uint32_t npv[2] = {0, 0};  // P.V products per tile
     uint32_t ux[2] = {0, 0};  // units per tile
-    // S_X = Q_X K^T for keys [64*half, 64*half + 64) of K stage st
-    auto issue_s_half = [&](int x, int half, int st) {
+    auto commit = [&](uint64_t* bar) {
+      if (elect_one()) mma_commit(bar);
+      __syncwarp();
+    };
+    // S_X = Q_X K^T for the 128 keys of K stage st, once the S buffer's
+    // previous product has been read; closes tile X's Q buffer when this is
+    // the unit's last product of that tile
+    auto issue_s = [&](int x, int st, bool last_of_unit) -> bool {
+      if (ns > 0 && !mbar_wait(&sh->s_free, (ns - 1) & 1, abort_flag)) return false;
+      tc_fence_after();
       const uint64_t q0 = dQ + ((x * kTileBytes) >> 4);
-      const uint64_t k0 = dK + ((st * kTileBytes + half * 64 * 128) >> 4);
-      const uint32_t d = tmem + x * 128 + half * 64;
+      const uint64_t k0 = dK + ((st * kTileBytes) >> 4);
       if (elect_one()) {
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
           const uint32_t off = ((kk >> 2) * kHalfBytes + (kk & 3) * 32) >> 4;
-          mma_bf16_ss(d, q0 + off, k0 + off, idesc_s, kk > 0);
+          mma_bf16_ss(tmem + kTmemS, q0 + off, k0 + off, idesc_s, kk > 0);
         }
+        mma_commit(&sh->s_full[x]);
+        if (last_of_unit) mma_commit(&sh->q_empty[x]);
       }
       __syncwarp();
+      ++ns;
+      return true;
     };
-    auto commit = [&](uint64_t* bar) {
-      if (elect_one()) mma_commit(bar);
+    // O_X (+)= P_X V for V stage st
+    auto issue_pv = [&](int x, int st, bool accumulate) -> bool {
+      if (!mbar_wait(&sh->p_full[x], npv[x] & 1, abort_flag)) return false;
+      tc_fence_after();
+      const uint64_t v0 = dV + ((st * kTileBytes) >> 4);
+      const uint32_t tPx = tmem + kTmemP + x * 64;
+      const uint32_t tOx = tmem + kTmemO + x * 128;
+      if (elect_one()) {
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          mma_bf16_ts(tOx, tPx + kk * 8, v0 + ((kk * 2048) >> 4), idesc_o, (accumulate || kk > 0) ? 1u : 0u);
+        mma_commit(&sh->pv_done[x]);
+      }
       __syncwarp();
+      ++npv[x];
+      return true;
     };
     for (uint32_t un = 0;; ++un) {
       int ui;
@@ -473,63 +517,35 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       if (ui < 0) break;
       const UnitInfo u = decode_unit(p, ui);
       const int nx = u.has_b ? 2 : 1;
-#pragma unroll
-      for (int x = 0; x < 2; ++x)
-        if (x < nx && !mbar_wait(&sh->q_full[x], ux[x] & 1, abort_flag)) goto mma_done;
+      const int n = u.nsteps;
       {
-        // prologue: S_X(0)
+        // prologue: S_A(0), S_B(0)
         const int st0 = it % kStages;
         if (!mbar_wait(&sh->k_full[st0], (it / kStages) & 1, abort_flag)) goto mma_done;
-        tc_fence_after();
-#pragma unroll
-        for (int x = 0; x < 2; ++x) {
-          if (x >= nx) break;
-          issue_s_half(x, 1, st0);
-          // columns 0..63 held P_X of this tile's previous step
-          if (sx[x] > 0 && !mbar_wait(&sh->pv_done[x], (sx[x] - 1) & 1, abort_flag)) goto mma_done;
-          tc_fence_after();
-          issue_s_half(x, 0, st0);
-          commit(&sh->s_full[x]);
-          if (u.nsteps == 1) commit(&sh->q_empty[x]);
+        for (int x = 0; x < nx; ++x) {
+          if (!mbar_wait(&sh->q_full[x], ux[x] & 1, abort_flag)) goto mma_done;
+          if (!issue_s(x, st0, n == 1)) goto mma_done;
         }
         commit(&sh->k_empty[st0]);
       }
-      for (int s = 0; s < u.nsteps; ++s) {
+      for (int s = 0; s < n; ++s) {
         const uint32_t cur = it + s;
         const int st = cur % kStages, nst = (cur + 1) % kStages;
-        const bool has_next = s + 1 < u.nsteps;
-        if (!mbar_wait(&sh->v_full[st], (cur / kStages) & 1, abort_flag)) goto mma_done;
-        if (has_next && !mbar_wait(&sh->k_full[nst], ((cur + 1) / kStages) & 1, abort_flag)) goto mma_done;
-        const uint64_t v0 = dV + ((st * kTileBytes) >> 4);
-#pragma unroll
-        for (int x = 0; x < 2; ++x) {
-          if (x >= nx) break;
-          if (!mbar_wait(&sh->p_full[x], sx[x] & 1, abort_flag)) goto mma_done;
-          if (s == 0 && ux[x] > 0 && !mbar_wait(&sh->o_free[x], (ux[x] - 1) & 1, abort_flag)) goto mma_done;
-          tc_fence_after();
-          const uint32_t tP = tmem + x * 128;
-          const uint32_t tOx = tmem + 256 + x * 128;
-          if (elect_one()) {
-#pragma unroll
-            for (int kk = 0; kk < 8; ++kk)
-              mma_bf16_ts(tOx, tP + kk * 8, v0 + ((kk * 2048) >> 4), idesc_o, (s > 0 || kk > 0) ? 1u : 0u);
-          }
-          __syncwarp();
-          commit(&sh->pv_done[x]);
-          if (has_next) {
-            issue_s_half(x, 1, nst);
-            if (!mbar_wait(&sh->pv_done[x], sx[x] & 1, abort_flag)) goto mma_done;
-            tc_fence_after();
-            issue_s_half(x, 0, nst);
-            commit(&sh->s_full[x]);
-            if (s + 1 == u.nsteps - 1) commit(&sh->q_empty[x]);
-          }
-          ++sx[x];
+        const bool has_next = s + 1 < n;
+        if (has_next) {
+          if (!mbar_wait(&sh->k_full[nst], ((cur + 1) / kStages) & 1, abort_flag)) goto mma_done;
+          if (!issue_s(0, nst, s + 2 == n)) goto mma_done;
         }
+        if (!mbar_wait(&sh->v_full[st], (cur / kStages) & 1, abort_flag)) goto mma_done;
+        if (!issue_pv(0, st, s > 0)) goto mma_done;
+        if (has_next) {
+          if (nx > 1 && !issue_s(1, nst, s + 2 == n)) goto mma_done;
+          commit(&sh->k_empty[nst]);
+        }
+        if (nx > 1 && !issue_pv(1, st, s > 0)) goto mma_done;
         commit(&sh->v_empty[st]);
-        if (has_next) commit(&sh->k_empty[nst]);
       }
-      it += u.nsteps;
+      it += n;
       ux[0] += 1;
       ux[1] += (nx > 1) ? 1 : 0;
     }
@@ -547,6 +563,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     const int gt = threadIdx.x - 320;  // 0..63
     uint32_t ux[2] = {0, 0};
     const int n_units = p.hdr[1];
+    const int64_t group_rows = p.wlen * p.G;  // group-rows of the window
     for (uint32_t un = 0;; ++un) {
       if (gt == 0) {
         // publish the next unit index (slot reuse waits for every reader)
@@ -581,6 +598,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
               h = u.h[x];
             } else {
               const int rr = __ldg(p.list + u.list0[x] + r);
+              if (rr < 0 || rr >= group_rows) {
+                // an inconsistent router list: record it, gather nothing
+                record_status(MOBA_ERR_DEVICE_CHECK);
+                continue;
+              }
               t = p.w0 + rr / p.G;
               h = u.g * p.G + rr % p.G;
             }

@@ -172,8 +172,9 @@ int check_shape(int64_t S, int Hq, int Hkv, int d, int B, int topk) {
   if (S > (int64_t)INT32_MAX - 2 * B) return fail(MOBA_ERR_UNSUPPORTED, "seqlen too large");
   const int64_t nb = (S + B - 1) / B;
   const int64_t k_eff = std::min<int64_t>(topk, nb);
-  if (k_eff < nb && k_eff > MOBA_MAX_TOPK)
-    return fail(MOBA_ERR_UNSUPPORTED, "topk %d above %d with fewer than all blocks is not supported", topk, MOBA_MAX_TOPK);
+  if (k_eff < nb && k_eff - 1 > MOBA_MAX_TOPK)
+    return fail(MOBA_ERR_UNSUPPORTED, "topk %d above %d + 1 with fewer than all blocks is not supported", topk,
+                MOBA_MAX_TOPK);
   if ((int64_t)Hq * S * k_eff > ((int64_t)1 << 40)) return fail(MOBA_ERR_UNSUPPORTED, "selection table too large");
   return MOBA_OK;
 }
@@ -579,6 +580,7 @@ int run_forward(const Plan& p, const DeviceInfo& dev, const void* q, const void*
     tm->count(launch_route(p, wg, routed, ws, st));
     tm->mark(kRoute);
     ap.w0 = w0;
+    ap.wlen = wg.wlen;
     launch_chained(moba::attn_kernel, dim3(dev.sms), dim3(moba::kAttnThreads), moba::kAttnSmemBytes, st, tmk, tmv, ap);
     tm->count(1);
     tm->mark(kAttn);
@@ -712,6 +714,7 @@ int run_backward(const Plan& p, const BwdLayout& bl, const DeviceInfo& dev, cons
     tm->count(launch_route(p, wg, routed, ws, st));
     tm->mark(kRoute);
     ap.w0 = w0;
+    ap.wlen = wg.wlen;
     bp.w0 = w0;
     bp.wlen = wg.wlen;
     launch_chained(moba::bwd_dq_kernel, dim3(dev.sms), dim3(moba::kDqThreads), moba::kDqSmemBytes, st, tmk, tmv,

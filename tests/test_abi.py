@@ -51,6 +51,7 @@ FAKE = 0x1000  # 16-byte aligned, never dereferenced: checks fail first
     ((FAKE, FAKE, FAKE, 4096, 0, 1, 128, 512, 3, FAKE, FAKE), moba.MOBA_ERR_INVALID_ARG),
     ((FAKE + 8, FAKE, FAKE, 4096, 1, 1, 128, 512, 3, FAKE, FAKE), moba.MOBA_ERR_INVALID_ARG),
     ((FAKE, FAKE, FAKE, 1 << 20, 1, 1, 128, 128, 100, FAKE, FAKE), moba.MOBA_ERR_UNSUPPORTED),
+    ((FAKE, FAKE, FAKE, 1 << 20, 1, 1, 128, 128, 66, FAKE, FAKE), moba.MOBA_ERR_UNSUPPORTED),  # 65 past blocks
 ])
 def test_invalid_arguments_are_rejected_before_launch(lib, args, code):
     rc = lib.moba_fwd(*args, None)
