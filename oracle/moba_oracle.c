@@ -27,6 +27,12 @@
  *     0/1 mask row over all keys, then softmax of the masked, scaled logits,
  *     scale 1/sqrt(d), and the natural-log log-sum-exp of those logits.
  *
+ * Speed without changing a result: every row is computed on its own, its
+ * sums in the order written; four independent inner products may be formed
+ * side by side (separate accumulators), bf16 rows are widened to fp64 into a
+ * small buffer before use, and threads take interleaved rows. None of this
+ * changes any rounding (the results are bit-identical to one key at a time).
+ *
  * Parity unpinned: the choice of q . mean(K_block) as the gate score, the
  * softmax scale 1/sqrt(d) and the LSE convention are not stated on the pages;
  * the tests pin the arithmetic of each step, not these choices.
@@ -49,6 +55,11 @@ static double bf16_to_f64(uint16_t x) {
 
 static int64_t nblocks_of(int64_t S, int B) { return (S + B - 1) / B; }
 
+/* One bf16 row of d values widened (exactly) to fp64. */
+static void row_to_f64(const uint16_t* x, int d, double* out) {
+    for (int c = 0; c < d; ++c) out[c] = bf16_to_f64(x[c]);
+}
+
 /* Step 1: block partition and key mean-pool.
  * m[g][j][c] = (1/|blk j|) * sum over t in block j of K[t][g][c], summed in
  * ascending t. The last block may be partial: the mean is over the keys it
@@ -70,15 +81,35 @@ void oracle_kmean(const uint16_t* k, int64_t S, int Hkv, int d, int B,
 }
 
 /* Step 2: gate scores of query row (t, h) against every past block.
- * s[j] = sum_c Q[t][h][c] * m[g(h)][j][c] for j < t / B (unscaled). */
+ * s[j] = sum_c Q[t][h][c] * m[g(h)][j][c] for j < t / B (unscaled), each
+ * sum taken over c in ascending order. Four blocks' sums are formed side by
+ * side (four separate accumulators, the same order of additions in each), so
+ * the results are those of one block at a time. */
 void oracle_gate_scores(const uint16_t* q, const double* m, int64_t S, int Hq,
                         int Hkv, int d, int B, int64_t t, int h, double* s) {
     int64_t nb = nblocks_of(S, B);
     int g = h / (Hq / Hkv);
     int64_t b = t / B;
     const uint16_t* qr = q + (t * Hq + h) * d;
-    for (int64_t j = 0; j < b; ++j) {
-        const double* mj = m + ((int64_t)g * nb + j) * d;
+    const double* mg = m + (int64_t)g * nb * d;
+    int64_t j = 0;
+    for (; j + 4 <= b; j += 4) {
+        const double *m0 = mg + j * d, *m1 = m0 + d, *m2 = m1 + d, *m3 = m2 + d;
+        double a0 = 0.0, a1 = 0.0, a2 = 0.0, a3 = 0.0;
+        for (int c = 0; c < d; ++c) {
+            double qc = bf16_to_f64(qr[c]);
+            a0 += qc * m0[c];
+            a1 += qc * m1[c];
+            a2 += qc * m2[c];
+            a3 += qc * m3[c];
+        }
+        s[j] = a0;
+        s[j + 1] = a1;
+        s[j + 2] = a2;
+        s[j + 3] = a3;
+    }
+    for (; j < b; ++j) {
+        const double* mj = mg + j * d;
         double acc = 0.0;
         for (int c = 0; c < d; ++c) acc += bf16_to_f64(qr[c]) * mj[c];
         s[j] = acc;
@@ -157,7 +188,7 @@ static void attend_row(const uint16_t* q, const uint16_t* k,
                        int B, int64_t t, int h, const int32_t* sel,
                        int64_t k_eff, double* out, double* lse,
                        unsigned char* blk_in, double* z, int64_t* zu,
-                       double* qd) {
+                       double* qd, double* kd) {
     int64_t nb = nblocks_of(S, B);
     int g = h / (Hq / Hkv);
     const double scale = 1.0 / sqrt((double)d);
@@ -165,26 +196,56 @@ static void attend_row(const uint16_t* q, const uint16_t* k,
     for (int64_t i = 0; i < k_eff; ++i)
         if (sel[i] >= 0) blk_in[sel[i]] = 1;
     for (int c = 0; c < d; ++c) qd[c] = bf16_to_f64(q[(t * Hq + h) * d + c]);
+    /* the mask row: the keys u in [0, S) with M[u] = 1, ascending (bu and
+     * ru walk u / B and u % B) */
     int64_t n = 0;
-    double mx = -INFINITY;
-    for (int64_t u = 0; u < S; ++u) {
-        int on = blk_in[u / B] && (u <= t);
-        if (!on) continue;
-        const uint16_t* ku = k + (u * Hkv + g) * d;
-        double acc = 0.0;
-        for (int c = 0; c < d; ++c) acc += qd[c] * bf16_to_f64(ku[c]);
-        z[n] = acc * scale;
-        zu[n] = u;
-        if (z[n] > mx) mx = z[n];
-        ++n;
+    for (int64_t u = 0, bu = 0, ru = 0; u < S; ++u) {
+        int on = blk_in[bu] && (u <= t);
+        if (on) zu[n++] = u;
+        if (++ru == B) {
+            ru = 0;
+            ++bu;
+        }
     }
+    /* logits of those keys, each inner product summed over c in ascending
+     * order; four keys side by side (four separate accumulators, the same
+     * order of additions in each) */
+    int64_t i = 0;
+    for (; i + 4 <= n; i += 4) {
+        double* k0 = kd;
+        double *k1 = k0 + d, *k2 = k1 + d, *k3 = k2 + d;
+        row_to_f64(k + (zu[i] * Hkv + g) * d, d, k0);
+        row_to_f64(k + (zu[i + 1] * Hkv + g) * d, d, k1);
+        row_to_f64(k + (zu[i + 2] * Hkv + g) * d, d, k2);
+        row_to_f64(k + (zu[i + 3] * Hkv + g) * d, d, k3);
+        double a0 = 0.0, a1 = 0.0, a2 = 0.0, a3 = 0.0;
+        for (int c = 0; c < d; ++c) {
+            a0 += qd[c] * k0[c];
+            a1 += qd[c] * k1[c];
+            a2 += qd[c] * k2[c];
+            a3 += qd[c] * k3[c];
+        }
+        z[i] = a0 * scale;
+        z[i + 1] = a1 * scale;
+        z[i + 2] = a2 * scale;
+        z[i + 3] = a3 * scale;
+    }
+    for (; i < n; ++i) {
+        row_to_f64(k + (zu[i] * Hkv + g) * d, d, kd);
+        double acc = 0.0;
+        for (int c = 0; c < d; ++c) acc += qd[c] * kd[c];
+        z[i] = acc * scale;
+    }
+    double mx = -INFINITY;
+    for (i = 0; i < n; ++i)
+        if (z[i] > mx) mx = z[i];
     double l = 0.0;
     for (int c = 0; c < d; ++c) out[c] = 0.0;
-    for (int64_t i = 0; i < n; ++i) {
+    for (i = 0; i < n; ++i) {
         double p = exp(z[i] - mx);
         l += p;
-        const uint16_t* vu = v + (zu[i] * Hkv + g) * d;
-        for (int c = 0; c < d; ++c) out[c] += p * bf16_to_f64(vu[c]);
+        row_to_f64(v + (zu[i] * Hkv + g) * d, d, kd);
+        for (int c = 0; c < d; ++c) out[c] += p * kd[c];
     }
     for (int c = 0; c < d; ++c) out[c] /= l;
     *lse = mx + log(l);
@@ -199,7 +260,7 @@ typedef struct {
     int Hq, Hkv, d, B, topk;
     const int64_t* rows_t;
     const int32_t* rows_h;
-    int64_t r0, r1;
+    int64_t r0, r1, rstep; /* rows r0, r0 + rstep, ... below r1 */
     const int32_t* sel_in; /* [nrows][k_eff] or NULL */
     int32_t* sel_out;      /* [nrows][k_eff] or NULL */
     double* info_out;      /* [nrows][4] or NULL */
@@ -218,9 +279,10 @@ static void* row_worker(void* arg) {
     double* z = (double*)malloc(sizeof(double) * (size_t)kmax);
     int64_t* zu = (int64_t*)malloc(sizeof(int64_t) * (size_t)kmax);
     double* qd = (double*)malloc(sizeof(double) * (size_t)J->d);
+    double* kd = (double*)malloc(sizeof(double) * 4 * (size_t)J->d);
     int32_t* selr = (int32_t*)malloc(sizeof(int32_t) * (size_t)k_eff);
     double info[4];
-    for (int64_t r = J->r0; r < J->r1; ++r) {
+    for (int64_t r = J->r0; r < J->r1; r += J->rstep) {
         int64_t t = J->rows_t[r];
         int h = J->rows_h[r];
         const int32_t* sel;
@@ -236,24 +298,28 @@ static void* row_worker(void* arg) {
         if (J->out)
             attend_row(J->q, J->k, J->v, J->S, J->Hq, J->Hkv, J->d, J->B, t,
                        h, sel, k_eff, J->out + r * J->d, J->lse + r, blk_in,
-                       z, zu, qd);
+                       z, zu, qd, kd);
     }
-    free(work); free(sbuf); free(blk_in); free(z); free(zu); free(qd); free(selr);
+    free(work); free(sbuf); free(blk_in); free(z); free(zu); free(qd); free(kd); free(selr);
     return NULL;
 }
 
+/* Thread i takes rows i, i + nthreads, i + 2 nthreads, ...: rows next to
+ * each other in the caller's order run at the same time, so when they read
+ * the same keys those stay in the shared cache. Every row is computed on its
+ * own; the order only affects speed. */
 static void run_rows(row_job base, int64_t nrows, int nthreads) {
     if (nthreads < 1) nthreads = 1;
     if (nthreads > 1024) nthreads = 1024;
     if (nthreads > nrows) nthreads = (int)(nrows > 0 ? nrows : 1);
     row_job jobs[1024];
     pthread_t th[1024];
-    int64_t per = (nrows + nthreads - 1) / nthreads;
     int started = 0;
     for (int i = 0; i < nthreads; ++i) {
         jobs[i] = base;
-        jobs[i].r0 = (int64_t)i * per;
-        jobs[i].r1 = jobs[i].r0 + per < nrows ? jobs[i].r0 + per : nrows;
+        jobs[i].r0 = i;
+        jobs[i].r1 = nrows;
+        jobs[i].rstep = nthreads;
         if (jobs[i].r0 >= jobs[i].r1) break;
         if (nthreads == 1) { row_worker(&jobs[i]); continue; }
         pthread_create(&th[i], NULL, row_worker, &jobs[i]);

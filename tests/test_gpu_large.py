@@ -59,11 +59,34 @@ def check_all_selections(q, k, sel_g, w, m):
     return near
 
 
+def attend_by_group(qo, ko, vo, w, rows_t, rows_h, sel_rows):
+    """The oracle's rows, one kv group at a time: q heads G*g .. G*g+G-1 with
+    kv head g alone, each as its own contiguous problem. Under the contiguous
+    grouping (q head h reads kv head h // G) these are the same computations
+    as in the whole problem; the oracle just reads each group's keys from a
+    contiguous array instead of every Hkv-th row."""
+    G = w.heads_q // w.heads_kv
+    out = np.empty((rows_t.size, qo.shape[2]), dtype=np.float64)
+    lse = np.empty(rows_t.size, dtype=np.float64)
+    for g in np.unique(rows_h // G):
+        idx = np.nonzero(rows_h // G == g)[0]
+        if w.heads_kv == 1:
+            qg, kg, vg = qo, ko, vo
+        else:
+            qg = np.ascontiguousarray(qo[:, g * G:(g + 1) * G])
+            kg = np.ascontiguousarray(ko[:, g:g + 1])
+            vg = np.ascontiguousarray(vo[:, g:g + 1])
+        o, l, _ = oracle.attend(qg, kg, vg, w.block_size, w.topk, rows_t[idx], (rows_h[idx] - g * G).astype(np.int32),
+                                sel=sel_rows[idx])
+        out[idx], lse[idx] = o, l
+    return out, lse
+
+
 def check_rows(qo, ko, vo, w, out_g, lse_g, sel_g, rows_t, rows_h):
     """Outputs of the given rows against the oracle run on (qo, ko, vo), which
     hold the whole sequence or a prefix of it that contains every row."""
     sel_rows = sel_g[rows_h, rows_t]  # already checked against the oracle's gate
-    out_o, lse_o, _ = oracle.attend(qo, ko, vo, w.block_size, w.topk, rows_t, rows_h, sel=sel_rows)
+    out_o, lse_o = attend_by_group(qo, ko, vo, w, rows_t, rows_h, sel_rows)
     out_rows = out_g[torch.from_numpy(rows_t), torch.from_numpy(rows_h.astype(np.int64))].float().numpy()
     return compare_outputs(out_rows, lse_g[rows_h, rows_t], out_o, lse_o)
 
@@ -92,8 +115,9 @@ def test_1m_every_selection_and_the_64k_prefix():
     w, q, k, v, out_g, lse_g, sel_g, near = run_workload("1m")
     P, G = 65536, w.heads_q // w.heads_kv
     heads = np.array([g * G + g % G for g in range(w.heads_kv)], dtype=np.int32)
-    rows_t = np.repeat(np.arange(P, dtype=np.int64), heads.size)
-    rows_h = np.tile(heads, P)
+    # head-major: consecutive rows of one head share their keys in the host's caches
+    rows_t = np.tile(np.arange(P, dtype=np.int64), heads.size)
+    rows_h = np.repeat(heads, P)
     pre = check_rows(q[:P], k[:P], v[:P], w, out_g, lse_g, sel_g, rows_t, rows_h)
     # beyond the prefix: drawn rows over the whole sequence and the last tokens
     dt, dh = drawn_rows(w, 2048, w.seed + 1000)
