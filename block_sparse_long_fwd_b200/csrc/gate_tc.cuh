@@ -106,6 +106,22 @@ __device__ __forceinline__ void gate_write_row(int32_t* out, const int (&ti)[KP]
 
 // grid (ceil((S - q0)*G / 128), Hkv), 128 threads; row = TMEM lane = group-row
 // blockIdx.x*128 + threadIdx.x.
+//
+// The CTA's past blocks are scored in super-chunks of up to four 64-block
+// chunks (256 TMEM columns): warp 0 streams each chunk's hi/lo means through
+// a two-stage TMA ring and issues its products into the chunk's 64 columns.
+// Once a super-chunk is scored, every row selects from it in two passes over
+// its TMEM columns:
+//   1. tau = the smallest of KP group maxima, the groups being KP disjoint
+//      sets of the row's columns (column i in group i mod KP). KP columns
+//      reach tau, so a column strictly below it cannot be among the row's
+//      best KP (an equal one still can: ties go to the lower block);
+//   2. the columns with score >= tau that also beat the row's current KP-th
+//      best (strictly: the list's blocks are lower) are inserted in
+//      ascending block order into the row's sorted list.
+// With KP disjoint groups over ~255 scores, about 14 columns survive the
+// filter per row instead of the ~48 insertions of a plain scan. Lists of 32
+// or more entries (few rows, many columns each) skip the filter.
 template <int KP>
 __global__ void __launch_bounds__(kGateTcThreads)
     gate_tc_kernel(const __grid_constant__ CUtensorMap tm_hi, const __grid_constant__ CUtensorMap tm_lo,
@@ -114,8 +130,8 @@ __global__ void __launch_bounds__(kGateTcThreads)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sQ = smem;
-  uint8_t* sM = smem + kGateQBytes;  // 2 stages x (hi, lo)
-  __shared__ uint64_t full_bar[2], mma_bar[2], drain_bar;
+  uint8_t* sM = smem + kGateQBytes;  // 2 stages x (hi, lo); stage 0 doubles as the score staging area
+  __shared__ uint64_t full_bar[2], mma_bar[2], sc_bar, drain_bar;
   __shared__ uint32_t tmem_base;
   __shared__ int abort_flag;
 
@@ -143,17 +159,19 @@ __global__ void __launch_bounds__(kGateTcThreads)
   }
 
   if (nchunks > 0) {
+    const uint32_t ncols = nchunks >= 3 ? 256u : (nchunks == 2 ? 128u : 64u);
     if (threadIdx.x == 0) {
       for (int i = 0; i < 2; ++i) {
         mbar_init(&full_bar[i], 1);
         mbar_init(&mma_bar[i], 1);
       }
+      mbar_init(&sc_bar, 1);
       mbar_init(&drain_bar, 1);
       abort_flag = 0;
       fence_barrier_init();
     }
     if (warp == 0) {
-      tmem_alloc(&tmem_base, 128);
+      tmem_alloc(&tmem_base, ncols);
       tmem_relinquish();
     }
     // gather the 128 Q rows (16-byte copies into the 128B-swizzled layout)
@@ -181,11 +199,14 @@ __global__ void __launch_bounds__(kGateTcThreads)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = tmem_base;
+    const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
     const uint32_t idesc = idesc_bf16_f32(128, kGateBlkChunk, false);
     const uint64_t dQ = sdesc_sw128(smem_u32(sQ), 16, 1024);
     const uint64_t dM = sdesc_sw128(smem_u32(sM), 16, 1024);
     const int row0 = g * p.nbp_pad;  // first mean row of this kv head
-    auto load_chunk = [&](int c) {   // thread 0 only
+    volatile int* ab = &abort_flag;
+    int loaded = 0;  // chunks warp 0 has asked TMA for
+    auto load_chunk = [&](int c) {  // one lane of warp 0
       const int st = c & 1;
       uint8_t* dst = sM + st * 2 * kGateSplitBytes;
       mbar_arrive_expect_tx(&full_bar[st], 2 * kGateSplitBytes);
@@ -195,122 +216,127 @@ __global__ void __launch_bounds__(kGateTcThreads)
       tma_load_2d(dst + kGateSplitBytes, &tm_lo, &full_bar[st], 0, r0);
       tma_load_2d(dst + kGateSplitBytes + kGateSplitHalf, &tm_lo, &full_bar[st], 64, r0);
     };
-    volatile int* ab = &abort_flag;
-    // scores of chunk c = Q.hi^T + Q.lo^T into TMEM columns [64*(c&1), +64)
-    auto issue_mma = [&](int c) -> bool {  // warp 0
-      const int st = c & 1;
-      if (!mbar_wait(&full_bar[st], (c >> 1) & 1, ab)) return false;
-      tc_fence_after();
-      if (elect_one()) {
-        const uint64_t m0 = dM + ((st * 2 * kGateSplitBytes) >> 4);
+    // staging of one 32-column piece of scores per row (for the insertions,
+    // which index columns per lane): 128 B per row in ring stage 0, 16-byte
+    // pieces swizzled by row so that 8 consecutive rows hit distinct banks
+    float* stg = reinterpret_cast<float*>(sM) + row * 32;
+    const int nsc = (nchunks + 3) / 4;
+    for (int sc = 0; sc < nsc; ++sc) {
+      const int c_lo = 4 * sc;
+      const int nc = min(4, nchunks - c_lo);
+      if (warp == 0) {
+        // scores of this super-chunk: chunk c_lo + c into TMEM columns 64c
+        if (elect_one()) {
+          load_chunk(c_lo);
+          if (nc > 1) load_chunk(c_lo + 1);
+        }
+        __syncwarp();
+        loaded = c_lo + min(nc, 2);
+        for (int c = 0; c < nc; ++c) {
+          const int gc = c_lo + c, st = gc & 1;
+          if (!mbar_wait(&full_bar[st], (gc >> 1) & 1, ab)) break;
+          tc_fence_after();
+          if (elect_one()) {
+            const uint64_t m0 = dM + ((st * 2 * kGateSplitBytes) >> 4);
 #pragma unroll
-        for (int part = 0; part < 2; ++part) {
+            for (int part = 0; part < 2; ++part) {
 #pragma unroll
-          for (int kk = 0; kk < 8; ++kk) {
-            const uint32_t qoff = ((kk >> 2) * (kGateQBytes / 2) + (kk & 3) * 32) >> 4;
-            const uint32_t moff = (part * kGateSplitBytes + (kk >> 2) * kGateSplitHalf + (kk & 3) * 32) >> 4;
-            mma_bf16_ss(tmem + st * kGateBlkChunk, dQ + qoff, m0 + moff, idesc, (part > 0 || kk > 0) ? 1u : 0u);
+              for (int kk = 0; kk < 8; ++kk) {
+                const uint32_t qoff = ((kk >> 2) * (kGateQBytes / 2) + (kk & 3) * 32) >> 4;
+                const uint32_t moff = (part * kGateSplitBytes + (kk >> 2) * kGateSplitHalf + (kk & 3) * 32) >> 4;
+                mma_bf16_ss(tmem + c * kGateBlkChunk, dQ + qoff, m0 + moff, idesc, (part > 0 || kk > 0) ? 1u : 0u);
+              }
+            }
+            mma_commit(&mma_bar[st]);
+          }
+          __syncwarp();
+          if (c + 2 < nc) {
+            // the stage is free once this chunk's products have read it
+            if (!mbar_wait(&mma_bar[st], (gc >> 1) & 1, ab)) break;
+            if (elect_one()) load_chunk(gc + 2);
+            __syncwarp();
+            loaded = gc + 3;
           }
         }
-        mma_commit(&mma_bar[st]);
+        if (elect_one()) mma_commit(&sc_bar);
+        __syncwarp();
       }
-      __syncwarp();
-      return true;
-    };
-    int loaded = 0;  // chunks thread 0 has asked TMA for
-    if (threadIdx.x == 0) {
-      load_chunk(0);
-      loaded = 1;
-      if (nchunks > 1) {
-        load_chunk(1);
-        loaded = 2;
-      }
-    }
-    bool ok = true;
-    if (warp == 0) ok = issue_mma(0);
-    const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
-    for (int c = 0; c < nchunks; ++c) {
-      if (warp == 0 && ok && c + 1 < nchunks) ok = issue_mma(c + 1);
-      if (ok && !*ab) ok = mbar_wait(&mma_bar[c & 1], (c >> 1) & 1, ab);
+      if (*ab || !mbar_wait(&sc_bar, sc & 1, ab)) break;
       __syncwarp();
       tc_fence_after();
-      // This row's 64 scores of chunk c: TMEM -> registers -> ring stage c & 1
-      // (free: MMA(c) has read it), swizzled so that a warp's 32 rows hit
-      // distinct banks. Candidates are the columns that beat the current
-      // k-th best; each lane then walks only its own candidates, so a warp
-      // pays for the busiest lane instead of for every column some lane needs.
-      const int j0 = c * kGateBlkChunk;
-      const int jn = min(kGateBlkChunk, bt - j0);  // this row's past blocks in the chunk
-      float* stage = reinterpret_cast<float*>(sM + (c & 1) * 2 * kGateSplitBytes) + row * kGateBlkChunk;
-      const float thr = tv[KP - 1];
-      uint64_t cand = 0;
+      // ---- selection over this super-chunk's columns [0, 64 nc)
+      const int jb = sc * 4 * kGateBlkChunk;                 // block of column 0
+      const int jn = max(0, min(nc * kGateBlkChunk, bt - jb));  // this row's past blocks here
+      float tau = -INFINITY;
+      if (KP <= 24) {
+        constexpr int NG = KP <= 24 ? KP : 1;
+        float gm[NG];
 #pragma unroll
-      for (int h32 = 0; h32 < 2; ++h32) {
-        uint32_t sc[32];
-        tmem_ld32(tmem + (c & 1) * kGateBlkChunk + lane_off + h32 * 32, sc);
-        tmem_ld_wait();
+        for (int i = 0; i < NG; ++i) gm[i] = -INFINITY;
 #pragma unroll
-        for (int q4 = 0; q4 < 8; ++q4) {
-          const int k16 = h32 * 8 + q4;  // 16-byte piece of the row
-          *reinterpret_cast<uint4*>(stage + ((k16 ^ (row & 15)) << 2)) =
-              make_uint4(sc[4 * q4], sc[4 * q4 + 1], sc[4 * q4 + 2], sc[4 * q4 + 3]);
+        for (int pc = 0; pc < 8; ++pc) {
+          if (pc < 2 * nc) {
+            uint32_t r[32];
+            tmem_ld32(tmem + pc * 32 + lane_off, r);
+            tmem_ld_wait();
+#pragma unroll
+            for (int e = 0; e < 32; ++e) {
+              const int col = pc * 32 + e;
+              const float v = col < jn ? __uint_as_float(r[e]) : -INFINITY;
+              gm[col % NG] = fmaxf(gm[col % NG], v);
+            }
+          }
         }
+        if (jn >= NG) {
+          tau = gm[0];
 #pragma unroll
-        for (int e = 0; e < 32; ++e) {
-          const int i = h32 * 32 + e;
-          if (i < jn && __uint_as_float(sc[e]) > thr) cand |= 1ull << i;
+          for (int i = 1; i < NG; ++i) tau = fminf(tau, gm[i]);
         }
       }
-      if (KP >= 8 && KP <= 24 && c == 0 && jn > KP) {
-        // First chunk, where every column beats an empty list (short lists
-        // insert cheaply and skip this): split the
-        // row's jn columns into KP strided groups; the smallest group
-        // maximum tau0 is met by KP distinct columns, so a column strictly
-        // below it cannot reach the top KP (a tie with it still can: ties go
-        // to the lower block). Columns below tau0 leave the candidate set.
-        float gm[KP > 24 ? 1 : KP];
 #pragma unroll
-        for (int g = 0; g < (KP > 24 ? 1 : KP); ++g) gm[g] = -INFINITY;
+      for (int pc = 0; pc < 8; ++pc) {
+        if (pc < 2 * nc) {
+          uint32_t r[32];
+          tmem_ld32(tmem + pc * 32 + lane_off, r);
+          tmem_ld_wait();
+          const float thr = tv[KP - 1];
+          uint32_t cand = 0;
 #pragma unroll
-        for (int i = 0; i < kGateBlkChunk; ++i) {
-          const float sv = i < jn ? stage[(((i >> 2) ^ (row & 15)) << 2) | (i & 3)] : -INFINITY;
-          gm[i % (KP > 24 ? 1 : KP)] = fmaxf(gm[i % (KP > 24 ? 1 : KP)], sv);
+          for (int e = 0; e < 32; ++e) {
+            const float v = __uint_as_float(r[e]);
+            if (pc * 32 + e < jn && v >= tau && v > thr) cand |= 1u << e;
+          }
+          if (__any_sync(0xffffffffu, cand != 0u)) {
+#pragma unroll
+            for (int k4 = 0; k4 < 8; ++k4)
+              *reinterpret_cast<uint4*>(stg + ((k4 ^ (row & 7)) << 2)) =
+                  make_uint4(r[4 * k4], r[4 * k4 + 1], r[4 * k4 + 2], r[4 * k4 + 3]);
+            __syncwarp();
+            while (cand) {
+              const int e = __ffs(cand) - 1;
+              cand &= cand - 1;
+              const float sv = stg[(((e >> 2) ^ (row & 7)) << 2) | (e & 3)];
+              if (sv > tv[KP - 1]) gate_insert<KP>(tv, ti, sv, jb + pc * 32 + e);
+            }
+            __syncwarp();
+          }
         }
-        float tau0 = gm[0];
-#pragma unroll
-        for (int g = 1; g < (KP > 24 ? 1 : KP); ++g) tau0 = fminf(tau0, gm[g]);
-        uint64_t keep = 0;
-#pragma unroll
-        for (int i = 0; i < kGateBlkChunk; ++i)
-          if (stage[(((i >> 2) ^ (row & 15)) << 2) | (i & 3)] >= tau0) keep |= 1ull << i;
-        cand &= keep;
       }
-      while (cand) {
-        const int i = __ffsll((long long)cand) - 1;
-        cand &= cand - 1;
-        const float sv = stage[(((i >> 2) ^ (row & 15)) << 2) | (i & 3)];
-        if (sv > tv[KP - 1]) gate_insert<KP>(tv, ti, sv, j0 + i);
-      }
-      // every thread is done with TMEM buffer c & 1 and ring stage c & 1;
-      // order this thread's generic accesses to the stage before the TMA
-      // write that refills it
+      // every thread is done with TMEM and the staging area; order the
+      // staging writes before the TMA writes that refill the stage
       fence_proxy_async_smem();
       tc_fence_before();
       __syncthreads();
       tc_fence_after();
-      if (*ab) break;
-      if (threadIdx.x == 0 && c + 2 < nchunks) {
-        load_chunk(c + 2);
-        loaded = c + 3;
-      }
     }
     if (*ab) {
       // after a timeout: let every issued copy and product land before the
       // shared memory and TMEM go away (bounded waits, flag ignored)
       volatile int keep_waiting = 0;
-      if (threadIdx.x == 0)
-        for (int c = 0; c < loaded; ++c) mbar_wait(&full_bar[c & 1], (c >> 1) & 1, &keep_waiting, (1ull << 28));
       if (warp == 0) {
+        if (elect_one())
+          for (int c = 0; c < loaded; ++c) mbar_wait(&full_bar[c & 1], (c >> 1) & 1, &keep_waiting, (1ull << 28));
+        __syncwarp();
         if (elect_one()) mma_commit(&drain_bar);
         __syncwarp();
         mbar_wait(&drain_bar, 0, &keep_waiting, (1ull << 28));
@@ -320,7 +346,7 @@ __global__ void __launch_bounds__(kGateTcThreads)
     __syncthreads();
     if (warp == 0) {
       tc_fence_after();
-      tmem_dealloc(tmem, 128);
+      tmem_dealloc(tmem, ncols);
     }
   }
   if (!valid) return;

@@ -46,27 +46,61 @@ __device__ __forceinline__ float warp_sum(float v) {
   return v;
 }
 
-// grid ceil(wlen * Hq / 8), 256 threads: one warp per (token, q head) row,
-// lane c owns channels 4c..4c+3. With NP > 0 and at most NP routed partials
-// per row, every partial row is loaded as soon as its slot is known, before
-// the weights (which wait for the partials' lse) are formed: the row then
-// costs three dependent memory round trips (selection, flag words, partials)
-// instead of four. It pays off for a few partials per row (small, latency
-// bound problems); with many, the registers it holds cost more occupancy
-// than it gains (measured: 1M workload merge 35 -> 39 ms with NP = 12), so
-// the host uses it for up to 4. The sums run in the same order either way.
+// Reductions over the 16 lanes of a half-warp (both halves at once).
+__device__ __forceinline__ float half_max(float v) {
+  for (int o = 8; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+
+__device__ __forceinline__ float half_sum(float v) {
+  for (int o = 8; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+// Two fp16 values packed in a 32-bit word, widened to fp32.
+__device__ __forceinline__ float2 half2_bits(uint32_t x) {
+  __half2 h;
+  memcpy(&h, &x, sizeof(h));
+  return __half22float2(h);
+}
+
+// acc += w * (eight fp16 values in o)
+__device__ __forceinline__ void fma_half8(float (&acc)[8], float w, uint4 o) {
+  const uint32_t word[4] = {o.x, o.y, o.z, o.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float2 f = half2_bits(word[i]);
+    acc[2 * i] = fmaf(w, f.x, acc[2 * i]);
+    acc[2 * i + 1] = fmaf(w, f.y, acc[2 * i + 1]);
+  }
+}
+
+// grid ceil(wlen * Hq / 16), 256 threads: one half-warp per (token, q head)
+// row, lane l (of 16) owns channels 8l..8l+7 (16-byte loads and stores).
+// Lane i of the half resolves routed partial i (its list slot from the
+// router's flag words, and its lse); with NP > 0 and at most NP routed
+// partials per row, every partial's O is requested as soon as its slot is
+// known, together with its lse, so a row costs three dependent memory round
+// trips (selection, flag words, partials). Rows with more partials take a
+// three-pass path. The sums run in a fixed order either way: ascending
+// block, own block last.
 template <int NP>
-__global__ void __launch_bounds__(256) merge_kernel(MergeParams m) {
+__global__ void __launch_bounds__(256, 3) merge_kernel(MergeParams m) {
   grid_dependency_sync();
   const WindowGeom& w = m.w;
-  const int lane = threadIdx.x & 31;
-  const int64_t row = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
-  if (row >= w.wlen * w.Hq) return;
+  const int l16 = threadIdx.x & 15;
+  const int hbase = threadIdx.x & 16;  // first lane of this half-warp
+  int64_t row = (int64_t)blockIdx.x * 16 + (threadIdx.x >> 4);
+  const int64_t nrows = w.wlen * w.Hq;
+  // both halves of a warp stay converged for the shuffles; a half past the
+  // end (or a token before q0) runs on a harmless row and writes nothing
+  bool live = row < nrows;
+  if (!live) row = nrows - 1;
   const int64_t tl = row / w.Hq;
   const int h = (int)(row % w.Hq);
   const int64_t t = w.w0 + tl;
-  if (t < w.q0) return;  // no query at this token (padding of a window's first tile)
-  const int64_t tq = t - w.q0, nq = w.S - w.q0;
+  if (t < w.q0) live = false;
+  const int64_t tq = max(t - w.q0, (int64_t)0), nq = w.S - w.q0;
   const int g = h / w.G, hl = h % w.G;
   const int bt = (int)(t / w.B);
   const int64_t rr = tl * w.G + hl;
@@ -75,7 +109,7 @@ __global__ void __launch_bounds__(256) merge_kernel(MergeParams m) {
   const int32_t* srow = m.sel + ((int64_t)h * nq + tq) * w.k_eff;
   const int P = w.k_eff - 1;
 
-  // lane i resolves routed partial i (slot and lse) once
+  // routed partial i: list slot (or -1) and lse (-inf when absent)
   auto slot = [&](int i, float& li) -> int64_t {
     li = -INFINITY;
     if (i >= P) return -1;
@@ -89,105 +123,72 @@ __global__ void __launch_bounds__(256) merge_kernel(MergeParams m) {
   };
 
   const float own_l = m.own_lse[tl * w.Hq + h];
-  const __half* own_row = m.own_o + (tl * w.Hq + h) * kHeadDim + lane * 4;
-  float4 own_v = make_float4(0.f, 0.f, 0.f, 0.f);
-  if (NP > 0) own_v = load_half4(own_row);  // early only where registers are cheap
-  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  const uint4 own_v = __ldg(reinterpret_cast<const uint4*>(m.own_o + (tl * w.Hq + h) * kHeadDim + l16 * 8));
+  float acc[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) acc[i] = 0.f;
   float L;
   if (NP > 0 && P <= NP) {
     float li;
-    const int64_t pos = slot(lane, li);
-    float4 o[NP > 0 ? NP : 1];
+    const int64_t pos = slot(l16, li);
+    uint4 o[NP > 0 ? NP : 1];
 #pragma unroll
     for (int k = 0; k < NP; ++k) {
-      const int64_t pk = __shfl_sync(0xffffffffu, pos, k);
-      o[k] = (k < P && pk >= 0) ? load_half4(m.part_o + pk * kHeadDim + lane * 4) : make_float4(0.f, 0.f, 0.f, 0.f);
+      const int64_t pk = __shfl_sync(0xffffffffu, pos, hbase + k);
+      o[k] = make_uint4(0u, 0u, 0u, 0u);
+      if (k < P && pk >= 0) o[k] = __ldg(reinterpret_cast<const uint4*>(m.part_o + pk * kHeadDim + l16 * 8));
     }
-    const float mx = fmaxf(own_l, warp_max(li));
-    const float sum = warp_sum(li == -INFINITY ? 0.f : expf(li - mx)) + expf(own_l - mx);
+    const float mx = fmaxf(own_l, half_max(li));
+    const float sum = half_sum(li == -INFINITY ? 0.f : expf(li - mx)) + expf(own_l - mx);
     L = mx + logf(sum);
     const float wl = li == -INFINITY ? 0.f : expf(li - L);  // lane i's weight (0 past P)
 #pragma unroll
-    for (int k = 0; k < NP; ++k) {
-      const float wk = __shfl_sync(0xffffffffu, wl, k);
-      acc.x += wk * o[k].x;
-      acc.y += wk * o[k].y;
-      acc.z += wk * o[k].z;
-      acc.w += wk * o[k].w;
-    }
-  } else if (P <= 32) {
-    float li;
-    const int64_t pos = slot(lane, li);
-    const float mx = fmaxf(own_l, warp_max(li));
-    const float sum = warp_sum(li == -INFINITY ? 0.f : expf(li - mx)) + expf(own_l - mx);
-    L = mx + logf(sum);
-    const float wl = li == -INFINITY ? 0.f : expf(li - L);  // lane i's weight
-    // partials in ascending block order, four loads in flight
-    const int n = min(P, 32);
-    for (int k0 = 0; k0 < n; k0 += 4) {
-      float4 o[4];
-      float wk[4];
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int k = k0 + u;
-        const int64_t pk = __shfl_sync(0xffffffffu, pos, k & 31);
-        wk[u] = __shfl_sync(0xffffffffu, wl, k & 31);
-        o[u] = (k < n && pk >= 0) ? load_half4(m.part_o + pk * kHeadDim + lane * 4) : make_float4(0.f, 0.f, 0.f, 0.f);
-        if (!(k < n && pk >= 0)) wk[u] = 0.f;
-      }
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        acc.x += wk[u] * o[u].x;
-        acc.y += wk[u] * o[u].y;
-        acc.z += wk[u] * o[u].z;
-        acc.w += wk[u] * o[u].w;
-      }
-    }
+    for (int k = 0; k < NP; ++k) fma_half8(acc, __shfl_sync(0xffffffffu, wl, hbase + k), o[k]);
   } else {
-    // every past block selected (topk >= number of blocks): chunks of 32
+    // any number of partials: maximum, sum, then the weighted partials, in
+    // groups of 16 (each pass finds its slots again)
     float mx = own_l;
-    for (int i0 = 0; i0 < P; i0 += 32) {
+    for (int i0 = 0; i0 < P; i0 += 16) {
       float li;
-      slot(i0 + lane, li);
-      mx = fmaxf(mx, warp_max(li));
+      slot(i0 + l16, li);
+      mx = fmaxf(mx, half_max(li));
     }
     float sum = 0.f;
-    for (int i0 = 0; i0 < P; i0 += 32) {
+    for (int i0 = 0; i0 < P; i0 += 16) {
       float li;
-      slot(i0 + lane, li);
-      sum += warp_sum(li == -INFINITY ? 0.f : expf(li - mx));
+      slot(i0 + l16, li);
+      sum += half_sum(li == -INFINITY ? 0.f : expf(li - mx));
     }
     sum += expf(own_l - mx);
     L = mx + logf(sum);
-    for (int i0 = 0; i0 < P; i0 += 32) {
+    for (int i0 = 0; i0 < P; i0 += 16) {
       float li;
-      const int64_t pos = slot(i0 + lane, li);
-      const int n = min(32, P - i0);
-      for (int k = 0; k < n; ++k) {
-        const int64_t pk = __shfl_sync(0xffffffffu, pos, k);
-        const float lk = __shfl_sync(0xffffffffu, li, k);
-        if (pk >= 0) {
-          const float wk = expf(lk - L);
-          const float4 o = load_half4(m.part_o + pk * kHeadDim + lane * 4);
-          acc.x += wk * o.x;
-          acc.y += wk * o.y;
-          acc.z += wk * o.z;
-          acc.w += wk * o.w;
+      const int64_t pos = slot(i0 + l16, li);
+      const float wl = li == -INFINITY ? 0.f : expf(li - L);
+      for (int k0 = 0; k0 < 16; k0 += 4) {
+        uint4 o[4];
+        float wk[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int64_t pk = __shfl_sync(0xffffffffu, pos, hbase + k0 + u);
+          wk[u] = __shfl_sync(0xffffffffu, wl, hbase + k0 + u);
+          o[u] = make_uint4(0u, 0u, 0u, 0u);
+          if (pk >= 0) o[u] = __ldg(reinterpret_cast<const uint4*>(m.part_o + pk * kHeadDim + l16 * 8));
         }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) fma_half8(acc, wk[u], o[u]);
       }
     }
   }
-  {
-    if (NP == 0) own_v = load_half4(own_row);
-    const float wk = expf(own_l - L);
-    acc.x += wk * own_v.x;
-    acc.y += wk * own_v.y;
-    acc.z += wk * own_v.z;
-    acc.w += wk * own_v.w;
-  }
-  uint2 packed = make_uint2(pack_bf16x2(acc.x, acc.y), pack_bf16x2(acc.z, acc.w));
-  *reinterpret_cast<uint2*>(m.out + (tq * w.Hq + h) * kHeadDim + lane * 4) = packed;
-  if (lane == 0) m.lse[(int64_t)h * m.lse_ld + tq] = L;
+  fma_half8(acc, expf(own_l - L), own_v);
+  if (!live) return;
+  uint4 packed;
+  packed.x = pack_bf16x2(acc[0], acc[1]);
+  packed.y = pack_bf16x2(acc[2], acc[3]);
+  packed.z = pack_bf16x2(acc[4], acc[5]);
+  packed.w = pack_bf16x2(acc[6], acc[7]);
+  *reinterpret_cast<uint4*>(m.out + (tq * w.Hq + h) * kHeadDim + l16 * 8) = packed;
+  if (l16 == 0) m.lse[(int64_t)h * m.lse_ld + tq] = L;
 }
 
 }  // namespace moba

@@ -298,7 +298,9 @@ void plan_shape(Plan& p, int64_t S, int64_t q0, int Hq, int Hkv, int B, int topk
   dense_blocks(p);
 }
 
-int make_plan(Plan* pl, int64_t S, int64_t q0, int Hq, int Hkv, int B, int topk) {
+// `share` > 1: the problem runs beside share - 1 others, each with its own
+// scratch, so its windows take a 1/share part of the budget.
+int make_plan(Plan* pl, int64_t S, int64_t q0, int Hq, int Hkv, int B, int topk, int share = 1) {
   Plan& p = *pl;
   plan_shape(p, S, q0, Hq, Hkv, B, topk);
   const int64_t S128 = (S - p.wbase + 127) / 128 * 128;  // tokens the windows cover
@@ -307,7 +309,7 @@ int make_plan(Plan* pl, int64_t S, int64_t q0, int Hq, int Hkv, int B, int topk)
     W = atoll(env);
     W = std::max<int64_t>(128, (W + 127) / 128 * 128);
   } else {
-    const size_t budget = window_budget();
+    const size_t budget = std::max<size_t>((size_t)64 << 20, window_budget() / std::max(share, 1));
     const size_t per = window_bytes(p, 128);
     W = std::max<int64_t>(1, (int64_t)(budget / std::max<size_t>(per, 1))) * 128;
     if (W > 1024 && W % 1024) W = W / 1024 * 1024;
@@ -597,9 +599,12 @@ int run_forward(const Plan& p, const DeviceInfo& dev, const void* q, const void*
     mp.lse_ld = p.lse_ld;
     mp.w = wg;
     const int64_t rows = wg.wlen * p.Hq;
-    const dim3 mg((unsigned)((rows + 7) / 8));
+    const dim3 mg((unsigned)((rows + 15) / 16));
     if (p.P <= 2) launch_chained(moba::merge_kernel<2>, mg, dim3(256), 0, st, mp);
     else if (p.P <= 4) launch_chained(moba::merge_kernel<4>, mg, dim3(256), 0, st, mp);
+    else if (p.P <= 8) launch_chained(moba::merge_kernel<8>, mg, dim3(256), 0, st, mp);
+    else if (p.P <= 12) launch_chained(moba::merge_kernel<12>, mg, dim3(256), 0, st, mp);
+    else if (p.P <= 16) launch_chained(moba::merge_kernel<16>, mg, dim3(256), 0, st, mp);
     else launch_chained(moba::merge_kernel<0>, mg, dim3(256), 0, st, mp);
     tm->count(1);
     tm->mark(kMerge);
@@ -933,10 +938,32 @@ int fwd_impl(const void* q, const void* k, const void* v, int64_t seqlen, int64_
   return finish_call(direct_run(p.total, run, stream), stream);
 }
 
+constexpr int kVarlenLanes = 4;
+cudaStream_t g_lane_streams[64][kVarlenLanes] = {};
+
+// The internal streams a packed batch's sequences run on (created once per
+// device).
+int lane_streams(cudaStream_t** out) {
+  int dev = 0;
+  MOBA_CUDA(cudaGetDevice(&dev));
+  if (dev < 0 || dev >= 64) return fail(MOBA_ERR_UNSUPPORTED, "device index %d out of range", dev);
+  std::lock_guard<std::mutex> lk(g_dev_mu);
+  for (int l = 0; l < kVarlenLanes; ++l)
+    if (!g_lane_streams[dev][l]) MOBA_CUDA(cudaStreamCreateWithFlags(&g_lane_streams[dev][l], cudaStreamNonBlocking));
+  *out = g_lane_streams[dev];
+  return MOBA_OK;
+}
+
 // A packed batch of independent sequences: sequence b holds tokens
 // cu[b] .. cu[b+1]-1 of q, k, v and out, and columns cu[b] .. of lse. The
-// sequences run one after another on one scratch buffer (the largest any of
-// them needs), as one graph when the same batch comes back.
+// sequences are dealt, longest first, onto up to four lanes (the least
+// loaded lane takes the next one); each lane has its own part of the scratch
+// and its own stream, forked from and joined back to the caller's stream, so
+// the small kernels of short sequences overlap and one sequence's attention
+// tail is filled by the next one's. Within a lane the sequences run one
+// after another. Replayed as one graph when the same batch comes back.
+// (Under moba_profile_begin the sequences run one after another on the
+// caller's stream, so that the per-stage times stay meaningful.)
 int varlen_impl(const void* q, const void* k, const void* v, const int64_t* cu, int batch, int heads_q, int heads_kv,
                 int head_dim, int block_size, int topk, void* out, float* lse, cudaStream_t stream) {
   g_err.clear();
@@ -952,37 +979,86 @@ int varlen_impl(const void* q, const void* k, const void* v, const int64_t* cu, 
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out))
     return fail(MOBA_ERR_INVALID_ARG, "device buffers must be 16-byte aligned");
   if (reinterpret_cast<uintptr_t>(lse) & 3) return fail(MOBA_ERR_INVALID_ARG, "lse must be 4-byte aligned");
-  std::vector<Plan> plans;
-  std::vector<int64_t> starts;
-  size_t total = 0;
+  std::vector<int> seqs;  // non-empty sequences, longest first
   for (int b = 0; b < batch; ++b) {
     const int64_t L = cu[b + 1] - cu[b];
     if (!L) continue;  // an empty sequence has nothing to compute
     int rc = check_shape(L, heads_q, heads_kv, head_dim, block_size, topk);
     if (rc) return rc;
+    seqs.push_back(b);
+  }
+  std::stable_sort(seqs.begin(), seqs.end(),
+                   [&](int a, int b) { return cu[a + 1] - cu[a] > cu[b + 1] - cu[b]; });
+  const bool serial = g_timer.on;
+  const int nlanes = serial ? 1 : std::min<int>(kVarlenLanes, (int)seqs.size());
+  std::vector<Plan> plans;
+  std::vector<int64_t> starts;
+  std::vector<int> lane_of;
+  std::vector<int64_t> lane_tokens(nlanes, 0);
+  std::vector<size_t> lane_bytes(nlanes, 0);
+  for (int b : seqs) {
+    const int64_t L = cu[b + 1] - cu[b];
     Plan p;
-    rc = make_plan(&p, L, 0, heads_q, heads_kv, block_size, topk);
+    int rc = make_plan(&p, L, 0, heads_q, heads_kv, block_size, topk, nlanes);
     if (rc) return rc;
     p.lse_ld = T;
-    total = std::max(total, p.total);
+    int l = 0;
+    for (int i = 1; i < nlanes; ++i)
+      if (lane_tokens[i] < lane_tokens[l]) l = i;
+    lane_tokens[l] += L;
+    lane_bytes[l] = std::max(lane_bytes[l], p.total);
     plans.push_back(p);
     starts.push_back(cu[b]);
+    lane_of.push_back(l);
+  }
+  std::vector<size_t> lane_off(nlanes, 0);
+  size_t total = 0;
+  for (int l = 0; l < nlanes; ++l) {
+    lane_off[l] = total;
+    total += (lane_bytes[l] + 255) & ~size_t(255);
   }
   DeviceInfo dev;
   int rc = device_info(&dev);
   if (rc) return rc;
   rc = take_pending_status(dev, stream);
   if (rc) return rc;
+  cudaStream_t* lanes = nullptr;
+  if (nlanes > 1) {
+    rc = lane_streams(&lanes);
+    if (rc) return rc;
+  }
   const size_t qrow = (size_t)heads_q * head_dim * 2, kvrow = (size_t)heads_kv * head_dim * 2;
   const Runner run = [&](uint8_t* ws, cudaStream_t st) {
-    for (size_t i = 0; i < plans.size(); ++i) {
+    auto seq = [&](size_t i, cudaStream_t s) {
       const size_t t0 = (size_t)starts[i];
-      const int r = run_forward(plans[i], dev, static_cast<const uint8_t*>(q) + t0 * qrow,
-                                static_cast<const uint8_t*>(k) + t0 * kvrow, static_cast<const uint8_t*>(v) + t0 * kvrow,
-                                static_cast<uint8_t*>(out) + t0 * qrow, lse + t0, ws, st);
-      if (r) return r;
+      return run_forward(plans[i], dev, static_cast<const uint8_t*>(q) + t0 * qrow,
+                         static_cast<const uint8_t*>(k) + t0 * kvrow, static_cast<const uint8_t*>(v) + t0 * kvrow,
+                         static_cast<uint8_t*>(out) + t0 * qrow, lse + t0, ws + lane_off[lane_of[i]], s);
+    };
+    if (nlanes == 1) {
+      for (size_t i = 0; i < plans.size(); ++i) {
+        const int r = seq(i, st);
+        if (r) return r;
+      }
+      return (int)MOBA_OK;
     }
-    return (int)MOBA_OK;
+    // fork the lanes from the caller's stream and join them back
+    cudaEvent_t fork = nullptr, join[kVarlenLanes] = {};
+    MOBA_CUDA(cudaEventCreateWithFlags(&fork, cudaEventDisableTiming));
+    MOBA_CUDA(cudaEventRecord(fork, st));
+    int r = MOBA_OK;
+    for (int l = 0; l < nlanes && !r; ++l) {
+      if (cudaStreamWaitEvent(lanes[l], fork, 0) != cudaSuccess) r = fail(MOBA_ERR_CUDA, "cudaStreamWaitEvent failed");
+      for (size_t i = 0; i < plans.size() && !r; ++i)
+        if (lane_of[i] == l) r = seq(i, lanes[l]);
+      if (!r && (cudaEventCreateWithFlags(&join[l], cudaEventDisableTiming) != cudaSuccess ||
+                 cudaEventRecord(join[l], lanes[l]) != cudaSuccess || cudaStreamWaitEvent(st, join[l], 0) != cudaSuccess))
+        r = fail(MOBA_ERR_CUDA, "joining the lane streams failed");
+    }
+    cudaEventDestroy(fork);
+    for (int l = 0; l < nlanes; ++l)
+      if (join[l]) cudaEventDestroy(join[l]);
+    return r;
   };
   if (!g_timer.on) {
     GraphKey key{0, q, k, v, out, lse, nullptr, T, 0, 0, T, heads_q, heads_kv, block_size, topk,
@@ -1273,7 +1349,7 @@ extern "C" int moba_selftest_device_check(cudaStream_t stream) {
     w.pair_tokens = 0;
     w.q0 = 0;
     w.list_cap = 1;
-    moba::merge_kernel<0><<<S / 8, 256, 0, stream>>>(mp);
+    moba::merge_kernel<0><<<S / 16, 256, 0, stream>>>(mp);
     if (cudaGetLastError() != cudaSuccess) rc = fail(MOBA_ERR_CUDA, "self-test launch failed");
   }
   const int st = moba_device_status(stream);
