@@ -38,8 +38,13 @@
 // Warp roles (384 threads, one CTA per SM, persistent over the unit list):
 //   warps 0-3  softmax + epilogue of tile A     warps 4-7  same for tile B
 //   warp 8     TMA producer for K/V (3-D tensor maps, 128B swizzle)
-//   warp 9     TMEM owner and single-thread MMA issuer
-//   warps 10-11 Q row gather (cp.async, 16 B per copy, swizzled by hand)
+//   warp 9     TMEM owner; issues the S = Q K^T products
+//   warp 10    Q row gather (cp.async, 16 B per copy, swizzled by hand)
+//   warp 11    issues the O += P V products
+// Two issuers keep the tensor core fed: an MMA issue returns at about the
+// rate the tensor core executes, so one issuer's barrier waits and fences
+// between its product groups would leave the pipe idle; with S and P.V
+// issued by different warps, one issuer's MMAs run while the other waits.
 // Every mbarrier wait is bounded; a timeout sets an error status and the
 // whole CTA winds down without trapping.
 #pragma once
@@ -78,7 +83,7 @@ struct AttnParams {
 };
 
 constexpr int kRing = 8;                               // unit indices in flight per CTA
-constexpr uint32_t kRingReaders = 1 + 32 + 256 + 64;   // producer lane, MMA warp, softmax, gather
+constexpr uint32_t kRingReaders = 1 + 32 + 32 + 256 + 32;  // producer lane, two issuer warps, softmax, gather
 
 struct AttnShared {
   uint64_t ring_full[kRing], ring_empty[kRing];
@@ -209,7 +214,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 
   if (threadIdx.x == 0) {
     for (int x = 0; x < 2; ++x) {
-      mbar_init(&sh->q_full[x], 64);
+      mbar_init(&sh->q_full[x], 32);  // the gather warp's lanes
       mbar_init(&sh->q_empty[x], 1);
       mbar_init(&sh->s_full[x], 1);
       mbar_init(&sh->p_full[x], 128);
@@ -226,7 +231,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       mbar_init(&sh->ring_full[i], 1);
       mbar_init(&sh->ring_empty[i], kRingReaders);
     }
-    mbar_init(&sh->drain, 1);
+    mbar_init(&sh->drain, 2);  // one commit from each issuer
     sh->abort_flag = 0;
     fence_barrier_init();
   }
@@ -449,14 +454,15 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         }
       }
     }
-  } else if (warp == 9) {
-    // ------------------------------------------------ MMA issuer
-    // Per unit: S_A(0), S_B(0); then per step s
-    //   S_A(s+1), PV_A(s), S_B(s+1), PV_B(s)
-    // Each S waits until the softmax warpgroup of the previous S has read it
-    // (s_free); each PV waits for its tile's P (p_full). The whole warp runs
-    // the loop (descriptors stay warp-uniform); one elected lane issues every
-    // MMA and commit.
+  } else if (warp == 9 || warp == 11) {
+    // ------------------------------------------------ MMA issuers
+    // warp 9, per unit: S_A(0), S_B(0), S_A(1), S_B(1), ...; each S waits
+    //   until the softmax warpgroup of the previous S has read it (s_free)
+    // warp 11, per unit: PV_A(0), PV_B(0), PV_A(1), ...; each waits for its
+    //   tile's P (p_full)
+    // Each whole warp runs its loop (descriptors stay warp-uniform); one
+    // elected lane issues every MMA and commit.
+    const bool s_issuer = warp == 9;
     const uint32_t idesc_s = idesc_bf16_f32(128, 128, false);
     const uint32_t idesc_o = idesc_bf16_f32(128, 128, true);
     // Descriptors are built once; moving the start address by b bytes adds
@@ -518,39 +524,30 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       const UnitInfo u = decode_unit(p, ui);
       const int nx = u.has_b ? 2 : 1;
       const int n = u.nsteps;
-      {
-        // prologue: S_A(0), S_B(0)
-        const int st0 = it % kStages;
-        if (!mbar_wait(&sh->k_full[st0], (it / kStages) & 1, abort_flag)) goto mma_done;
-        for (int x = 0; x < nx; ++x) {
-          if (!mbar_wait(&sh->q_full[x], ux[x] & 1, abort_flag)) goto mma_done;
-          if (!issue_s(x, st0, n == 1)) goto mma_done;
-        }
-        commit(&sh->k_empty[st0]);
-      }
       for (int s = 0; s < n; ++s) {
         const uint32_t cur = it + s;
-        const int st = cur % kStages, nst = (cur + 1) % kStages;
-        const bool has_next = s + 1 < n;
-        if (has_next) {
-          if (!mbar_wait(&sh->k_full[nst], ((cur + 1) / kStages) & 1, abort_flag)) goto mma_done;
-          if (!issue_s(0, nst, s + 2 == n)) goto mma_done;
+        const int st = cur % kStages;
+        if (s_issuer) {
+          if (!mbar_wait(&sh->k_full[st], (cur / kStages) & 1, abort_flag)) goto mma_done;
+          for (int x = 0; x < nx; ++x) {
+            if (s == 0 && !mbar_wait(&sh->q_full[x], ux[x] & 1, abort_flag)) goto mma_done;
+            if (!issue_s(x, st, s + 1 == n)) goto mma_done;
+          }
+          commit(&sh->k_empty[st]);
+        } else {
+          if (!mbar_wait(&sh->v_full[st], (cur / kStages) & 1, abort_flag)) goto mma_done;
+          for (int x = 0; x < nx; ++x)
+            if (!issue_pv(x, st, s > 0)) goto mma_done;
+          commit(&sh->v_empty[st]);
         }
-        if (!mbar_wait(&sh->v_full[st], (cur / kStages) & 1, abort_flag)) goto mma_done;
-        if (!issue_pv(0, st, s > 0)) goto mma_done;
-        if (has_next) {
-          if (nx > 1 && !issue_s(1, nst, s + 2 == n)) goto mma_done;
-          commit(&sh->k_empty[nst]);
-        }
-        if (nx > 1 && !issue_pv(1, st, s > 0)) goto mma_done;
-        commit(&sh->v_empty[st]);
       }
       it += n;
       ux[0] += 1;
       ux[1] += (nx > 1) ? 1 : 0;
     }
   mma_done:
-    // every issued MMA must finish before TMEM is released
+    // every issued MMA must finish before TMEM is released (each issuer
+    // commits once to the drain barrier; both wait for both)
     __syncwarp();
     if (elect_one()) mma_commit(&sh->drain);
     __syncwarp();
@@ -559,8 +556,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       mbar_wait(&sh->drain, 0, &keep_waiting, (1ull << 28));
     }
   } else {
-    // ------------------------------------------------ Q gather (warps 10, 11)
-    const int gt = threadIdx.x - 320;  // 0..63
+    // ------------------------------------------------ Q gather (warp 10)
+    const int gt = threadIdx.x - 320;  // 0..31
     uint32_t ux[2] = {0, 0};
     const int n_units = p.hdr[1];
     const int64_t group_rows = p.wlen * p.G;  // group-rows of the window
@@ -578,17 +575,18 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       if (ui < 0) break;
       const UnitInfo u = decode_unit(p, ui);
       const int nx = u.has_b ? 2 : 1;
-      // Thread gt copies whole rows gt and gt + 64 of each tile (16 chunks of
-      // 16 B each). Their element offsets in q are found first (a routed
-      // tile reads its row list), before waiting for the tiles' buffers, so
-      // the list reads overlap the previous unit's last step; then both
-      // tiles' copies are in flight together and complete with one wait.
-      int64_t off[2][2];
+      // Thread gt copies whole rows gt, gt + 32, gt + 64, gt + 96 of each
+      // tile (16 chunks of 16 B each). Their element offsets in q are found
+      // first (a routed tile reads its row list), before waiting for the
+      // tiles' buffers, so the list reads overlap the previous unit's last
+      // step; then both tiles' copies are in flight together and complete
+      // with one wait.
+      int64_t off[2][4];
 #pragma unroll
       for (int x = 0; x < 2; ++x) {
 #pragma unroll
-        for (int k = 0; k < 2; ++k) {
-          const int r = gt + 64 * k;
+        for (int k = 0; k < 4; ++k) {
+          const int r = gt + 32 * k;
           off[x][k] = -1;
           if (x < nx && r < u.rows[x]) {
             int64_t t;
@@ -617,8 +615,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         if (!mbar_wait(&sh->q_empty[x], (ux[x] & 1) ^ 1, abort_flag)) goto gather_done;
         const uint32_t dst0 = smem_u32(sQ + x * kTileBytes);
 #pragma unroll
-        for (int k = 0; k < 2; ++k) {
-          const int r = gt + 64 * k;
+        for (int k = 0; k < 4; ++k) {
+          const int r = gt + 32 * k;
           const bool valid = off[x][k] >= 0;
           const __nv_bfloat16* src = valid ? p.q + off[x][k] : p.q;
 #pragma unroll

@@ -37,6 +37,11 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
   return t;
 }
 
+// x / d and x % d for 32-bit operands (d > 0): a 64-bit division costs
+// several times more instructions, and the token and row indices that the
+// kernels divide fit in 32 bits (the host caps seqlen below 2^31).
+__device__ __forceinline__ uint32_t udiv32(uint32_t x, uint32_t d) { return x / d; }
+
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }

@@ -63,6 +63,7 @@ struct GateParams {
   int32_t* sel;            // [Hq][S - q0][k_eff]
   int64_t S, q0;           // q0: first token with a query
   int Hq, G, B, nbp_pad, k_eff;
+  int q_tma;               // 1: G divides 128 and tm_q is valid (Q tiles by TMA)
 };
 
 template <int KP>
@@ -125,29 +126,35 @@ __device__ __forceinline__ void gate_write_row(int32_t* out, const int (&ti)[KP]
 template <int KP>
 __global__ void __launch_bounds__(kGateTcThreads)
     gate_tc_kernel(const __grid_constant__ CUtensorMap tm_hi, const __grid_constant__ CUtensorMap tm_lo,
-                   GateParams p) {
+                   const __grid_constant__ CUtensorMap tm_q, GateParams p) {
   grid_dependency_sync();
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sQ = smem;
   uint8_t* sM = smem + kGateQBytes;  // 2 stages x (hi, lo); stage 0 doubles as the score staging area
-  __shared__ uint64_t full_bar[2], mma_bar[2], sc_bar, drain_bar;
+  __shared__ uint64_t full_bar[2], mma_bar[2], sc_bar, drain_bar, q_bar;
   __shared__ uint32_t tmem_base;
   __shared__ int abort_flag;
 
   const int g = blockIdx.y;
   const int warp = threadIdx.x >> 5;
   const int row = threadIdx.x;
-  const int64_t rr0 = p.q0 * p.G + (int64_t)blockIdx.x * 128;  // this CTA's first group-row
-  const int64_t rr = rr0 + row;
-  const int64_t t = rr / p.G;
-  const int h = g * p.G + (int)(rr % p.G);
+  // group-row rr = t * G + hl; this CTA's rows start at rr0 = t_cta * G + rem0
+  const uint32_t G = (uint32_t)p.G;
+  const int64_t bxr = (int64_t)blockIdx.x * 128;
+  const int64_t t_cta_off = bxr / p.G;  // the one 64-bit division of a thread
+  const uint32_t rem0 = (uint32_t)(bxr - t_cta_off * p.G);
+  const int64_t t_cta = p.q0 + t_cta_off;  // first token of this CTA's group-rows
+  const uint32_t xr = rem0 + (uint32_t)row;
+  const uint32_t tr = udiv32(xr, G);
+  const int64_t t = t_cta + tr;
+  const int h = g * p.G + (int)(xr - tr * G);
   const bool valid = t < p.S;
-  const int bt = valid ? (int)(t / p.B) : 0;
+  const int bt = valid ? (int)udiv32((uint32_t)t, (uint32_t)p.B) : 0;
   const int P = p.k_eff - 1;
-  int64_t t_last = (rr0 + 127) / p.G;
+  int64_t t_last = t_cta + udiv32(rem0 + 127u, G);
   if (t_last > p.S - 1) t_last = p.S - 1;
-  const int b_cta = (int)(t_last / p.B);  // past blocks of this CTA: j < b_cta
+  const int b_cta = (int)udiv32((uint32_t)t_last, (uint32_t)p.B);  // past blocks of this CTA: j < b_cta
   const int nchunks = (b_cta + kGateBlkChunk - 1) / kGateBlkChunk;
 
   float tv[KP];
@@ -167,27 +174,57 @@ __global__ void __launch_bounds__(kGateTcThreads)
       }
       mbar_init(&sc_bar, 1);
       mbar_init(&drain_bar, 1);
+      mbar_init(&q_bar, 1);
       abort_flag = 0;
       fence_barrier_init();
     }
+    const int row0 = g * p.nbp_pad;  // first mean row of this kv head
+    auto load_chunk = [&](int c) {  // one lane of warp 0
+      const int st = c & 1;
+      uint8_t* dst = sM + st * 2 * kGateSplitBytes;
+      mbar_arrive_expect_tx(&full_bar[st], 2 * kGateSplitBytes);
+      const int r0 = row0 + c * kGateBlkChunk;
+      tma_load_2d(dst, &tm_hi, &full_bar[st], 0, r0);
+      tma_load_2d(dst + kGateSplitHalf, &tm_hi, &full_bar[st], 64, r0);
+      tma_load_2d(dst + kGateSplitBytes, &tm_lo, &full_bar[st], 0, r0);
+      tma_load_2d(dst + kGateSplitBytes + kGateSplitHalf, &tm_lo, &full_bar[st], 64, r0);
+    };
+    // the first two chunks of means do not depend on Q: their copies run
+    // while the Q rows are gathered (the thread that initialised the
+    // barriers issues them)
+    if (threadIdx.x == 0) {
+      if (p.q_tma) {
+        // the CTA's 128 group-rows are 128 / G whole tokens x G heads: one
+        // box (64 channels x G heads x 128/G tokens, 128B swizzle) per half
+        // lands them in the layout the MMA reads (rows past S read zeros)
+        mbar_arrive_expect_tx(&q_bar, kGateQBytes);
+        const int tok = (int)(t_cta - p.q0);
+        tma_load_3d(sQ, &tm_q, &q_bar, 0, g * p.G, tok);
+        tma_load_3d(sQ + kGateQBytes / 2, &tm_q, &q_bar, 64, g * p.G, tok);
+      }
+      load_chunk(0);
+      if (nchunks > 1) load_chunk(1);
+    }
     if (warp == 0) {
+      __syncwarp();
       tmem_alloc(&tmem_base, ncols);
       tmem_relinquish();
     }
     // gather the 128 Q rows (16-byte copies into the 128B-swizzled layout)
-    {
+    if (!p.q_tma) {
       const uint32_t dst0 = smem_u32(sQ);
 #pragma unroll 4
       for (int i = 0; i < 16; ++i) {
         const int idx = threadIdx.x + 128 * i;  // 2048 chunks of 16 B
         const int r = idx >> 4, c16 = idx & 15;
         const int half = c16 >> 3, c = c16 & 7;
-        const int64_t rr_r = rr0 + r;
-        const int64_t t_r = rr_r / p.G;
+        const uint32_t x = rem0 + (uint32_t)r;
+        const uint32_t dt = udiv32(x, G);
+        const int64_t t_r = t_cta + dt;
         const __nv_bfloat16* src = p.q;
         uint32_t bytes = 0;
         if (t_r < p.S) {
-          src = p.q + ((t_r - p.q0) * p.Hq + g * p.G + (int)(rr_r % p.G)) * kHeadDim + c16 * 8;
+          src = p.q + ((t_r - p.q0) * p.Hq + g * p.G + (int)(x - dt * G)) * kHeadDim + c16 * 8;
           bytes = 16;
         }
         cp_async_16(dst0 + half * (kGateQBytes / 2) + r * 128 + ((c ^ (r & 7)) << 4), src, bytes);
@@ -199,39 +236,38 @@ __global__ void __launch_bounds__(kGateTcThreads)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = tmem_base;
+    if (p.q_tma && warp == 0) {
+      // the products read Q: warp 0 (the issuer) waits for its copy (a
+      // timeout sets the abort flag, and nothing is issued)
+      mbar_wait(&q_bar, 0, &abort_flag);
+      __syncwarp();
+    }
     const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
     const uint32_t idesc = idesc_bf16_f32(128, kGateBlkChunk, false);
     const uint64_t dQ = sdesc_sw128(smem_u32(sQ), 16, 1024);
     const uint64_t dM = sdesc_sw128(smem_u32(sM), 16, 1024);
-    const int row0 = g * p.nbp_pad;  // first mean row of this kv head
     volatile int* ab = &abort_flag;
-    int loaded = 0;  // chunks warp 0 has asked TMA for
-    auto load_chunk = [&](int c) {  // one lane of warp 0
-      const int st = c & 1;
-      uint8_t* dst = sM + st * 2 * kGateSplitBytes;
-      mbar_arrive_expect_tx(&full_bar[st], 2 * kGateSplitBytes);
-      const int r0 = row0 + c * kGateBlkChunk;
-      tma_load_2d(dst, &tm_hi, &full_bar[st], 0, r0);
-      tma_load_2d(dst + kGateSplitHalf, &tm_hi, &full_bar[st], 64, r0);
-      tma_load_2d(dst + kGateSplitBytes, &tm_lo, &full_bar[st], 0, r0);
-      tma_load_2d(dst + kGateSplitBytes + kGateSplitHalf, &tm_lo, &full_bar[st], 64, r0);
-    };
+    int loaded = min(nchunks, 2);  // chunks asked of TMA so far
     // staging of one 32-column piece of scores per row (for the insertions,
     // which index columns per lane): 128 B per row in ring stage 0, 16-byte
     // pieces swizzled by row so that 8 consecutive rows hit distinct banks
     float* stg = reinterpret_cast<float*>(sM) + row * 32;
     const int nsc = (nchunks + 3) / 4;
     for (int sc = 0; sc < nsc; ++sc) {
+      if (*ab) break;
       const int c_lo = 4 * sc;
       const int nc = min(4, nchunks - c_lo);
       if (warp == 0) {
         // scores of this super-chunk: chunk c_lo + c into TMEM columns 64c
-        if (elect_one()) {
-          load_chunk(c_lo);
-          if (nc > 1) load_chunk(c_lo + 1);
+        // (the first super-chunk's first two chunks are already on their way)
+        if (sc > 0) {
+          if (elect_one()) {
+            load_chunk(c_lo);
+            if (nc > 1) load_chunk(c_lo + 1);
+          }
+          __syncwarp();
+          loaded = c_lo + min(nc, 2);
         }
-        __syncwarp();
-        loaded = c_lo + min(nc, 2);
         for (int c = 0; c < nc; ++c) {
           const int gc = c_lo + c, st = gc & 1;
           if (!mbar_wait(&full_bar[st], (gc >> 1) & 1, ab)) break;
@@ -334,8 +370,10 @@ __global__ void __launch_bounds__(kGateTcThreads)
       // shared memory and TMEM go away (bounded waits, flag ignored)
       volatile int keep_waiting = 0;
       if (warp == 0) {
-        if (elect_one())
+        if (elect_one()) {
           for (int c = 0; c < loaded; ++c) mbar_wait(&full_bar[c & 1], (c >> 1) & 1, &keep_waiting, (1ull << 28));
+          if (p.q_tma) mbar_wait(&q_bar, 0, &keep_waiting, (1ull << 28));
+        }
         __syncwarp();
         if (elect_one()) mma_commit(&drain_bar);
         __syncwarp();

@@ -96,13 +96,16 @@ __global__ void __launch_bounds__(256, 3) merge_kernel(MergeParams m) {
   // end (or a token before q0) runs on a harmless row and writes nothing
   bool live = row < nrows;
   if (!live) row = nrows - 1;
-  const int64_t tl = row / w.Hq;
-  const int h = (int)(row % w.Hq);
+  // 32-bit divisions: a window's rows (wlen * Hq) and every token index fit
+  // in 32 bits (the host bounds the window's list slots and seqlen by 2^31)
+  const uint32_t tl32 = udiv32((uint32_t)row, (uint32_t)w.Hq);
+  const int64_t tl = tl32;
+  const int h = (int)((uint32_t)row - tl32 * (uint32_t)w.Hq);
   const int64_t t = w.w0 + tl;
   if (t < w.q0) live = false;
   const int64_t tq = max(t - w.q0, (int64_t)0), nq = w.S - w.q0;
-  const int g = h / w.G, hl = h % w.G;
-  const int bt = (int)(t / w.B);
+  const int g = (int)udiv32((uint32_t)h, (uint32_t)w.G), hl = h - g * w.G;
+  const int bt = (int)udiv32((uint32_t)t, (uint32_t)w.B);
   const int64_t rr = tl * w.G + hl;
   const int64_t word = rr >> 5;
   const uint32_t below = (1u << (rr & 31)) - 1u;

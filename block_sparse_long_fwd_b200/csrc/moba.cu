@@ -315,9 +315,10 @@ int make_plan(Plan* pl, int64_t S, int64_t q0, int Hq, int Hkv, int B, int topk,
     if (W > 1024 && W % 1024) W = W / 1024 * 1024;
   }
   W = std::min(W, S128);
-  // list slots and positions are 32-bit
-  while (W > 128 && W * Hq * (int64_t)p.P >= ((int64_t)1 << 31) - 1) W = std::max<int64_t>(128, W / 2 / 128 * 128);
-  if (W * Hq * (int64_t)p.P >= ((int64_t)1 << 31) - 1) return fail(MOBA_ERR_UNSUPPORTED, "window too large");
+  // list slots, positions and a window's rows (token x head) are 32-bit
+  const int64_t per_tok = (int64_t)Hq * std::max(p.P, 1);
+  while (W > 128 && W * per_tok >= ((int64_t)1 << 31) - 1) W = std::max<int64_t>(128, W / 2 / 128 * 128);
+  if (W * per_tok >= ((int64_t)1 << 31) - 1) return fail(MOBA_ERR_UNSUPPORTED, "window too large");
   layout_for_window(p, W);
   return MOBA_OK;
 }
@@ -356,10 +357,26 @@ void launch_chained(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem
 }
 
 template <int KP>
-void launch_gate_tc(const Plan& p, const CUtensorMap& mhi, const CUtensorMap& mlo, const moba::GateParams& gp,
-                    cudaStream_t st) {
+void launch_gate_tc(const Plan& p, const CUtensorMap& mhi, const CUtensorMap& mlo, const CUtensorMap& mq,
+                    const moba::GateParams& gp, cudaStream_t st) {
   dim3 grid((unsigned)(((p.S - p.q0) * p.G + 127) / 128), p.Hkv);
-  launch_chained(moba::gate_tc_kernel<KP>, grid, dim3(moba::kGateTcThreads), moba::kGateSmemBytes, st, mhi, mlo, gp);
+  launch_chained(moba::gate_tc_kernel<KP>, grid, dim3(moba::kGateTcThreads), moba::kGateSmemBytes, st, mhi, mlo, mq,
+                 gp);
+}
+
+// q [S - q0][Hq][128] bf16 as 3-D (channel, head, token) for the gate's Q
+// tiles: box 64 x G x 128/G (one 64-channel half of 128 group-rows), 128-byte
+// swizzle. Only when G divides 128.
+int make_gate_q_map(CUtensorMap* map, const void* q, int64_t ntok, int Hq, int G) {
+  cuuint64_t dims[3] = {(cuuint64_t)moba::kHeadDim, (cuuint64_t)Hq, (cuuint64_t)ntok};
+  cuuint64_t strides[2] = {(cuuint64_t)moba::kHeadDim * 2, (cuuint64_t)Hq * moba::kHeadDim * 2};
+  cuuint32_t box[3] = {64, (cuuint32_t)G, (cuuint32_t)(128 / G)};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(q), dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(MOBA_ERR_CUDA, "cuTensorMapEncodeTiled (gate q) failed (%d)", (int)r);
+  return MOBA_OK;
 }
 
 // Gate + top-k into sel. kmean (fp32) is split into khi/klo (bf16, padded
@@ -382,7 +399,16 @@ int launch_gate(const Plan& p, const void* q, const float* kmean, int splits, __
   if (rc) return -rc;
   rc = make_mean_map(&mlo, klo, (int64_t)p.Hkv * nbp_pad);
   if (rc) return -rc;
+  // Q tiles by TMA when a CTA's 128 group-rows are whole tokens (G | 128)
+  CUtensorMap mq;
+  memset(&mq, 0, sizeof(mq));
+  const bool q_tma = p.G <= 128 && 128 % p.G == 0;
+  if (q_tma) {
+    rc = make_gate_q_map(&mq, q, p.S - p.q0, p.Hq, p.G);
+    if (rc) return -rc;
+  }
   moba::GateParams gp;
+  gp.q_tma = q_tma ? 1 : 0;
   gp.q = static_cast<const __nv_bfloat16*>(q);
   gp.sel = sel;
   gp.S = p.S;
@@ -392,15 +418,15 @@ int launch_gate(const Plan& p, const void* q, const float* kmean, int splits, __
   gp.B = p.B;
   gp.nbp_pad = nbp_pad;
   gp.k_eff = p.k_eff;
-  if (p.P <= 2) launch_gate_tc<2>(p, mhi, mlo, gp, st);
-  else if (p.P <= 4) launch_gate_tc<4>(p, mhi, mlo, gp, st);
-  else if (p.P <= 8) launch_gate_tc<8>(p, mhi, mlo, gp, st);
-  else if (p.P <= 12) launch_gate_tc<12>(p, mhi, mlo, gp, st);
-  else if (p.P <= 16) launch_gate_tc<16>(p, mhi, mlo, gp, st);
-  else if (p.P <= 24) launch_gate_tc<24>(p, mhi, mlo, gp, st);
-  else if (p.P <= 32) launch_gate_tc<32>(p, mhi, mlo, gp, st);
-  else if (p.P <= 48) launch_gate_tc<48>(p, mhi, mlo, gp, st);
-  else launch_gate_tc<64>(p, mhi, mlo, gp, st);
+  if (p.P <= 2) launch_gate_tc<2>(p, mhi, mlo, mq, gp, st);
+  else if (p.P <= 4) launch_gate_tc<4>(p, mhi, mlo, mq, gp, st);
+  else if (p.P <= 8) launch_gate_tc<8>(p, mhi, mlo, mq, gp, st);
+  else if (p.P <= 12) launch_gate_tc<12>(p, mhi, mlo, mq, gp, st);
+  else if (p.P <= 16) launch_gate_tc<16>(p, mhi, mlo, mq, gp, st);
+  else if (p.P <= 24) launch_gate_tc<24>(p, mhi, mlo, mq, gp, st);
+  else if (p.P <= 32) launch_gate_tc<32>(p, mhi, mlo, mq, gp, st);
+  else if (p.P <= 48) launch_gate_tc<48>(p, mhi, mlo, mq, gp, st);
+  else launch_gate_tc<64>(p, mhi, mlo, mq, gp, st);
   return 2;
 }
 
@@ -1412,7 +1438,7 @@ int plan_within(Plan* pl, int64_t S, int Hq, int Hkv, int B, int topk, size_t ca
   plan_shape(p, S, 0, Hq, Hkv, B, topk);
   int64_t W = (S + 127) / 128 * 128;
   while (true) {
-    if (W * Hq * (int64_t)p.P < ((int64_t)1 << 31) - 1) {
+    if (W * Hq * (int64_t)std::max(p.P, 1) < ((int64_t)1 << 31) - 1) {
       layout_for_window(p, W);
       if (p.total <= cap) return MOBA_OK;
     }

@@ -62,6 +62,8 @@ CASES = [
     (600,   2,  1,   256, 8,    4),   # topk >= blocks: the dense path
     (500,   2,  2,   128, 1,    5),   # own block only
     (1,     2,  1,   128, 3,    6),   # one token
+    (4096,  4,  1,   512, 4,    7),   # 4K tokens, four q heads on one kv head, three routed blocks per row:
+                                      # dK / dV summed over a group's heads and over routed and own rows
 ]
 
 
