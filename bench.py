@@ -47,8 +47,9 @@ def load_peaks():
 
 
 def attn_traffic(workload_name: str):
-    """DRAM bytes per attention launch from the committed ncu record, or None
-    when the record is for another workload or an older attention kernel."""
+    """DRAM bytes of the attention kernel per step (its launches summed) from
+    the committed ncu record, or None when the record is for another workload
+    or an older attention kernel."""
     import hashlib
     rec = os.path.join(ROOT, "profiles", "attn_kernel_traffic.txt")
     src = os.path.join(ROOT, "block_sparse_long_fwd_b200", "csrc", "attn.cuh")
@@ -60,7 +61,7 @@ def attn_traffic(workload_name: str):
                 kv[k.strip()] = v.strip()
         sha = hashlib.sha256(open(src, "rb").read()).hexdigest()
         if kv.get("kernel_source_sha256") == sha and kv.get("workload") == workload_name:
-            return int(kv["bytes_per_launch"])
+            return int(kv["bytes_per_step"])
     except (OSError, ValueError, KeyError):
         pass
     return None
