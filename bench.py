@@ -243,6 +243,44 @@ def chunk_flops(w, q0: int) -> float:
     return 4.0 * w.head_dim * w.heads_q * float(keys.sum())
 
 
+DECODE_ROWS = 64  # chunks of at most this many query tokens are reported against HBM
+
+
+def chunk_kv_bytes(w, q_h, k, q0: int) -> int:
+    """Algorithmic HBM bytes of the attention for the queries of tokens
+    q0..S-1: per kv head, the K and V rows of every block that some of its q
+    heads' rows attend (own block up to the last query token, plus the past
+    blocks the gate picks), the chunk's Q rows and its partial outputs. The
+    picks are recomputed here from the library's pooled block means (a
+    measurement helper: which blocks are read, not how they are combined)."""
+    import torch
+
+    import block_sparse_long_fwd_b200 as moba
+    S, B, d = w.seqlen, w.block_size, w.head_dim
+    G = w.heads_q // w.heads_kv
+    P = min(w.topk, w.nblocks) - 1
+    km = moba.pool(k, B).double().cpu().numpy()  # [Hkv][nbp][d]
+    q = q_h[q0:].view(torch.int16).numpy().astype(np.uint32) << 16
+    q = q.view(np.float32).astype(np.float64)  # [n][Hq][d]
+    keys = 0  # K/V rows read, summed over kv heads
+    own_last = {}  # own block -> its last token with a query
+    for t in range(q0, S):
+        own_last[t // B] = t
+    for g in range(w.heads_kv):
+        past = set()
+        for tl in range(S - q0):
+            t = q0 + tl
+            b = t // B
+            if b and P:
+                s = q[tl, g * G:(g + 1) * G] @ km[g, :b].T  # [G][b]
+                for row in s:
+                    past.update(np.argsort(-row, kind="stable")[:P].tolist())
+        past -= set(own_last)
+        keys += len(past) * B + sum(t - b * B + 1 for b, t in own_last.items())
+    rows = (S - q0) * w.heads_q
+    return int(keys * d * 2 * 2 + rows * d * 2 + rows * min(w.topk, w.nblocks) * (d * 2 + 4))
+
+
 def run_chunk(args, w):
     """--chunk N: the last N tokens' queries against the whole cache
     (moba_fwd_chunk; N = 1 is one decode step). One GPU."""
@@ -311,6 +349,22 @@ def run_chunk(args, w):
     flops = chunk_flops(w, q0)
     attn_ms = stages["attention"] / max(calls, 1)
     achieved = flops / (attn_ms / 1e3) / 1e12
+    if n <= DECODE_ROWS:
+        # a few query tokens: the attention streams the K/V rows of the blocks
+        # they attend, so it is bound by HBM, not by the tensor cores
+        kv_bytes = chunk_kv_bytes(w, q_h, k, q0)
+        gbs = kv_bytes / (attn_ms / 1e3) / 1e9
+        roofline = {"bound": "hbm", "kernel": "attn_kernel", "achieved": gbs, "peak": peaks["hbm_gbs"],
+                    "unit": "GB/s", "frac": gbs / peaks["hbm_gbs"], "traffic": None,
+                    "peak_source": f"{peaks_src} HBM copy",
+                    "algorithmic": f"{kv_bytes:.4e} bytes: K and V rows of the distinct blocks the chunk's rows attend "
+                                   "(per kv head), its Q rows and its partial outputs / attention ms",
+                    "tflops": achieved}
+    else:
+        roofline = {"bound": "tensor", "kernel": "attn_kernel", "achieved": achieved,
+                    "peak": peaks["bf16_tflops"], "unit": "TFLOP/s", "frac": achieved / peaks["bf16_tflops"],
+                    "traffic": None, "peak_source": f"{peaks_src} bf16 burst",
+                    "algorithmic": f"{flops:.4e} selected-block FLOPs of the chunk's rows / attention ms"}
     line = {
         "metric": METRIC, "value": n * args.steps / (total_ms / 1e3), "unit": "tokens/s", "n_gpus": 1,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True,
@@ -319,10 +373,7 @@ def run_chunk(args, w):
                        block_means="cached (pooled once)" if args.cached_means else "pooled every call"),
         "eff_tflops": flops * args.steps / (total_ms / 1e3) / 1e12,
         "stage_ms_per_step": {kk: vv / max(calls, 1) for kk, vv in stages.items() if not kk.startswith("bwd_")},
-        "roofline": {"bound": "tensor", "kernel": "attn_kernel", "achieved": achieved,
-                     "peak": peaks["bf16_tflops"], "unit": "TFLOP/s", "frac": achieved / peaks["bf16_tflops"],
-                     "traffic": None, "peak_source": f"{peaks_src} bf16 burst",
-                     "algorithmic": f"{flops:.4e} selected-block FLOPs of the chunk's rows / attention ms"},
+        "roofline": roofline,
         "e2e": {"value": n * e2e_steps / (e2e_ms / 1e3), "unit": "tokens/s",
                 "h2d_bytes_per_step": int(n * (Hq + 2 * Hkv) * d * 2),
                 "d2h_bytes_per_step": int(out_h.nbytes + lse_h.nbytes)},

@@ -304,7 +304,9 @@ __global__ void __launch_bounds__(kGateTcThreads)
       const int jb = sc * 4 * kGateBlkChunk;                 // block of column 0
       const int jn = max(0, min(nc * kGateBlkChunk, bt - jb));  // this row's past blocks here
       float tau = -INFINITY;
-      if (KP <= 24) {
+      // the group-maximum bound pays only while some row's list is not yet
+      // full; after that the rows' running KP-th best filters the columns
+      if (KP <= 24 && __any_sync(0xffffffffu, tv[KP - 1] == -INFINITY)) {
         constexpr int NG = KP <= 24 ? KP : 1;
         float gm[NG];
 #pragma unroll
