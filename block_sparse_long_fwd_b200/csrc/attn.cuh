@@ -29,9 +29,10 @@
 // waits for a P.V product, and both tiles' softmaxes run concurrently while
 // the tensor core works through S_A(s+1), PV_A(s), S_B(s+1), PV_B(s).
 // The running max moves (and O, l are rescaled) only when it grows by more
-// than 8 in log2 units. A quarter of the exponentials are evaluated on the
-// FMA pipe (range reduction 2^x = 2^n 2^f, |f| <= 1/2, and a minimax cubic
-// for 2^f) to take load off the MUFU unit.
+// than 8 in log2 units. Every exponential is one MUFU ex2: with the tensor
+// core this busy the SM runs at its power limit, and moving a share of them
+// to a polynomial on the FMA pipe cost more (issue slots, energy) than it
+// saved on the MUFU unit (measured at 1M tokens: 1,124 against 1,186 TFLOP/s).
 //
 // TMEM (512 columns): S 0..127, P_A 128..191, P_B 192..255 (bf16 pairs),
 // O_A 256..383, O_B 384..511.
@@ -155,47 +156,19 @@ __device__ __forceinline__ UnitInfo decode_unit(const AttnParams& p, int idx) {
   return u;
 }
 
-// Minimax cubic for 2^f on [-1/2, 1/2] (relative error 7.5e-5), fitted for
-// this kernel with the Remez exchange algorithm. 2^x = 2^n * 2^f with
-// n = rint(x) taken from the low mantissa bits of x + 1.5*2^23; 2^n is then
-// added to the exponent field of the cubic's value.
-constexpr float kExp2C0 = 0.9999280571937561f;
-constexpr float kExp2C1 = 0.6932609677314758f;
-constexpr float kExp2C2 = 0.2426111251115799f;
-constexpr float kExp2C3 = 0.0551716685295105f;
-
 // P = 2^(s*c - m) for one 128-column row of S held as raw fp32 bits in r,
 // on column pairs with packed fp32 arithmetic, into 64 registers of bf16
 // pairs (pk[i] = columns 2i, 2i+1). Row sums accumulate into sum2 (four
-// packed pairs). With kPoly, one pair in four is evaluated on the FMA pipe
-// (minimax cubic above) instead of MUFU; columns masked to -inf must use the
-// MUFU path (kPoly false).
-template <bool kPoly>
+// packed pairs).
 __device__ __forceinline__ void exp_row(const uint32_t (&r)[128], uint64_t c2, uint64_t nm2, uint64_t (&sum2)[4],
                                         uint32_t (&pk)[64]) {
 #pragma unroll
-  for (int ch = 0; ch < 4; ++ch) {
-#pragma unroll
-    for (int e = ch * 32; e < ch * 32 + 32; e += 2) {
-      const uint64_t x2 = f2_fma((uint64_t)r[e] | ((uint64_t)r[e + 1] << 32), c2, nm2);
-      float a, b;
-      if (kPoly && (e & 6) == 6) {
-        const uint64_t xx = f2_pack(fmaxf(f2_lo(x2), -125.f), fmaxf(f2_hi(x2), -125.f));
-        const uint64_t t2 = f2_add(xx, f2_pack(12582912.f, 12582912.f));    // + 1.5 * 2^23
-        const uint64_t n2 = f2_add(t2, f2_pack(-12582912.f, -12582912.f));  // rint(x)
-        const uint64_t fr = f2_fma(n2, f2_pack(-1.f, -1.f), xx);            // x - rint(x)
-        uint64_t q = f2_fma(f2_pack(kExp2C3, kExp2C3), fr, f2_pack(kExp2C2, kExp2C2));
-        q = f2_fma(q, fr, f2_pack(kExp2C1, kExp2C1));
-        q = f2_fma(q, fr, f2_pack(kExp2C0, kExp2C0));
-        a = __int_as_float(__float_as_int(f2_lo(q)) + (__float_as_int(f2_lo(t2)) << 23));
-        b = __int_as_float(__float_as_int(f2_hi(q)) + (__float_as_int(f2_hi(t2)) << 23));
-      } else {
-        a = ex2_approx(f2_lo(x2));
-        b = ex2_approx(f2_hi(x2));
-      }
-      sum2[(e >> 1) & 3] = f2_add(sum2[(e >> 1) & 3], f2_pack(a, b));
-      pk[e >> 1] = pack_bf16x2(a, b);
-    }
+  for (int e = 0; e < 128; e += 2) {
+    const uint64_t x2 = f2_fma((uint64_t)r[e] | ((uint64_t)r[e + 1] << 32), c2, nm2);
+    const float a = ex2_approx(f2_lo(x2));
+    const float b = ex2_approx(f2_hi(x2));
+    sum2[(e >> 1) & 3] = f2_add(sum2[(e >> 1) & 3], f2_pack(a, b));
+    pk[e >> 1] = pack_bf16x2(a, b);
   }
 }
 
@@ -343,11 +316,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           const uint64_t c2 = f2_pack(p.scale_log2, p.scale_log2);
           const uint64_t nm2 = f2_pack(-m_ref, -m_ref);
           uint64_t sum2[4] = {0ull, 0ull, 0ull, 0ull};
-          if (diag) {
-            exp_row<false>(r, c2, nm2, sum2, pk);
-          } else {
-            exp_row<true>(r, c2, nm2, sum2, pk);
-          }
+          exp_row(r, c2, nm2, sum2, pk);
           const uint64_t s01 = f2_add(f2_add(sum2[0], sum2[1]), f2_add(sum2[2], sum2[3]));
           l_run = l_run * factor + (f2_lo(s01) + f2_hi(s01));
           m_run = m_ref;
