@@ -46,6 +46,14 @@ def load_peaks():
         return dict(FALLBACK_PEAKS), "fallback"
 
 
+def tensor_peak(peaks, peaks_src, ms_per_step):
+    """bf16 dense peak for a kernel timed inside a step: the burst figure for
+    steps under 200 ms, the sustained (power-capped) one for longer steps."""
+    long_step = ms_per_step > 200.0
+    key = "bf16_tflops_sustained" if long_step else "bf16_tflops"
+    return peaks[key], f"{peaks_src} bf16 {'sustained' if long_step else 'burst'}"
+
+
 def attn_traffic(workload_name: str):
     """DRAM bytes of the attention kernel per step (its launches summed) from
     the committed ncu record, or None when the record is for another workload
@@ -361,9 +369,10 @@ def run_chunk(args, w):
                                    "(per kv head), its Q rows and its partial outputs / attention ms",
                     "tflops": achieved}
     else:
+        peak, psrc = tensor_peak(peaks, peaks_src, total_ms / args.steps)
         roofline = {"bound": "tensor", "kernel": "attn_kernel", "achieved": achieved,
-                    "peak": peaks["bf16_tflops"], "unit": "TFLOP/s", "frac": achieved / peaks["bf16_tflops"],
-                    "traffic": None, "peak_source": f"{peaks_src} bf16 burst",
+                    "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
+                    "traffic": None, "peak_source": psrc,
                     "algorithmic": f"{flops:.4e} selected-block FLOPs of the chunk's rows / attention ms"}
     line = {
         "metric": METRIC, "value": n * args.steps / (total_ms / 1e3), "unit": "tokens/s", "n_gpus": 1,
@@ -451,6 +460,7 @@ def run_backward(args, w):
     fwd_flops = chunk_flops(w, 0)
     per = {kk: vv / max(calls, 1) for kk, vv in stages.items() if kk not in ("attention", "merge")}
     dkdv_flops = 2.0 * fwd_flops  # S^T, dP^T, dV, dK
+    peak, psrc = tensor_peak(peaks, peaks_src, total_ms / args.steps)
     achieved = dkdv_flops / (per["bwd_dkdv"] / 1e3) / 1e12
     line = {
         "metric": METRIC, "value": S * args.steps / (total_ms / 1e3), "unit": "tokens/s", "n_gpus": 1,
@@ -460,8 +470,8 @@ def run_backward(args, w):
         "eff_tflops": 2.5 * fwd_flops * args.steps / (total_ms / 1e3) / 1e12,
         "stage_ms_per_step": per,
         "roofline": {"bound": "tensor", "kernel": "bwd_dkdv_kernel", "achieved": achieved,
-                     "peak": peaks["bf16_tflops"], "unit": "TFLOP/s", "frac": achieved / peaks["bf16_tflops"],
-                     "traffic": None, "peak_source": f"{peaks_src} bf16 burst",
+                     "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
+                     "traffic": None, "peak_source": psrc,
                      "algorithmic": f"{dkdv_flops:.4e} FLOPs (S^T, dP^T, dV, dK per attended pair) / dK-dV ms",
                      "dq_kernel_tflops": 1.5 * fwd_flops / (per["bwd_dq"] / 1e3) / 1e12},
         "e2e": {"value": S * e2e_steps / (e2e_ms / 1e3), "unit": "tokens/s",
@@ -550,6 +560,7 @@ def run_varlen(args, w):
     flops = sum(chunk_flops(sw, 0) for sw in subs)
     attn_ms = stages["attention"] / args.steps
     achieved = flops / (attn_ms / 1e3) / 1e12
+    peak, psrc = tensor_peak(peaks, peaks_src, total_ms / args.steps)
     line = {
         "metric": METRIC, "value": T * args.steps / (total_ms / 1e3), "unit": "tokens/s", "n_gpus": 1,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True,
@@ -559,8 +570,8 @@ def run_varlen(args, w):
         "eff_tflops": flops * args.steps / (total_ms / 1e3) / 1e12,
         "stage_ms_per_step": {kk: vv / args.steps for kk, vv in stages.items() if not kk.startswith("bwd_")},
         "roofline": {"bound": "tensor", "kernel": "attn_kernel", "achieved": achieved,
-                     "peak": peaks["bf16_tflops"], "unit": "TFLOP/s", "frac": achieved / peaks["bf16_tflops"],
-                     "traffic": None, "peak_source": f"{peaks_src} bf16 burst",
+                     "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
+                     "traffic": None, "peak_source": psrc,
                      "algorithmic": f"{flops:.4e} selected-block FLOPs of all sequences / attention ms"},
         "e2e": {"value": T * e2e_steps / (e2e_ms / 1e3), "unit": "tokens/s",
                 "h2d_bytes_per_step": int(q_h.nbytes + k_h.nbytes + v_h.nbytes),
@@ -688,8 +699,7 @@ def run_ours(args, w):
         value = job_tokens_per_s(world, S, args.steps, total_ms)
         ms_per_step = total_ms / args.steps
         attn_ms = stages["attention"] / max(calls, 1)
-        long_step = ms_per_step > 200.0
-        peak = peaks["bf16_tflops_sustained"] if long_step else peaks["bf16_tflops"]
+        peak, psrc = tensor_peak(peaks, peaks_src, ms_per_step)
         achieved = flops / (attn_ms / 1e3) / 1e12
         sb = stage_bytes(wr)
         stage_roof = {}
@@ -708,7 +718,7 @@ def run_ours(args, w):
             "ms_per_step_kernel_by_kernel": prof_ms,
             "roofline": {"bound": "tensor", "kernel": "attn_kernel", "achieved": achieved, "peak": peak,
                          "unit": "TFLOP/s", "frac": achieved / peak, "traffic": attn_traffic(wr.name),
-                         "peak_source": f"{peaks_src} bf16 {'sustained' if long_step else 'burst'}",
+                         "peak_source": psrc,
                          "algorithmic": f"{flops:.4e} selected-block FLOPs per step / attention ms per step"},
             "stage_roofline_hbm": stage_roof,
             "e2e": {"value": job_tokens_per_s(world, S, e2e_steps, e2e_total), "unit": "tokens/s",
