@@ -756,6 +756,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--seqlen", type=int, default=0, help="override the workload's seqlen (profiling cases)")
+    ap.add_argument("--heads", type=str, default="",
+                    help="override the workload's q:kv heads, e.g. 4:1 (profiling cases)")
     ap.add_argument("--no-pad", action="store_true", help="no untimed load after the timed steps (profiling)")
     ap.add_argument("--chunk", type=int, default=0,
                     help="time only the last N tokens' queries against the whole cache (1 = one decode step)")
@@ -772,6 +774,14 @@ def main():
     if args.seqlen:
         w = si.Workload(f"{w.name}_s{args.seqlen}", args.seqlen, w.heads_q, w.heads_kv, w.head_dim, w.block_size,
                         w.topk, w.seed)
+    if args.heads:
+        try:
+            hq, hkv = (int(x) for x in args.heads.split(":"))
+        except ValueError:
+            ap.error("--heads takes q:kv, e.g. 4:1")
+        if hq < 1 or hkv < 1 or hq % hkv:
+            ap.error("--heads: q heads must be a positive multiple of kv heads")
+        w = si.Workload(f"{w.name}_h{hq}kv{hkv}", w.seqlen, hq, hkv, w.head_dim, w.block_size, w.topk, w.seed)
     # one timed mode at a time, checked before any GPU work
     if sum(bool(x) for x in (args.chunk, args.varlen, args.backward)) > 1:
         ap.error("--chunk, --varlen and --backward are separate modes: give at most one")

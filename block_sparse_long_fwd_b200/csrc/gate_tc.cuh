@@ -13,9 +13,11 @@
 // per channel. The 128 rows of a CTA read their scores from TMEM (thread =
 // row = TMEM lane) and keep the KP best (score, block) pairs in registers; a
 // block enters only with a strictly larger score, so equal scores keep the
-// lower index. Chunks of block means come in by TMA into a two-stage ring,
-// the Q rows by cp.async, and two TMEM score buffers let the MMA of the next
-// chunk run while the current one is scanned.
+// lower index. Q comes in by TMA (or cp.async when a tile's rows are not
+// whole tokens), chunks of block means by TMA into one shared-memory stage.
+// A CTA holds one Q tile, one means stage and 128 TMEM columns, so three or
+// four CTAs share an SM: the scan of one CTA's rows, which bounds the
+// kernel, overlaps the copies and products of the others.
 #pragma once
 
 #include "common.cuh"
@@ -23,16 +25,39 @@
 namespace moba {
 
 constexpr int kGateTcThreads = 128;
-constexpr int kGateBlkChunk = 64;                              // blocks per MMA chunk
-constexpr uint32_t kGateQBytes = 128 * kHeadDim * 2;          // 32 KB Q tile
-constexpr uint32_t kGateSplitBytes = kGateBlkChunk * kHeadDim * 2;  // 16 KB: one part of a chunk
-constexpr uint32_t kGateSplitHalf = kGateSplitBytes / 2;      // one 64-channel half
-constexpr int kGateSmemBytes = kGateQBytes + 2 * 2 * kGateSplitBytes + 1024 + 256;
+constexpr int kGatePadRows = 64;   // block-mean rows per kv head are padded to a multiple of this
+constexpr int kGateBoxRows = 32;   // block-mean rows of one TMA box
+constexpr int kGateScCols = 128;   // TMEM columns of a super-chunk (the scores scanned at once)
+constexpr int kGatePieces = kGateScCols / 32;          // 32-column pieces of a super-chunk
+constexpr uint32_t kGateQBytes = 128 * kHeadDim * 2;  // 32 KB Q tile
 
-// Block-mean rows are padded to a multiple of the chunk so a chunk never
+// Shapes that depend on the list length KP.
+template <int KP>
+struct GateCfg {
+  // lists of up to 16 entries: 32-block chunks (a 16 KB means stage) and four
+  // CTAs per SM within 128 registers a thread; longer lists take more
+  // registers: 64-block chunks, and as many CTAs as fit
+  static constexpr int kChunk = KP <= 16 ? 32 : 64;
+  static constexpr int kMinCtas = KP <= 16 ? 4 : (KP <= 48 ? 3 : 2);
+  static constexpr int kScChunks = kGateScCols / kChunk;
+  static constexpr uint32_t kSplitBytes = kChunk * kHeadDim * 2;  // one part (hi or lo) of a chunk
+  static constexpr uint32_t kSplitHalf = kSplitBytes / 2;          // one 64-channel half
+  static constexpr int kSmemBytes = kGateQBytes + 2 * kSplitBytes + 1024 + 256;  // Q tile, one means stage
+  // the bound on a row's KP-th best score comes from the maxima of kGroups
+  // disjoint column groups (about 3 KP of them, a power of two, at most 32);
+  // lists of more than 32 entries go without it
+  static constexpr bool kBound = KP <= 32;
+  static constexpr int kGroups = KP <= 2 ? 8 : (KP <= 4 ? 16 : 32);
+  // the means stage doubles as the per-row score staging area (128 rows x 128 B)
+  static_assert(2 * kSplitBytes >= 128 * 128, "the staging area does not fit the means stage");
+  static_assert(kChunk % kGateBoxRows == 0 && kGatePadRows % kChunk == 0, "chunk shape");
+  static_assert(!kBound || kGroups >= KP, "the bound needs at least KP groups");
+};
+
+// Block-mean rows are padded to a multiple of kGatePadRows so a chunk never
 // crosses into the next kv head.
 __host__ __device__ inline int gate_rows_padded(int nbp) {
-  return (nbp + kGateBlkChunk - 1) / kGateBlkChunk * kGateBlkChunk;
+  return (nbp + kGatePadRows - 1) / kGatePadRows * kGatePadRows;
 }
 
 // Block means -> hi, lo bf16 [Hkv][nbp_pad][128]; padding rows are zero.
@@ -65,6 +90,40 @@ struct GateParams {
   int Hq, G, B, nbp_pad, k_eff;
   int q_tma;               // 1: G divides 128 and tm_q is valid (Q tiles by TMA)
 };
+
+// Sorts N values (a power of two) in descending order: a bitonic network,
+// every index a compile-time constant so the values stay in registers.
+template <int N>
+__device__ __forceinline__ void sort_desc(float (&a)[N]) {
+#pragma unroll
+  for (int k = 2; k <= N; k <<= 1) {
+#pragma unroll
+    for (int j = k >> 1; j > 0; j >>= 1) {
+#pragma unroll
+      for (int i = 0; i < N; ++i) {
+        const int l = i ^ j;
+        if (l > i) {
+          const float x = a[i], y = a[l];
+          if ((i & k) == 0) {
+            a[i] = fmaxf(x, y);
+            a[l] = fminf(x, y);
+          } else {
+            a[i] = fminf(x, y);
+            a[l] = fmaxf(x, y);
+          }
+        }
+      }
+    }
+  }
+}
+
+// The smallest float above x (x finite or -inf): v > x exactly when
+// v >= float_above(x). Bit arithmetic, so it holds for subnormals too.
+__device__ __forceinline__ float float_above(float x) {
+  const uint32_t u = __float_as_uint(x);
+  if (u == 0x80000000u) return __uint_as_float(1u);  // -0: the smallest positive subnormal
+  return __uint_as_float((int32_t)u >= 0 ? u + 1u : u - 1u);
+}
 
 template <int KP>
 __device__ __forceinline__ void gate_insert(float (&tv)[KP], int (&ti)[KP], float s, int j) {
@@ -108,31 +167,38 @@ __device__ __forceinline__ void gate_write_row(int32_t* out, const int (&ti)[KP]
 // grid (ceil((S - q0)*G / 128), Hkv), 128 threads; row = TMEM lane = group-row
 // blockIdx.x*128 + threadIdx.x.
 //
-// The CTA's past blocks are scored in super-chunks of up to four 64-block
-// chunks (256 TMEM columns): warp 0 streams each chunk's hi/lo means through
-// a two-stage TMA ring and issues its products into the chunk's 64 columns.
-// Once a super-chunk is scored, every row selects from it in two passes over
-// its TMEM columns:
-//   1. tau = the smallest of KP group maxima, the groups being KP disjoint
-//      sets of the row's columns (column i in group i mod KP). KP columns
-//      reach tau, so a column strictly below it cannot be among the row's
-//      best KP (an equal one still can: ties go to the lower block);
+// The CTA's past blocks are scored in super-chunks of kGateScCols columns:
+// warp 0 streams each chunk's hi/lo means through the one means stage and
+// issues its products into the chunk's TMEM columns. Every row then selects
+// in two passes over its scores:
+//   1. tau = the KP-th largest of the maxima of kGroups disjoint column
+//      groups (column c in group c mod kGroups) over all the row's past
+//      blocks. KP columns reach tau, so a column strictly below it cannot be
+//      among the row's best KP (an equal one still can: ties go to the lower
+//      block);
 //   2. the columns with score >= tau that also beat the row's current KP-th
 //      best (strictly: the list's blocks are lower) are inserted in
 //      ascending block order into the row's sorted list.
-// With KP disjoint groups over ~255 scores, about 14 columns survive the
-// filter per row instead of the ~48 insertions of a plain scan. Lists of 32
-// or more entries (few rows, many columns each) skip the filter.
+// With 32 groups, about 13 columns per row survive (in a warp, at most ~17),
+// against ~30 (~55) for the smallest of KP group maxima over one
+// super-chunk, and every candidate costs a sorted insertion. When a CTA's
+// blocks fill one super-chunk, both passes read the same scores; with more,
+// pass 1 runs over all super-chunks first and pass 2 issues their products
+// again (the products are ~2 % of the kernel's time; TMEM for all scores
+// would leave room for fewer CTAs). Lists of more than 32 entries skip pass 1.
 template <int KP>
-__global__ void __launch_bounds__(kGateTcThreads)
+__global__ void __launch_bounds__(kGateTcThreads, GateCfg<KP>::kMinCtas)
     gate_tc_kernel(const __grid_constant__ CUtensorMap tm_hi, const __grid_constant__ CUtensorMap tm_lo,
                    const __grid_constant__ CUtensorMap tm_q, GateParams p) {
+  using Cfg = GateCfg<KP>;
+  constexpr int kChunk = Cfg::kChunk;
+  constexpr int NG = Cfg::kGroups;
   grid_dependency_sync();
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sQ = smem;
-  uint8_t* sM = smem + kGateQBytes;  // 2 stages x (hi, lo); stage 0 doubles as the score staging area
-  __shared__ uint64_t full_bar[2], mma_bar[2], sc_bar, drain_bar, q_bar;
+  uint8_t* sM = smem + kGateQBytes;  // the means stage (hi, lo); doubles as the score staging area
+  __shared__ uint64_t full_bar, mma_bar, sc_bar, drain_bar, q_bar;
   __shared__ uint32_t tmem_base;
   __shared__ int abort_flag;
 
@@ -155,7 +221,7 @@ __global__ void __launch_bounds__(kGateTcThreads)
   int64_t t_last = t_cta + udiv32(rem0 + 127u, G);
   if (t_last > p.S - 1) t_last = p.S - 1;
   const int b_cta = (int)udiv32((uint32_t)t_last, (uint32_t)p.B);  // past blocks of this CTA: j < b_cta
-  const int nchunks = (b_cta + kGateBlkChunk - 1) / kGateBlkChunk;
+  const int nchunks = (b_cta + kChunk - 1) / kChunk;
 
   float tv[KP];
   int ti[KP];
@@ -166,12 +232,11 @@ __global__ void __launch_bounds__(kGateTcThreads)
   }
 
   if (nchunks > 0) {
-    const uint32_t ncols = nchunks >= 3 ? 256u : (nchunks == 2 ? 128u : 64u);
+    uint32_t ncols = 32;  // a power of two >= 32 covering one super-chunk
+    while ((int)ncols < min(nchunks, Cfg::kScChunks) * kChunk) ncols <<= 1;
     if (threadIdx.x == 0) {
-      for (int i = 0; i < 2; ++i) {
-        mbar_init(&full_bar[i], 1);
-        mbar_init(&mma_bar[i], 1);
-      }
+      mbar_init(&full_bar, 1);
+      mbar_init(&mma_bar, 1);
       mbar_init(&sc_bar, 1);
       mbar_init(&drain_bar, 1);
       mbar_init(&q_bar, 1);
@@ -179,19 +244,24 @@ __global__ void __launch_bounds__(kGateTcThreads)
       fence_barrier_init();
     }
     const int row0 = g * p.nbp_pad;  // first mean row of this kv head
-    auto load_chunk = [&](int c) {  // one lane of warp 0
-      const int st = c & 1;
-      uint8_t* dst = sM + st * 2 * kGateSplitBytes;
-      mbar_arrive_expect_tx(&full_bar[st], 2 * kGateSplitBytes);
-      const int r0 = row0 + c * kGateBlkChunk;
-      tma_load_2d(dst, &tm_hi, &full_bar[st], 0, r0);
-      tma_load_2d(dst + kGateSplitHalf, &tm_hi, &full_bar[st], 64, r0);
-      tma_load_2d(dst + kGateSplitBytes, &tm_lo, &full_bar[st], 0, r0);
-      tma_load_2d(dst + kGateSplitBytes + kGateSplitHalf, &tm_lo, &full_bar[st], 64, r0);
+    // one lane of warp 0: the k-th chunk asked for completes phase k of
+    // full_bar (chunks come in the order they are used)
+    auto load_chunk = [&](int c) {
+      mbar_arrive_expect_tx(&full_bar, 2 * Cfg::kSplitBytes);
+      const int r0 = row0 + c * kChunk;
+#pragma unroll
+      for (int part = 0; part < 2; ++part) {
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+#pragma unroll
+          for (int bx = 0; bx < kChunk / kGateBoxRows; ++bx)
+            tma_load_2d(sM + part * Cfg::kSplitBytes + half * Cfg::kSplitHalf + bx * kGateBoxRows * 128,
+                        part ? &tm_lo : &tm_hi, &full_bar, half * 64, r0 + bx * kGateBoxRows);
+        }
+      }
     };
-    // the first two chunks of means do not depend on Q: their copies run
-    // while the Q rows are gathered (the thread that initialised the
-    // barriers issues them)
+    // the first chunk of means does not depend on Q: its copy runs while the
+    // Q rows come in (the thread that initialised the barriers issues it)
     if (threadIdx.x == 0) {
       if (p.q_tma) {
         // the CTA's 128 group-rows are 128 / G whole tokens x G heads: one
@@ -203,7 +273,6 @@ __global__ void __launch_bounds__(kGateTcThreads)
         tma_load_3d(sQ + kGateQBytes / 2, &tm_q, &q_bar, 64, g * p.G, tok);
       }
       load_chunk(0);
-      if (nchunks > 1) load_chunk(1);
     }
     if (warp == 0) {
       __syncwarp();
@@ -243,120 +312,137 @@ __global__ void __launch_bounds__(kGateTcThreads)
       __syncwarp();
     }
     const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
-    const uint32_t idesc = idesc_bf16_f32(128, kGateBlkChunk, false);
+    const uint32_t idesc = idesc_bf16_f32(128, kChunk, false);
     const uint64_t dQ = sdesc_sw128(smem_u32(sQ), 16, 1024);
     const uint64_t dM = sdesc_sw128(smem_u32(sM), 16, 1024);
     volatile int* ab = &abort_flag;
-    int loaded = min(nchunks, 2);  // chunks asked of TMA so far
+    int loaded = 1;          // chunks asked of TMA so far
+    int seq = 0;             // chunks whose products were issued (warp 0): phases of full_bar, mma_bar
+    bool prefetched = false;  // warp 0: the next phase's first chunk is already on its way
     // staging of one 32-column piece of scores per row (for the insertions,
-    // which index columns per lane): 128 B per row in ring stage 0, 16-byte
+    // which index columns per lane): 128 B per row in the means stage, 16-byte
     // pieces swizzled by row so that 8 consecutive rows hit distinct banks
     float* stg = reinterpret_cast<float*>(sM) + row * 32;
-    const int nsc = (nchunks + 3) / 4;
-    for (int sc = 0; sc < nsc; ++sc) {
+    const int nsc = (nchunks + Cfg::kScChunks - 1) / Cfg::kScChunks;
+    // phases: pass 1 over the super-chunks, then pass 2 over them again; one
+    // super-chunk (or no bound): the passes share each phase's scores
+    const bool two_pass = Cfg::kBound && nsc > 1;
+    const int nphase = two_pass ? 2 * nsc : nsc;
+    float gm[NG];
+#pragma unroll
+    for (int i = 0; i < NG; ++i) gm[i] = -INFINITY;
+    float tau = -INFINITY;
+    for (int ph = 0; ph < nphase; ++ph) {
       if (*ab) break;
-      const int c_lo = 4 * sc;
-      const int nc = min(4, nchunks - c_lo);
+      const int sc = ph < nsc ? ph : ph - nsc;
+      const bool pass1_only = two_pass && ph < nsc;           // group maxima, no insertions
+      const bool maxima = Cfg::kBound && (pass1_only || !two_pass);
+      const int c_lo = Cfg::kScChunks * sc;
+      const int nc = min(Cfg::kScChunks, nchunks - c_lo);
       if (warp == 0) {
-        // scores of this super-chunk: chunk c_lo + c into TMEM columns 64c
-        // (the first super-chunk's first two chunks are already on their way)
-        if (sc > 0) {
-          if (elect_one()) {
-            load_chunk(c_lo);
-            if (nc > 1) load_chunk(c_lo + 1);
-          }
+        // scores of this super-chunk: chunk c_lo + c into TMEM columns
+        // c * kChunk (the first phase's first chunk is already on its way)
+        if (ph > 0 && !prefetched) {
+          if (elect_one()) load_chunk(c_lo);
           __syncwarp();
-          loaded = c_lo + min(nc, 2);
+          ++loaded;
         }
-        for (int c = 0; c < nc; ++c) {
-          const int gc = c_lo + c, st = gc & 1;
-          if (!mbar_wait(&full_bar[st], (gc >> 1) & 1, ab)) break;
+        prefetched = false;
+        for (int c = 0; c < nc; ++c, ++seq) {
+          if (!mbar_wait(&full_bar, seq & 1, ab)) break;
           tc_fence_after();
           if (elect_one()) {
-            const uint64_t m0 = dM + ((st * 2 * kGateSplitBytes) >> 4);
 #pragma unroll
             for (int part = 0; part < 2; ++part) {
 #pragma unroll
               for (int kk = 0; kk < 8; ++kk) {
                 const uint32_t qoff = ((kk >> 2) * (kGateQBytes / 2) + (kk & 3) * 32) >> 4;
-                const uint32_t moff = (part * kGateSplitBytes + (kk >> 2) * kGateSplitHalf + (kk & 3) * 32) >> 4;
-                mma_bf16_ss(tmem + c * kGateBlkChunk, dQ + qoff, m0 + moff, idesc, (part > 0 || kk > 0) ? 1u : 0u);
+                const uint32_t moff = (part * Cfg::kSplitBytes + (kk >> 2) * Cfg::kSplitHalf + (kk & 3) * 32) >> 4;
+                mma_bf16_ss(tmem + c * kChunk, dQ + qoff, dM + moff, idesc, (part > 0 || kk > 0) ? 1u : 0u);
               }
             }
-            mma_commit(&mma_bar[st]);
+            mma_commit(&mma_bar);
           }
           __syncwarp();
-          if (c + 2 < nc) {
+          const bool more = c + 1 < nc;
+          // a pass-1 phase stages no scores: the next phase's first chunk can
+          // come in while the rows take their maxima
+          const bool ahead = !more && pass1_only;
+          if (more || ahead) {
             // the stage is free once this chunk's products have read it
-            if (!mbar_wait(&mma_bar[st], (gc >> 1) & 1, ab)) break;
-            if (elect_one()) load_chunk(gc + 2);
+            if (!mbar_wait(&mma_bar, seq & 1, ab)) break;
+            const int next = more ? c_lo + c + 1 : (ph + 1 < nsc ? c_lo + nc : 0);
+            if (elect_one()) load_chunk(next);
             __syncwarp();
-            loaded = gc + 3;
+            ++loaded;
+            prefetched = ahead;
           }
         }
         if (elect_one()) mma_commit(&sc_bar);
         __syncwarp();
       }
-      if (*ab || !mbar_wait(&sc_bar, sc & 1, ab)) break;
+      if (*ab || !mbar_wait(&sc_bar, ph & 1, ab)) break;
       __syncwarp();
       tc_fence_after();
-      // ---- selection over this super-chunk's columns [0, 64 nc)
-      const int jb = sc * 4 * kGateBlkChunk;                 // block of column 0
-      const int jn = max(0, min(nc * kGateBlkChunk, bt - jb));  // this row's past blocks here
-      float tau = -INFINITY;
-      // the group-maximum bound pays only while some row's list is not yet
-      // full; after that the rows' running KP-th best filters the columns
-      if (KP <= 24 && __any_sync(0xffffffffu, tv[KP - 1] == -INFINITY)) {
-        constexpr int NG = KP <= 24 ? KP : 1;
-        float gm[NG];
+      // ---- selection over this super-chunk's columns [0, nc * kChunk)
+      const int jb = sc * kGateScCols;                   // block of column 0
+      const int jn = max(0, min(nc * kChunk, bt - jb));  // this row's past blocks here
+      if (maxima) {
+        // pass 1: group maxima (column c of a super-chunk is in group c mod NG)
 #pragma unroll
-        for (int i = 0; i < NG; ++i) gm[i] = -INFINITY;
-#pragma unroll
-        for (int pc = 0; pc < 8; ++pc) {
-          if (pc < 2 * nc) {
+        for (int pc = 0; pc < kGatePieces; ++pc) {
+          if (pc * 32 < nc * kChunk) {
             uint32_t r[32];
             tmem_ld32(tmem + pc * 32 + lane_off, r);
             tmem_ld_wait();
+            const int rem = jn - pc * 32;  // columns of this piece that are the row's past blocks
+            if (rem >= 32) {
 #pragma unroll
-            for (int e = 0; e < 32; ++e) {
-              const int col = pc * 32 + e;
-              const float v = col < jn ? __uint_as_float(r[e]) : -INFINITY;
-              gm[col % NG] = fmaxf(gm[col % NG], v);
+              for (int e = 0; e < 32; ++e) gm[e % NG] = fmaxf(gm[e % NG], __uint_as_float(r[e]));
+            } else {
+#pragma unroll
+              for (int e = 0; e < 32; ++e) gm[e % NG] = fmaxf(gm[e % NG], e < rem ? __uint_as_float(r[e]) : -INFINITY);
             }
           }
         }
-        if (jn >= NG) {
-          tau = gm[0];
-#pragma unroll
-          for (int i = 1; i < NG; ++i) tau = fminf(tau, gm[i]);
+        if (!two_pass || ph == nsc - 1) {
+          // every maximum is in: tau = the KP-th largest (-inf while fewer
+          // than KP groups hold a past block)
+          sort_desc<NG>(gm);
+          tau = gm[KP - 1];
         }
       }
+      if (!pass1_only) {
+        // pass 2: the candidates of this super-chunk into the row's list
 #pragma unroll
-      for (int pc = 0; pc < 8; ++pc) {
-        if (pc < 2 * nc) {
-          uint32_t r[32];
-          tmem_ld32(tmem + pc * 32 + lane_off, r);
-          tmem_ld_wait();
-          const float thr = tv[KP - 1];
-          uint32_t cand = 0;
+        for (int pc = 0; pc < kGatePieces; ++pc) {
+          if (pc * 32 < nc * kChunk) {
+            uint32_t r[32];
+            tmem_ld32(tmem + pc * 32 + lane_off, r);
+            tmem_ld_wait();
+            // a column is a candidate when it is one of the row's past blocks,
+            // reaches tau and beats the row's KP-th best; the last two tests
+            // are one: v >= max(tau, the float just above the KP-th best)
+            const float lo = fmaxf(tau, float_above(tv[KP - 1]));
+            uint32_t cand = 0;
 #pragma unroll
-          for (int e = 0; e < 32; ++e) {
-            const float v = __uint_as_float(r[e]);
-            if (pc * 32 + e < jn && v >= tau && v > thr) cand |= 1u << e;
-          }
-          if (__any_sync(0xffffffffu, cand != 0u)) {
+            for (int e = 0; e < 32; ++e) cand |= (__uint_as_float(r[e]) >= lo) ? (1u << e) : 0u;
+            const int rem = jn - pc * 32;
+            cand &= rem >= 32 ? 0xffffffffu : (rem > 0 ? (1u << rem) - 1u : 0u);
+            if (__any_sync(0xffffffffu, cand != 0u)) {
 #pragma unroll
-            for (int k4 = 0; k4 < 8; ++k4)
-              *reinterpret_cast<uint4*>(stg + ((k4 ^ (row & 7)) << 2)) =
-                  make_uint4(r[4 * k4], r[4 * k4 + 1], r[4 * k4 + 2], r[4 * k4 + 3]);
-            __syncwarp();
-            while (cand) {
-              const int e = __ffs(cand) - 1;
-              cand &= cand - 1;
-              const float sv = stg[(((e >> 2) ^ (row & 7)) << 2) | (e & 3)];
-              if (sv > tv[KP - 1]) gate_insert<KP>(tv, ti, sv, jb + pc * 32 + e);
+              for (int k4 = 0; k4 < 8; ++k4)
+                *reinterpret_cast<uint4*>(stg + ((k4 ^ (row & 7)) << 2)) =
+                    make_uint4(r[4 * k4], r[4 * k4 + 1], r[4 * k4 + 2], r[4 * k4 + 3]);
+              __syncwarp();
+              while (cand) {
+                const int e = __ffs(cand) - 1;
+                cand &= cand - 1;
+                const float sv = stg[(((e >> 2) ^ (row & 7)) << 2) | (e & 3)];
+                if (sv > tv[KP - 1]) gate_insert<KP>(tv, ti, sv, jb + pc * 32 + e);
+              }
+              __syncwarp();
             }
-            __syncwarp();
           }
         }
       }
@@ -373,7 +459,9 @@ __global__ void __launch_bounds__(kGateTcThreads)
       volatile int keep_waiting = 0;
       if (warp == 0) {
         if (elect_one()) {
-          for (int c = 0; c < loaded; ++c) mbar_wait(&full_bar[c & 1], (c >> 1) & 1, &keep_waiting, (1ull << 28));
+          // one stage: at most one copy of means is in flight, the last one
+          // asked for, and only if its products were never issued
+          if (seq < loaded) mbar_wait(&full_bar, (loaded - 1) & 1, &keep_waiting, (1ull << 28));
           if (p.q_tma) mbar_wait(&q_bar, 0, &keep_waiting, (1ull << 28));
         }
         __syncwarp();

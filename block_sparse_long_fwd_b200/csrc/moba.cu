@@ -52,6 +52,14 @@ struct DeviceInfo {
 
 std::mutex g_dev_mu;
 DeviceInfo g_dev[64];
+
+// The gate kernel for lists of KP entries takes GateCfg<KP>::kSmemBytes of
+// dynamic shared memory.
+template <int KP>
+cudaError_t set_gate_smem() {
+  return cudaFuncSetAttribute(moba::gate_tc_kernel<KP>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              moba::GateCfg<KP>::kSmemBytes);
+}
 PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
 
 int device_info(DeviceInfo* out) {
@@ -73,24 +81,16 @@ int device_info(DeviceInfo* out) {
                                      moba::kDqSmemBytes));
       MOBA_CUDA(cudaFuncSetAttribute(moba::bwd_dkdv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      moba::kBwdSmemBytes));
-      MOBA_CUDA(cudaFuncSetAttribute(moba::gate_tc_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                     moba::kGateSmemBytes));
-      MOBA_CUDA(cudaFuncSetAttribute(moba::gate_tc_kernel<4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                     moba::kGateSmemBytes));
-      MOBA_CUDA(cudaFuncSetAttribute(moba::gate_tc_kernel<8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                     moba::kGateSmemBytes));
-      MOBA_CUDA(cudaFuncSetAttribute(moba::gate_tc_kernel<12>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                     moba::kGateSmemBytes));
-      MOBA_CUDA(cudaFuncSetAttribute(moba::gate_tc_kernel<16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                     moba::kGateSmemBytes));
-      MOBA_CUDA(cudaFuncSetAttribute(moba::gate_tc_kernel<24>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                     moba::kGateSmemBytes));
-      MOBA_CUDA(cudaFuncSetAttribute(moba::gate_tc_kernel<48>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                     moba::kGateSmemBytes));
-      MOBA_CUDA(cudaFuncSetAttribute(moba::gate_tc_kernel<32>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                     moba::kGateSmemBytes));
-      MOBA_CUDA(cudaFuncSetAttribute(moba::gate_tc_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                     moba::kGateSmemBytes));
+      MOBA_CUDA(set_gate_smem<2>());
+      MOBA_CUDA(set_gate_smem<4>());
+      MOBA_CUDA(set_gate_smem<8>());
+      MOBA_CUDA(set_gate_smem<11>());
+      MOBA_CUDA(set_gate_smem<12>());
+      MOBA_CUDA(set_gate_smem<16>());
+      MOBA_CUDA(set_gate_smem<24>());
+      MOBA_CUDA(set_gate_smem<32>());
+      MOBA_CUDA(set_gate_smem<48>());
+      MOBA_CUDA(set_gate_smem<64>());
       // host-mapped copy of the status word (kernels store an error code
       // there too, so a later call sees it without a device read)
       int* h = nullptr;
@@ -328,7 +328,7 @@ int make_plan(Plan* pl, int64_t S, int64_t q0, int Hq, int Hkv, int B, int topk,
 int make_mean_map(CUtensorMap* map, const void* base, int64_t rows) {
   cuuint64_t dims[2] = {(cuuint64_t)moba::kHeadDim, (cuuint64_t)rows};
   cuuint64_t strides[1] = {(cuuint64_t)moba::kHeadDim * 2};
-  cuuint32_t box[2] = {64, (cuuint32_t)moba::kGateBlkChunk};
+  cuuint32_t box[2] = {64, (cuuint32_t)moba::kGateBoxRows};
   cuuint32_t estr[2] = {1, 1};
   CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -360,8 +360,8 @@ template <int KP>
 void launch_gate_tc(const Plan& p, const CUtensorMap& mhi, const CUtensorMap& mlo, const CUtensorMap& mq,
                     const moba::GateParams& gp, cudaStream_t st) {
   dim3 grid((unsigned)(((p.S - p.q0) * p.G + 127) / 128), p.Hkv);
-  launch_chained(moba::gate_tc_kernel<KP>, grid, dim3(moba::kGateTcThreads), moba::kGateSmemBytes, st, mhi, mlo, mq,
-                 gp);
+  launch_chained(moba::gate_tc_kernel<KP>, grid, dim3(moba::kGateTcThreads), moba::GateCfg<KP>::kSmemBytes, st, mhi,
+                 mlo, mq, gp);
 }
 
 // q [S - q0][Hq][128] bf16 as 3-D (channel, head, token) for the gate's Q
@@ -421,6 +421,7 @@ int launch_gate(const Plan& p, const void* q, const float* kmean, int splits, __
   if (p.P <= 2) launch_gate_tc<2>(p, mhi, mlo, mq, gp, st);
   else if (p.P <= 4) launch_gate_tc<4>(p, mhi, mlo, mq, gp, st);
   else if (p.P <= 8) launch_gate_tc<8>(p, mhi, mlo, mq, gp, st);
+  else if (p.P == 11) launch_gate_tc<11>(p, mhi, mlo, mq, gp, st);  // top-12: a list of exactly k - 1
   else if (p.P <= 12) launch_gate_tc<12>(p, mhi, mlo, mq, gp, st);
   else if (p.P <= 16) launch_gate_tc<16>(p, mhi, mlo, mq, gp, st);
   else if (p.P <= 24) launch_gate_tc<24>(p, mhi, mlo, mq, gp, st);
@@ -515,7 +516,7 @@ bool window_routed(const Plan& p, const moba::WindowGeom& wg) {
 }
 
 // The router for one query window (flags, counts, scan, fill); returns the
-// number of kernels launched.
+// number of kernels launched, or -status.
 int launch_route(const Plan& p, const moba::WindowGeom& wg, bool routed, uint8_t* ws, cudaStream_t st) {
   const int32_t* sel = reinterpret_cast<const int32_t*>(ws + p.o_sel);
   uint32_t* flags = reinterpret_cast<uint32_t*>(ws + p.o_flags);
@@ -530,6 +531,9 @@ int launch_route(const Plan& p, const moba::WindowGeom& wg, bool routed, uint8_t
   int n = 0;
   if (routed) {
     dim3 gf((unsigned)((wg.wwords + 7) / 8), p.Hkv);
+    // the flags kernel writes only the words of picked blocks
+    if (cudaMemsetAsync(flags, 0, (size_t)nbk * (size_t)wg.wwords * sizeof(uint32_t), st) != cudaSuccess)
+      return -fail(MOBA_ERR_CUDA, "cudaMemsetAsync (route flags) failed");
     launch_chained(moba::route_flags_kernel, gf, dim3(256), 0, st, sel, wg, flags);
     dim3 gb(p.nbp, p.Hkv);
     launch_chained(moba::route_count_kernel, gb, dim3(256), 0, st, static_cast<const uint32_t*>(flags), wg, cnt);
@@ -605,7 +609,9 @@ int run_forward(const Plan& p, const DeviceInfo& dev, const void* q, const void*
   for (int64_t w0 = p.wbase; w0 < p.S; w0 += p.W) {
     const moba::WindowGeom wg = window_geom(p, w0);
     const bool routed = window_routed(p, wg);
-    tm->count(launch_route(p, wg, routed, ws, st));
+    const int nr = launch_route(p, wg, routed, ws, st);
+    if (nr < 0) return -nr;
+    tm->count(nr);
     tm->mark(kRoute);
     ap.w0 = w0;
     ap.wlen = wg.wlen;
@@ -742,7 +748,9 @@ int run_backward(const Plan& p, const BwdLayout& bl, const DeviceInfo& dev, cons
   for (int64_t w0 = 0; w0 < p.S; w0 += p.W) {
     const moba::WindowGeom wg = window_geom(p, w0);
     const bool routed = window_routed(p, wg);
-    tm->count(launch_route(p, wg, routed, ws, st));
+    const int nr = launch_route(p, wg, routed, ws, st);
+    if (nr < 0) return -nr;
+    tm->count(nr);
     tm->mark(kRoute);
     ap.w0 = w0;
     ap.wlen = wg.wlen;

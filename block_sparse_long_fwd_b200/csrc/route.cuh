@@ -10,7 +10,8 @@
 // Rows are processed in query windows [w0, w0 + wlen). Within a window, a
 // group-row is rr = (t - w0) * G + hl for query t and head h = g*G + hl.
 // 1. flags: bit rr%32 of word flags[g][j][rr/32] is set when row rr routes
-//    to block j (past blocks only; the own block goes to the diagonal pass).
+//    to block j (past blocks only; the own block goes to the diagonal pass);
+//    the words are cleared first, and only the blocks picked are written.
 // 2. count: popcount per bucket.
 // 3. scan (one CTA): exclusive offsets of the lists and of their 128-row
 //    tiles, plus the own-block tiles of the window, longest first.
@@ -52,7 +53,11 @@ __device__ __forceinline__ int64_t bucket_word_begin(const WindowGeom& w, int j)
   return wb < w.wwords ? wb : w.wwords;
 }
 
-// 1. grid (ceil(wwords / 8), Hkv), 256 threads: one warp per flag word.
+// 1. grid (ceil(wwords / 8), Hkv), 256 threads: one warp per flag word (32
+// group-rows). The flag words start zeroed (the host clears them), so only
+// the blocks some row of the word picked are visited: each step takes the
+// smallest block still pending in any lane, and the lanes that picked it
+// advance to their next entry (a row's past entries are ascending).
 __global__ void __launch_bounds__(256) route_flags_kernel(const int32_t* __restrict__ sel, WindowGeom w,
                                                           uint32_t* __restrict__ flags) {
   grid_dependency_sync();
@@ -63,14 +68,9 @@ __global__ void __launch_bounds__(256) route_flags_kernel(const int32_t* __restr
   const int64_t rr = word * 32 + lane;
   const int64_t tl = rr / w.G;
   const int64_t t = w.w0 + tl;
-  const bool in_window = tl < w.wlen;
-  const bool valid = in_window && t >= w.q0;  // a token before q0 has no query: no bits
+  const bool valid = tl < w.wlen && t >= w.q0;  // a token before q0 has no query: no bits
   const int h = g * w.G + (int)(rr % w.G);
-  // every word writes its bits for all blocks below its rows' own blocks
-  // (zeros for rows without a query), since the count and fill kernels read
-  // every word from the first one that can hold a bit of the block
-  const int bt = in_window ? (int)(t / w.B) : 0;
-  const int bmax = __reduce_max_sync(0xffffffffu, bt);
+  const int bt = valid ? (int)(t / w.B) : 0;
   const int P = w.k_eff - 1;
   const int32_t* srow = sel + ((int64_t)h * (w.S - w.q0) + (valid ? t - w.q0 : 0)) * w.k_eff;
   int ptr = 0;
@@ -81,7 +81,9 @@ __global__ void __launch_bounds__(256) route_flags_kernel(const int32_t* __restr
   };
   int cur = entry(0);
   uint32_t* dst = flags + (int64_t)g * w.nbp * w.wwords + word;
-  for (int j = 0; j < bmax; ++j) {
+  for (;;) {
+    const int j = __reduce_min_sync(0xffffffffu, cur);
+    if (j == 0x7fffffff) break;
     const bool hit = (cur == j);
     if (hit) cur = entry(++ptr);
     const uint32_t bits = __ballot_sync(0xffffffffu, hit);

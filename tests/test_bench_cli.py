@@ -38,6 +38,8 @@ def test_chunk_flops_of_the_whole_sequence_match_the_library_count():
     ["--warmup", "2"],
     ["--cached-means"],
     ["--chunk", "-1"],
+    ["--heads", "6:4"],
+    ["--heads", "x"],
 ])
 def test_incompatible_modes_are_rejected_before_any_gpu_work(args):
     r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py")] + args, capture_output=True, text=True,
