@@ -62,13 +62,13 @@ __host__ __device__ inline int gate_rows_padded(int nbp) {
 
 // Block means -> hi, lo bf16 [Hkv][nbp_pad][128]; padding rows are zero.
 // part holds `splits` partial means per block, [Hkv][nbp][splits][128],
-// added in order (one split: part is the mean itself). grid (nbp_pad, Hkv),
-// 128 threads.
+// added in order (one split: part is the mean itself). grid (rows, Hkv),
+// 128 threads: rows j0 .. j0 + gridDim.x - 1.
 __global__ void __launch_bounds__(128) kmean_split_kernel(const float* __restrict__ part, int splits, int nbp,
-                                                          int nbp_pad, __nv_bfloat16* __restrict__ hi,
+                                                          int nbp_pad, int j0, __nv_bfloat16* __restrict__ hi,
                                                           __nv_bfloat16* __restrict__ lo) {
   grid_dependency_sync();
-  const int j = blockIdx.x, g = blockIdx.y, c = threadIdx.x;
+  const int j = j0 + (int)blockIdx.x, g = blockIdx.y, c = threadIdx.x;
   const int64_t o = ((int64_t)g * nbp_pad + j) * kHeadDim + c;
   if (j < nbp) {
     const float* src = part + ((int64_t)g * nbp + j) * splits * kHeadDim + c;
@@ -87,6 +87,7 @@ struct GateParams {
   const __nv_bfloat16* q;  // [S - q0][Hq][128]: the tokens with a query
   int32_t* sel;            // [Hq][S - q0][k_eff]
   int64_t S, q0;           // q0: first token with a query
+  int64_t t_begin, t_end;  // the rows of tokens [t_begin, t_end) (q0 <= t_begin < t_end <= S)
   int Hq, G, B, nbp_pad, k_eff;
   int q_tma;               // 1: G divides 128 and tm_q is valid (Q tiles by TMA)
 };
@@ -164,8 +165,8 @@ __device__ __forceinline__ void gate_write_row(int32_t* out, const int (&ti)[KP]
   for (int i = npast + 1; i < k_eff; ++i) out[i] = -1;
 }
 
-// grid (ceil((S - q0)*G / 128), Hkv), 128 threads; row = TMEM lane = group-row
-// blockIdx.x*128 + threadIdx.x.
+// grid (ceil((t_end - t_begin)*G / 128), Hkv), 128 threads; row = TMEM lane =
+// group-row (t_begin - q0)*G + blockIdx.x*128 + threadIdx.x.
 //
 // The CTA's past blocks are scored in super-chunks of kGateScCols columns:
 // warp 0 streams each chunk's hi/lo means through the one means stage and
@@ -207,7 +208,7 @@ __global__ void __launch_bounds__(kGateTcThreads, GateCfg<KP>::kMinCtas)
   const int row = threadIdx.x;
   // group-row rr = t * G + hl; this CTA's rows start at rr0 = t_cta * G + rem0
   const uint32_t G = (uint32_t)p.G;
-  const int64_t bxr = (int64_t)blockIdx.x * 128;
+  const int64_t bxr = (p.t_begin - p.q0) * p.G + (int64_t)blockIdx.x * 128;
   const int64_t t_cta_off = bxr / p.G;  // the one 64-bit division of a thread
   const uint32_t rem0 = (uint32_t)(bxr - t_cta_off * p.G);
   const int64_t t_cta = p.q0 + t_cta_off;  // first token of this CTA's group-rows
@@ -215,11 +216,11 @@ __global__ void __launch_bounds__(kGateTcThreads, GateCfg<KP>::kMinCtas)
   const uint32_t tr = udiv32(xr, G);
   const int64_t t = t_cta + tr;
   const int h = g * p.G + (int)(xr - tr * G);
-  const bool valid = t < p.S;
+  const bool valid = t < p.t_end;
   const int bt = valid ? (int)udiv32((uint32_t)t, (uint32_t)p.B) : 0;
   const int P = p.k_eff - 1;
   int64_t t_last = t_cta + udiv32(rem0 + 127u, G);
-  if (t_last > p.S - 1) t_last = p.S - 1;
+  if (t_last > p.t_end - 1) t_last = p.t_end - 1;
   const int b_cta = (int)udiv32((uint32_t)t_last, (uint32_t)p.B);  // past blocks of this CTA: j < b_cta
   const int nchunks = (b_cta + kChunk - 1) / kChunk;
 
@@ -292,7 +293,7 @@ __global__ void __launch_bounds__(kGateTcThreads, GateCfg<KP>::kMinCtas)
         const int64_t t_r = t_cta + dt;
         const __nv_bfloat16* src = p.q;
         uint32_t bytes = 0;
-        if (t_r < p.S) {
+        if (t_r < p.t_end) {
           src = p.q + ((t_r - p.q0) * p.Hq + g * p.G + (int)(x - dt * G)) * kHeadDim + c16 * 8;
           bytes = 16;
         }

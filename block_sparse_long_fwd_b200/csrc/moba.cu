@@ -323,8 +323,8 @@ int make_plan(Plan* pl, int64_t S, int64_t q0, int Hq, int Hkv, int B, int topk,
   return MOBA_OK;
 }
 
-// Block-mean rows as a 2-D tensor [Hkv * nbp_pad][128] bf16; box 64 x 64,
-// 128-byte swizzle (one 64-channel half of a 64-block chunk per load).
+// Block-mean rows as a 2-D tensor [Hkv * nbp_pad][128] bf16; box 64 x 32,
+// 128-byte swizzle (one 64-channel half of 32 blocks per load).
 int make_mean_map(CUtensorMap* map, const void* base, int64_t rows) {
   cuuint64_t dims[2] = {(cuuint64_t)moba::kHeadDim, (cuuint64_t)rows};
   cuuint64_t strides[1] = {(cuuint64_t)moba::kHeadDim * 2};
@@ -359,7 +359,7 @@ void launch_chained(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem
 template <int KP>
 void launch_gate_tc(const Plan& p, const CUtensorMap& mhi, const CUtensorMap& mlo, const CUtensorMap& mq,
                     const moba::GateParams& gp, cudaStream_t st) {
-  dim3 grid((unsigned)(((p.S - p.q0) * p.G + 127) / 128), p.Hkv);
+  dim3 grid((unsigned)(((gp.t_end - gp.t_begin) * p.G + 127) / 128), p.Hkv);
   launch_chained(moba::gate_tc_kernel<KP>, grid, dim3(moba::kGateTcThreads), moba::GateCfg<KP>::kSmemBytes, st, mhi,
                  mlo, mq, gp);
 }
@@ -379,21 +379,33 @@ int make_gate_q_map(CUtensorMap* map, const void* q, int64_t ntok, int Hq, int G
   return MOBA_OK;
 }
 
-// Gate + top-k into sel. kmean (fp32) is split into khi/klo (bf16, padded
-// rows) first. Rows that need no scores (topk 1, or every past block) are
-// written directly. Returns the number of kernels launched, or -status.
-int launch_gate(const Plan& p, const void* q, const float* kmean, int splits, __nv_bfloat16* khi,
-                __nv_bfloat16* klo, int32_t* sel, cudaStream_t st) {
-  const bool full = p.k_eff == p.nb;
-  if (p.P == 0 || full || p.nbp <= 0) {
-    const int64_t n = (p.S - p.q0) * p.Hq;
-    launch_chained(moba::sel_fill_kernel, dim3((unsigned)((n + 255) / 256)), dim3(256), 0, st, sel, p.S, p.q0, p.Hq,
-                   p.B, p.k_eff, full ? 1 : 0);
-    return 1;
-  }
+// Rows that need no scores (topk 1, or every past block): sel written
+// directly, no inputs read.
+bool gate_free(const Plan& p) { return p.P == 0 || p.k_eff == p.nb || p.nbp <= 0; }
+
+void launch_sel_fill(const Plan& p, int32_t* sel, cudaStream_t st) {
+  const int64_t n = (p.S - p.q0) * p.Hq;
+  launch_chained(moba::sel_fill_kernel, dim3((unsigned)((n + 255) / 256)), dim3(256), 0, st, sel, p.S, p.q0, p.Hq, p.B,
+                 p.k_eff, p.k_eff == p.nb ? 1 : 0);
+}
+
+// Block means [j0, j1) (fp32, `splits` partial sums each) into the padded
+// bf16 hi/lo rows the gate reads; the range ending at nbp also writes the
+// zero padding rows up to the chunk multiple.
+void launch_mean_split(const Plan& p, const float* kmean, int splits, __nv_bfloat16* khi, __nv_bfloat16* klo, int j0,
+                       int j1, cudaStream_t st) {
   const int nbp_pad = moba::gate_rows_padded(p.nbp);
-  launch_chained(moba::kmean_split_kernel, dim3(nbp_pad, p.Hkv), dim3(128), 0, st, kmean, splits, p.nbp, nbp_pad, khi,
-                 klo);
+  if (j1 >= p.nbp) j1 = nbp_pad;
+  if (j1 <= j0) return;
+  launch_chained(moba::kmean_split_kernel, dim3(j1 - j0, p.Hkv), dim3(128), 0, st, kmean, splits, p.nbp, nbp_pad, j0,
+                 khi, klo);
+}
+
+// The gate's scores and top-k for the rows of tokens [t_begin, t_end), from
+// the hi/lo block means. Returns -status on failure, else 0.
+int launch_gate_rows(const Plan& p, const void* q, const __nv_bfloat16* khi, const __nv_bfloat16* klo, int32_t* sel,
+                     int64_t t_begin, int64_t t_end, cudaStream_t st) {
+  const int nbp_pad = moba::gate_rows_padded(p.nbp);
   CUtensorMap mhi, mlo;
   int rc = make_mean_map(&mhi, khi, (int64_t)p.Hkv * nbp_pad);
   if (rc) return -rc;
@@ -413,6 +425,8 @@ int launch_gate(const Plan& p, const void* q, const float* kmean, int splits, __
   gp.sel = sel;
   gp.S = p.S;
   gp.q0 = p.q0;
+  gp.t_begin = t_begin;
+  gp.t_end = t_end;
   gp.Hq = p.Hq;
   gp.G = p.G;
   gp.B = p.B;
@@ -428,14 +442,30 @@ int launch_gate(const Plan& p, const void* q, const float* kmean, int splits, __
   else if (p.P <= 32) launch_gate_tc<32>(p, mhi, mlo, mq, gp, st);
   else if (p.P <= 48) launch_gate_tc<48>(p, mhi, mlo, mq, gp, st);
   else launch_gate_tc<64>(p, mhi, mlo, mq, gp, st);
-  return 2;
+  return 0;
 }
 
-void launch_pool(const Plan& p, const void* k, float* kmean, int splits, cudaStream_t st) {
-  if (p.nbp <= 0) return;
-  dim3 grid(p.nbp, p.Hkv, splits);
+// Gate + top-k into sel for every row. kmean (fp32) is split into khi/klo
+// (bf16, padded rows) first. Returns the number of kernels launched, or
+// -status.
+int launch_gate(const Plan& p, const void* q, const float* kmean, int splits, __nv_bfloat16* khi,
+                __nv_bfloat16* klo, int32_t* sel, cudaStream_t st) {
+  if (gate_free(p)) {
+    launch_sel_fill(p, sel, st);
+    return 1;
+  }
+  launch_mean_split(p, kmean, splits, khi, klo, 0, p.nbp, st);
+  const int rc = launch_gate_rows(p, q, khi, klo, sel, p.q0, p.S, st);
+  return rc < 0 ? rc : 2;
+}
+
+// Means of the complete blocks [j0, j1) (every one by default).
+void launch_pool(const Plan& p, const void* k, float* kmean, int splits, cudaStream_t st, int j0 = 0, int j1 = -1) {
+  if (j1 < 0 || j1 > p.nbp) j1 = p.nbp;
+  if (j1 <= j0) return;
+  dim3 grid(j1 - j0, p.Hkv, splits);
   launch_chained(moba::pool_kernel, grid, dim3(moba::kPoolThreads), 0, st, static_cast<const __nv_bfloat16*>(k), p.Hkv,
-                 p.B, p.nbp, splits, kmean);
+                 p.B, p.nbp, splits, j0, kmean);
 }
 
 // Optional per-stage device timing: an event after every stage, tagged with
@@ -552,8 +582,17 @@ int launch_route(const Plan& p, const moba::WindowGeom& wg, bool routed, uint8_t
   return n;
 }
 
+// Callbacks around each query window [w0, w0 + wlen) of run_forward, for
+// the pipelined copies of moba_fwd_host: `inputs` before the window's first
+// kernel (which may read q, k, v rows [0, w0 + wlen) and nothing beyond),
+// `done` after its merge (out rows and lse columns of the window are final).
+// With hooks, the pool, mean split and gate run window by window too.
+struct WindowHooks {
+  std::function<int(int64_t w0, int64_t wlen)> inputs, done;
+};
+
 int run_forward(const Plan& p, const DeviceInfo& dev, const void* q, const void* k, const void* v, void* out,
-                float* lse, uint8_t* ws, cudaStream_t st) {
+                float* lse, uint8_t* ws, cudaStream_t st, const WindowHooks* hooks = nullptr) {
   StageTimer* tm = &g_timer;
   tm->st = st;
   if (tm->on) tm->calls++;
@@ -577,18 +616,23 @@ int run_forward(const Plan& p, const DeviceInfo& dev, const void* q, const void*
   if (rc) return rc;
 
   tm->mark(-1);
-  if (p.P > 0 && p.k_eff < p.nb && p.nbp > 0 && !p.means) {
-    launch_pool(p, k, kmean, p.splits, st);
-    tm->count(1);
-    tm->mark(kPool);
-  }
-  {
-    const int n = launch_gate(p, q, kmean, mean_splits, reinterpret_cast<__nv_bfloat16*>(ws + p.o_khi),
-                              reinterpret_cast<__nv_bfloat16*>(ws + p.o_klo), sel, st);
+  const bool pooled = p.P > 0 && p.k_eff < p.nb && p.nbp > 0 && !p.means;
+  __nv_bfloat16* khi = reinterpret_cast<__nv_bfloat16*>(ws + p.o_khi);
+  __nv_bfloat16* klo = reinterpret_cast<__nv_bfloat16*>(ws + p.o_klo);
+  if (!hooks) {
+    if (pooled) {
+      launch_pool(p, k, kmean, p.splits, st);
+      tm->count(1);
+      tm->mark(kPool);
+    }
+    const int n = launch_gate(p, q, kmean, mean_splits, khi, klo, sel, st);
     if (n < 0) return -n;
     tm->count(n);
+    tm->mark(kGate);
+  } else if (gate_free(p)) {
+    launch_sel_fill(p, sel, st);  // reads no input
   }
-  tm->mark(kGate);
+  int j_done = 0;  // windowed: blocks pooled and split so far
 
   moba::AttnParams ap;
   ap.q = static_cast<const __nv_bfloat16*>(q);
@@ -608,6 +652,22 @@ int run_forward(const Plan& p, const DeviceInfo& dev, const void* q, const void*
 
   for (int64_t w0 = p.wbase; w0 < p.S; w0 += p.W) {
     const moba::WindowGeom wg = window_geom(p, w0);
+    if (hooks) {
+      int hr = hooks->inputs(w0, wg.wlen);
+      if (hr) return hr;
+      if (!gate_free(p)) {
+        // the blocks this window completes, then the gate of its rows (their
+        // past blocks all end at or before the window's end)
+        const int j_new = (int)std::min<int64_t>(p.nbp, (w0 + wg.wlen) / p.B);
+        if (j_new > j_done) {
+          if (pooled) launch_pool(p, k, kmean, p.splits, st, j_done, j_new);
+          launch_mean_split(p, kmean, mean_splits, khi, klo, j_done, j_new, st);
+          j_done = j_new;
+        }
+        hr = launch_gate_rows(p, q, khi, klo, sel, std::max(w0, p.q0), w0 + wg.wlen, st);
+        if (hr < 0) return -hr;
+      }
+    }
     const bool routed = window_routed(p, wg);
     const int nr = launch_route(p, wg, routed, ws, st);
     if (nr < 0) return -nr;
@@ -640,6 +700,10 @@ int run_forward(const Plan& p, const DeviceInfo& dev, const void* q, const void*
     else launch_chained(moba::merge_kernel<0>, mg, dim3(256), 0, st, mp);
     tm->count(1);
     tm->mark(kMerge);
+    if (hooks) {
+      const int hr = hooks->done(w0, wg.wlen);
+      if (hr) return hr;
+    }
   }
   MOBA_CUDA(cudaGetLastError());
   return MOBA_OK;
@@ -1103,6 +1167,139 @@ int varlen_impl(const void* q, const void* k, const void* v, const int64_t* cu, 
   return finish_call(direct_run(total, run, stream), stream);
 }
 
+cudaStream_t g_copy_streams[64][2] = {};
+
+// The internal copy streams of moba_fwd_host (host to device, device to
+// host), created once per device.
+int copy_streams(cudaStream_t* h2d, cudaStream_t* d2h) {
+  int dev = 0;
+  MOBA_CUDA(cudaGetDevice(&dev));
+  if (dev < 0 || dev >= 64) return fail(MOBA_ERR_UNSUPPORTED, "device index %d out of range", dev);
+  std::lock_guard<std::mutex> lk(g_dev_mu);
+  for (int i = 0; i < 2; ++i)
+    if (!g_copy_streams[dev][i]) MOBA_CUDA(cudaStreamCreateWithFlags(&g_copy_streams[dev][i], cudaStreamNonBlocking));
+  *h2d = g_copy_streams[dev][0];
+  *d2h = g_copy_streams[dev][1];
+  return MOBA_OK;
+}
+
+// moba_fwd on host buffers, pipelined by query window: the q, k, v rows a
+// window needs go up on one copy stream ahead of its kernels (pool, gate,
+// router, attention and merge all run window by window), and its out rows
+// and lse columns come back on another while the next window computes. So
+// only the first window's inputs and the last window's outputs are not
+// hidden behind kernels.
+int host_impl(const void* q_host, const void* k_host, const void* v_host, int64_t seqlen, int heads_q, int heads_kv,
+              int head_dim, int block_size, int topk, void* out_host, float* lse_host, cudaStream_t stream) {
+  g_err.clear();
+  if (!q_host || !k_host || !v_host || !out_host || !lse_host) return fail(MOBA_ERR_INVALID_ARG, "null pointer argument");
+  int rc = check_shape(seqlen, heads_q, heads_kv, head_dim, block_size, topk);
+  if (rc) return rc;
+  DeviceInfo dev;
+  rc = device_info(&dev);
+  if (rc) return rc;
+  rc = take_pending_status(dev, stream);
+  if (rc) return rc;
+  Plan p;
+  rc = make_plan(&p, seqlen, 0, heads_q, heads_kv, block_size, topk);
+  if (rc) return rc;
+  cudaStream_t h2d = nullptr, d2h = nullptr;
+  rc = copy_streams(&h2d, &d2h);
+  if (rc) return rc;
+  const size_t qrow = (size_t)heads_q * head_dim * 2, kvrow = (size_t)heads_kv * head_dim * 2;
+  const size_t qb = (size_t)seqlen * qrow, kb = (size_t)seqlen * kvrow, lb = (size_t)seqlen * heads_q * 4;
+  Carve c;
+  const size_t oq = c.take(qb), ok = c.take(kb), ov = c.take(kb), oo = c.take(qb), ol = c.take(lb);
+  keep_freed_scratch();
+  void* buf = nullptr;
+  cudaError_t e = cudaMallocAsync(&buf, c.off, stream);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return fail(MOBA_ERR_OOM, "device buffers of %zu bytes: %s", c.off, cudaGetErrorString(e));
+  }
+  void* ws = nullptr;
+  const size_t total = scratch_request(p.total);
+  e = cudaMallocAsync(&ws, total, stream);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    cudaFreeAsync(buf, stream);
+    cudaStreamSynchronize(stream);
+    return fail(MOBA_ERR_OOM, "scratch allocation of %zu bytes failed: %s", total, cudaGetErrorString(e));
+  }
+  uint8_t* b = static_cast<uint8_t*>(buf);
+  const uint8_t* qh = static_cast<const uint8_t*>(q_host);
+  const uint8_t* kh = static_cast<const uint8_t*>(k_host);
+  const uint8_t* vh = static_cast<const uint8_t*>(v_host);
+
+  // one event per window each way, plus the fork from and the joins back to
+  // the caller's stream
+  const int64_t nwin = (p.S - p.wbase + p.W - 1) / p.W;
+  std::vector<cudaEvent_t> ev(2 * (size_t)nwin + 3, nullptr);
+  for (auto& x : ev)
+    if (!rc && cudaEventCreateWithFlags(&x, cudaEventDisableTiming) != cudaSuccess)
+      rc = fail(MOBA_ERR_CUDA, "cudaEventCreate failed");
+  cudaEvent_t ev_alloc = ev[2 * nwin], ev_h2d_end = ev[2 * nwin + 1], ev_d2h_end = ev[2 * nwin + 2];
+  auto ev_in = [&](int64_t i) { return ev[2 * i]; };
+  auto ev_out = [&](int64_t i) { return ev[2 * i + 1]; };
+  bool h2d_forked = false, d2h_forked = false;
+  if (!rc) {
+    // the copy streams start once the buffers exist
+    if (cudaEventRecord(ev_alloc, stream) != cudaSuccess || cudaStreamWaitEvent(h2d, ev_alloc, 0) != cudaSuccess ||
+        cudaStreamWaitEvent(d2h, ev_alloc, 0) != cudaSuccess)
+      rc = fail(MOBA_ERR_CUDA, "forking the copy streams failed");
+    else
+      h2d_forked = d2h_forked = true;
+  }
+  // inputs, window by window: rows [done, w0 + wlen) of k (pool), q (gate),
+  // v (attention)
+  int64_t done = 0;
+  for (int64_t i = 0; i < nwin && !rc; ++i) {
+    const int64_t w0 = p.wbase + i * p.W, hi = std::min(p.S, w0 + p.W);
+    const int64_t n = hi - done;
+    if (cudaMemcpyAsync(b + ok + done * kvrow, kh + done * kvrow, n * kvrow, cudaMemcpyHostToDevice, h2d) !=
+            cudaSuccess ||
+        cudaMemcpyAsync(b + oq + done * qrow, qh + done * qrow, n * qrow, cudaMemcpyHostToDevice, h2d) != cudaSuccess ||
+        cudaMemcpyAsync(b + ov + done * kvrow, vh + done * kvrow, n * kvrow, cudaMemcpyHostToDevice, h2d) !=
+            cudaSuccess ||
+        cudaEventRecord(ev_in(i), h2d) != cudaSuccess)
+      rc = fail(MOBA_ERR_CUDA, "host to device copy failed: %s", cudaGetErrorString(cudaGetLastError()));
+    done = hi;
+  }
+  WindowHooks hooks;
+  hooks.inputs = [&](int64_t w0, int64_t) -> int {
+    if (cudaStreamWaitEvent(stream, ev_in((w0 - p.wbase) / p.W), 0) != cudaSuccess)
+      return fail(MOBA_ERR_CUDA, "waiting for the input copies failed");
+    return MOBA_OK;
+  };
+  hooks.done = [&](int64_t w0, int64_t wlen) -> int {
+    cudaEvent_t x = ev_out((w0 - p.wbase) / p.W);
+    if (cudaEventRecord(x, stream) != cudaSuccess || cudaStreamWaitEvent(d2h, x, 0) != cudaSuccess ||
+        cudaMemcpyAsync(static_cast<uint8_t*>(out_host) + w0 * qrow, b + oo + w0 * qrow, wlen * qrow,
+                        cudaMemcpyDeviceToHost, d2h) != cudaSuccess ||
+        cudaMemcpy2DAsync(lse_host + w0, (size_t)seqlen * 4, b + ol + w0 * 4, (size_t)seqlen * 4, wlen * 4,
+                          heads_q, cudaMemcpyDeviceToHost, d2h) != cudaSuccess)
+      return fail(MOBA_ERR_CUDA, "device to host copy failed: %s", cudaGetErrorString(cudaGetLastError()));
+    return MOBA_OK;
+  };
+  if (!rc)
+    rc = run_forward(p, dev, b + oq, b + ok, b + ov, b + oo, reinterpret_cast<float*>(b + ol),
+                     static_cast<uint8_t*>(ws), stream, &hooks);
+  // join both copy streams back before the buffers go
+  if (h2d_forked && (cudaEventRecord(ev_h2d_end, h2d) != cudaSuccess ||
+                     cudaStreamWaitEvent(stream, ev_h2d_end, 0) != cudaSuccess) && !rc)
+    rc = fail(MOBA_ERR_CUDA, "joining the copy streams failed");
+  if (d2h_forked && (cudaEventRecord(ev_d2h_end, d2h) != cudaSuccess ||
+                     cudaStreamWaitEvent(stream, ev_d2h_end, 0) != cudaSuccess) && !rc)
+    rc = fail(MOBA_ERR_CUDA, "joining the copy streams failed");
+  cudaFreeAsync(ws, stream);
+  cudaFreeAsync(buf, stream);
+  const cudaError_t es = cudaStreamSynchronize(stream);
+  for (auto& x : ev)
+    if (x) cudaEventDestroy(x);
+  if (!rc && es != cudaSuccess) rc = fail(MOBA_ERR_CUDA, "stream synchronise failed: %s", cudaGetErrorString(es));
+  return finish_call(rc, stream);
+}
+
 }  // namespace
 
 extern "C" {
@@ -1179,40 +1376,8 @@ int moba_profile_end(float* stage_ms, int* launches, int* calls) {
 int moba_fwd_host(const void* q_host, const void* k_host, const void* v_host, int64_t seqlen, int heads_q,
                   int heads_kv, int head_dim, int block_size, int topk, void* out_host, float* lse_host,
                   cudaStream_t stream) {
-  g_err.clear();
-  if (!q_host || !k_host || !v_host || !out_host || !lse_host) return fail(MOBA_ERR_INVALID_ARG, "null pointer argument");
-  int rc = check_shape(seqlen, heads_q, heads_kv, head_dim, block_size, topk);
-  if (rc) return rc;
-  DeviceInfo dev;
-  rc = device_info(&dev);
-  if (rc) return rc;
-  const size_t qb = (size_t)seqlen * heads_q * head_dim * 2, kb = (size_t)seqlen * heads_kv * head_dim * 2;
-  const size_t lb = (size_t)seqlen * heads_q * 4;
-  Carve c;
-  const size_t oq = c.take(qb), ok = c.take(kb), ov = c.take(kb), oo = c.take(qb), ol = c.take(lb);
-  keep_freed_scratch();
-  void* buf = nullptr;
-  cudaError_t e = cudaMallocAsync(&buf, c.off, stream);
-  if (e != cudaSuccess) {
-    cudaGetLastError();
-    return fail(MOBA_ERR_OOM, "device buffers of %zu bytes: %s", c.off, cudaGetErrorString(e));
-  }
-  uint8_t* b = static_cast<uint8_t*>(buf);
-  rc = MOBA_OK;
-  if (cudaMemcpyAsync(b + oq, q_host, qb, cudaMemcpyHostToDevice, stream) != cudaSuccess ||
-      cudaMemcpyAsync(b + ok, k_host, kb, cudaMemcpyHostToDevice, stream) != cudaSuccess ||
-      cudaMemcpyAsync(b + ov, v_host, kb, cudaMemcpyHostToDevice, stream) != cudaSuccess)
-    rc = fail(MOBA_ERR_CUDA, "host to device copy failed: %s", cudaGetErrorString(cudaGetLastError()));
-  if (!rc)
-    rc = fwd_impl(b + oq, b + ok, b + ov, seqlen, 0, heads_q, heads_kv, head_dim, block_size, topk, b + oo,
-                  reinterpret_cast<float*>(b + ol), stream, false);
-  if (!rc && (cudaMemcpyAsync(out_host, b + oo, qb, cudaMemcpyDeviceToHost, stream) != cudaSuccess ||
-              cudaMemcpyAsync(lse_host, b + ol, lb, cudaMemcpyDeviceToHost, stream) != cudaSuccess))
-    rc = fail(MOBA_ERR_CUDA, "device to host copy failed: %s", cudaGetErrorString(cudaGetLastError()));
-  cudaFreeAsync(buf, stream);
-  cudaError_t es = cudaStreamSynchronize(stream);
-  if (!rc && es != cudaSuccess) rc = fail(MOBA_ERR_CUDA, "stream synchronise failed: %s", cudaGetErrorString(es));
-  return rc;
+  return host_impl(q_host, k_host, v_host, seqlen, heads_q, heads_kv, head_dim, block_size, topk, out_host, lse_host,
+                   stream);
 }
 
 int moba_pool(const void* k, int64_t seqlen, int heads_kv, int head_dim, int block_size, float* kmean,

@@ -22,9 +22,9 @@ namespace moba {
 constexpr int kPoolThreads = 256;
 
 __global__ void __launch_bounds__(kPoolThreads) pool_kernel(const __nv_bfloat16* __restrict__ k, int Hkv, int B,
-                                                            int nbp, int splits, float* __restrict__ out) {
+                                                            int nbp, int splits, int j0, float* __restrict__ out) {
   grid_dependency_sync();
-  const int j = blockIdx.x, g = blockIdx.y, sp = blockIdx.z;
+  const int j = j0 + (int)blockIdx.x, g = blockIdx.y, sp = blockIdx.z;
   const int rows = B / splits;
   const int chunk = threadIdx.x & 15, rg = threadIdx.x >> 4;
   const int64_t row_stride = (int64_t)Hkv * kHeadDim;  // elements between consecutive tokens

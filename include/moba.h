@@ -204,11 +204,18 @@ int moba_bwd(const void* q, const void* k, const void* v, const void* out,
              void* dk, void* dv, cudaStream_t stream);
 
 /*
- * moba_fwd_host - moba_fwd on HOST buffers (same layouts): copies q, k, v to
- * the device, runs the forward pass and copies out and lse back, all on
- * `stream`, and synchronises the stream before returning. Host buffers that
- * are page-locked (cudaHostAlloc / pinned) copy fastest. Device buffers come
- * from the stream-ordered allocator and are released before returning.
+ * moba_fwd_host - moba_fwd on HOST buffers (same layouts and results):
+ * copies q, k, v to the device, runs the forward pass and copies out and lse
+ * back, and synchronises `stream` before returning. The work is pipelined
+ * by query window: the rows of q, k and v a window needs go up on a
+ * library-internal copy stream ahead of that window's kernels (pool, gate,
+ * router, attention and merge run window by window, on `stream`), and the
+ * window's out rows and lse columns come back on a second internal stream
+ * while the next window computes; both copy streams are forked from and
+ * joined back to `stream`. Host buffers that are page-locked (cudaHostAlloc /
+ * pinned) overlap; pageable ones are copied correctly but without overlap.
+ * Device buffers come from the stream-ordered allocator and are released
+ * before returning. out_host and lse_host must not alias the inputs.
  */
 int moba_fwd_host(const void* q_host, const void* k_host, const void* v_host,
                   int64_t seqlen, int heads_q, int heads_kv, int head_dim,

@@ -217,6 +217,30 @@ def test_host_entry_point_matches_device_entry_point():
     assert np.array_equal(lse_h.numpy(), lse_d)
 
 
+@pytest.mark.parametrize("S,Hq,Hkv,B,topk,window,pinned", [
+    (3000, 4, 2, 256, 3, 256, True),    # 12 windows, one per block
+    (3000, 6, 2, 256, 5, 384, True),    # G = 3 (Q gathered by cp.async); windows straddle blocks
+    (3000, 4, 2, 256, 3, 384, False),   # pageable host buffers
+    (1000, 2, 1, 256, 8, 256, True),    # topk >= blocks: no gate, windows still pipelined
+])
+def test_host_entry_point_pipelined_over_windows(monkeypatch, S, Hq, Hkv, B, topk, window, pinned):
+    # moba_fwd_host copies each window's rows up ahead of its kernels and its
+    # outputs back behind them; results are those of the device entry point
+    import block_sparse_long_fwd_b200 as moba
+    w, q, k, v = make_inputs(S, Hq, Hkv, B, topk, 91)
+    to_t = lambda a: torch.from_numpy(a.view(np.int16)).view(torch.bfloat16)
+    host = [to_t(x) for x in (q, k, v)]
+    if pinned:
+        host = [x.pin_memory() for x in host]
+    monkeypatch.setenv("MOBA_WINDOW", str(window))  # the same windows on both paths
+    out_h, lse_h = moba.fwd_host(*host, B, topk)
+    out_h2, lse_h2 = moba.fwd_host(*host, B, topk)
+    out_d, lse_d, _, _ = run_gpu(q, k, v, B, topk)
+    assert torch.equal(out_h, out_d) and torch.equal(out_h2, out_d)
+    assert np.array_equal(lse_h.numpy(), lse_d) and np.array_equal(lse_h2.numpy(), lse_d)
+    assert moba.device_status() == moba.MOBA_OK
+
+
 def test_repeated_calls_replay_a_graph_with_identical_results():
     # the third call with the same buffers replays a captured CUDA graph
     import block_sparse_long_fwd_b200 as moba
