@@ -85,7 +85,7 @@ __device__ __forceinline__ void fma_half8(float (&acc)[8], float w, uint4 o) {
 // three-pass path. The sums run in a fixed order either way: ascending
 // block, own block last.
 template <int NP>
-__global__ void __launch_bounds__(256, 3) merge_kernel(MergeParams m) {
+__global__ void __launch_bounds__(256, NP > 0 && NP <= 12 ? 4 : 3) merge_kernel(MergeParams m) {
   grid_dependency_sync();
   const WindowGeom& w = m.w;
   const int l16 = threadIdx.x & 15;

@@ -560,11 +560,12 @@ int launch_route(const Plan& p, const moba::WindowGeom& wg, bool routed, uint8_t
   const int nbk = p.Hkv * p.nbp;
   int n = 0;
   if (routed) {
-    dim3 gf((unsigned)((wg.wwords + 7) / 8), p.Hkv);
+    dim3 gf((unsigned)((wg.wwords + 3) / 4), p.Hkv);
     // the flags kernel writes only the words of picked blocks
     if (cudaMemsetAsync(flags, 0, (size_t)nbk * (size_t)wg.wwords * sizeof(uint32_t), st) != cudaSuccess)
       return -fail(MOBA_ERR_CUDA, "cudaMemsetAsync (route flags) failed");
-    launch_chained(moba::route_flags_kernel, gf, dim3(256), 0, st, sel, wg, flags);
+    launch_chained(moba::route_flags_kernel, gf, dim3(moba::kFlagsThreads),
+                   (size_t)moba::kFlagsThreads * std::max(p.P, 1) * sizeof(int32_t), st, sel, wg, flags);
     dim3 gb(p.nbp, p.Hkv);
     launch_chained(moba::route_count_kernel, gb, dim3(256), 0, st, static_cast<const uint32_t*>(flags), wg, cnt);
     n += 2;

@@ -53,18 +53,23 @@ __device__ __forceinline__ int64_t bucket_word_begin(const WindowGeom& w, int j)
   return wb < w.wwords ? wb : w.wwords;
 }
 
-// 1. grid (ceil(wwords / 8), Hkv), 256 threads: one warp per flag word (32
-// group-rows). The flag words start zeroed (the host clears them), so only
-// the blocks some row of the word picked are visited: each step takes the
-// smallest block still pending in any lane, and the lanes that picked it
-// advance to their next entry (a row's past entries are ascending).
-__global__ void __launch_bounds__(256) route_flags_kernel(const int32_t* __restrict__ sel, WindowGeom w,
-                                                          uint32_t* __restrict__ flags) {
+// 1. grid (ceil(wwords / 4), Hkv), 128 threads: one warp per flag word (32
+// group-rows); dynamic shared memory 128 * (k_eff - 1) ints. The flag words
+// start zeroed (the host clears them), so only the blocks some row of the
+// word picked are visited: each step takes the smallest block still pending
+// in any lane, and the lanes that picked it advance to their next entry (a
+// row's past entries are ascending). Every lane first copies its row's
+// entries into shared memory with all loads in flight, so the steps read
+// them at shared-memory latency.
+constexpr int kFlagsThreads = 128;
+__global__ void __launch_bounds__(kFlagsThreads) route_flags_kernel(const int32_t* __restrict__ sel, WindowGeom w,
+                                                                    uint32_t* __restrict__ flags) {
   grid_dependency_sync();
+  extern __shared__ int32_t ent[];  // [P][kFlagsThreads]: entry i of this thread's row at ent[i * 128 + tid]
   const int g = blockIdx.y;
   const int lane = threadIdx.x & 31;
-  const int64_t word = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
-  if (word >= w.wwords) return;
+  const int64_t word = (int64_t)blockIdx.x * (kFlagsThreads / 32) + (threadIdx.x >> 5);
+  if (word >= w.wwords) return;  // a whole warp: no block-wide barrier below
   const int64_t rr = word * 32 + lane;
   const int64_t tl = rr / w.G;
   const int64_t t = w.w0 + tl;
@@ -73,19 +78,23 @@ __global__ void __launch_bounds__(256) route_flags_kernel(const int32_t* __restr
   const int bt = valid ? (int)(t / w.B) : 0;
   const int P = w.k_eff - 1;
   const int32_t* srow = sel + ((int64_t)h * (w.S - w.q0) + (valid ? t - w.q0 : 0)) * w.k_eff;
+  int32_t* mine = ent + threadIdx.x;
+  for (int i = 0; i < P; ++i) {
+    const int v = valid ? __ldg(srow + i) : -1;
+    mine[i * kFlagsThreads] = (v >= 0 && v < bt) ? v : 0x7fffffff;
+  }
+  __syncwarp();
   int ptr = 0;
-  auto entry = [&](int i) -> int {
-    if (!valid || i >= P) return 0x7fffffff;
-    const int v = __ldg(srow + i);
-    return (v >= 0 && v < bt) ? v : 0x7fffffff;
-  };
-  int cur = entry(0);
+  int cur = P > 0 ? mine[0] : 0x7fffffff;
   uint32_t* dst = flags + (int64_t)g * w.nbp * w.wwords + word;
   for (;;) {
     const int j = __reduce_min_sync(0xffffffffu, cur);
     if (j == 0x7fffffff) break;
     const bool hit = (cur == j);
-    if (hit) cur = entry(++ptr);
+    if (hit) {
+      ++ptr;
+      cur = ptr < P ? mine[ptr * kFlagsThreads] : 0x7fffffff;
+    }
     const uint32_t bits = __ballot_sync(0xffffffffu, hit);
     if (lane == 0) dst[(int64_t)j * w.wwords] = bits;
   }
