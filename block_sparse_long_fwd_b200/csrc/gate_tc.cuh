@@ -90,6 +90,7 @@ struct GateParams {
   int64_t t_begin, t_end;  // the rows of tokens [t_begin, t_end) (q0 <= t_begin < t_end <= S)
   int Hq, G, B, nbp_pad, k_eff;
   int q_tma;               // 1: G divides 128 and tm_q is valid (Q tiles by TMA)
+  int one_pass;            // 1: the grid fits one wave, so latency beats issue: no separate pass 1
 };
 
 // Sorts N values (a power of two) in descending order: a bitonic network,
@@ -326,8 +327,13 @@ __global__ void __launch_bounds__(kGateTcThreads, GateCfg<KP>::kMinCtas)
     float* stg = reinterpret_cast<float*>(sM) + row * 32;
     const int nsc = (nchunks + Cfg::kScChunks - 1) / Cfg::kScChunks;
     // phases: pass 1 over the super-chunks, then pass 2 over them again; one
-    // super-chunk (or no bound): the passes share each phase's scores
-    const bool two_pass = Cfg::kBound && nsc > 1;
+    // super-chunk (or no bound, or a grid of one wave, where each CTA's chain
+    // of copies and products is the kernel's time): the passes share each
+    // phase's scores. Then the bound grows phase by phase: the maxima are
+    // sorted in place and later columns fold into the sorted slots, so the
+    // NG slots still hold NG distinct columns and their KP-th largest is
+    // still a lower bound on the row's KP-th best.
+    const bool two_pass = Cfg::kBound && nsc > 1 && !p.one_pass;
     const int nphase = two_pass ? 2 * nsc : nsc;
     float gm[NG];
 #pragma unroll
@@ -407,8 +413,8 @@ __global__ void __launch_bounds__(kGateTcThreads, GateCfg<KP>::kMinCtas)
           }
         }
         if (!two_pass || ph == nsc - 1) {
-          // every maximum is in: tau = the KP-th largest (-inf while fewer
-          // than KP groups hold a past block)
+          // the maxima so far are in: tau = the KP-th largest (-inf while
+          // fewer than KP slots hold a past block)
           sort_desc<NG>(gm);
           tau = gm[KP - 1];
         }

@@ -358,8 +358,10 @@ void launch_chained(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem
 
 template <int KP>
 void launch_gate_tc(const Plan& p, const CUtensorMap& mhi, const CUtensorMap& mlo, const CUtensorMap& mq,
-                    const moba::GateParams& gp, cudaStream_t st) {
+                    moba::GateParams gp, int sms, cudaStream_t st) {
   dim3 grid((unsigned)(((gp.t_end - gp.t_begin) * p.G + 127) / 128), p.Hkv);
+  // a grid that fits one wave (four CTAs per SM) takes the single pass
+  gp.one_pass = (int64_t)grid.x * grid.y <= 4 * (int64_t)sms ? 1 : 0;
   launch_chained(moba::gate_tc_kernel<KP>, grid, dim3(moba::kGateTcThreads), moba::GateCfg<KP>::kSmemBytes, st, mhi,
                  mlo, mq, gp);
 }
@@ -419,8 +421,13 @@ int launch_gate_rows(const Plan& p, const void* q, const __nv_bfloat16* khi, con
     rc = make_gate_q_map(&mq, q, p.S - p.q0, p.Hq, p.G);
     if (rc) return -rc;
   }
+  DeviceInfo dev;
+  rc = device_info(&dev);
+  if (rc) return -rc;
+  const int sms = dev.sms;
   moba::GateParams gp;
   gp.q_tma = q_tma ? 1 : 0;
+  gp.one_pass = 0;
   gp.q = static_cast<const __nv_bfloat16*>(q);
   gp.sel = sel;
   gp.S = p.S;
@@ -432,16 +439,16 @@ int launch_gate_rows(const Plan& p, const void* q, const __nv_bfloat16* khi, con
   gp.B = p.B;
   gp.nbp_pad = nbp_pad;
   gp.k_eff = p.k_eff;
-  if (p.P <= 2) launch_gate_tc<2>(p, mhi, mlo, mq, gp, st);
-  else if (p.P <= 4) launch_gate_tc<4>(p, mhi, mlo, mq, gp, st);
-  else if (p.P <= 8) launch_gate_tc<8>(p, mhi, mlo, mq, gp, st);
-  else if (p.P == 11) launch_gate_tc<11>(p, mhi, mlo, mq, gp, st);  // top-12: a list of exactly k - 1
-  else if (p.P <= 12) launch_gate_tc<12>(p, mhi, mlo, mq, gp, st);
-  else if (p.P <= 16) launch_gate_tc<16>(p, mhi, mlo, mq, gp, st);
-  else if (p.P <= 24) launch_gate_tc<24>(p, mhi, mlo, mq, gp, st);
-  else if (p.P <= 32) launch_gate_tc<32>(p, mhi, mlo, mq, gp, st);
-  else if (p.P <= 48) launch_gate_tc<48>(p, mhi, mlo, mq, gp, st);
-  else launch_gate_tc<64>(p, mhi, mlo, mq, gp, st);
+  if (p.P <= 2) launch_gate_tc<2>(p, mhi, mlo, mq, gp, sms, st);
+  else if (p.P <= 4) launch_gate_tc<4>(p, mhi, mlo, mq, gp, sms, st);
+  else if (p.P <= 8) launch_gate_tc<8>(p, mhi, mlo, mq, gp, sms, st);
+  else if (p.P == 11) launch_gate_tc<11>(p, mhi, mlo, mq, gp, sms, st);  // top-12: a list of exactly k - 1
+  else if (p.P <= 12) launch_gate_tc<12>(p, mhi, mlo, mq, gp, sms, st);
+  else if (p.P <= 16) launch_gate_tc<16>(p, mhi, mlo, mq, gp, sms, st);
+  else if (p.P <= 24) launch_gate_tc<24>(p, mhi, mlo, mq, gp, sms, st);
+  else if (p.P <= 32) launch_gate_tc<32>(p, mhi, mlo, mq, gp, sms, st);
+  else if (p.P <= 48) launch_gate_tc<48>(p, mhi, mlo, mq, gp, sms, st);
+  else launch_gate_tc<64>(p, mhi, mlo, mq, gp, sms, st);
   return 0;
 }
 

@@ -29,6 +29,11 @@ CASES = [
     (5000, 8,  2,   512, 6,    4999),   # decode, four q heads per kv head
     (2000, 2,  1,   256, 64,   1500),   # topk >= blocks: the dense path
     (300,  2,  1,   128, 3,    0),      # q_start 0 is the whole forward
+    # 320 past blocks (three 128-column super-chunks): the chunk's gate grid
+    # fits one wave and takes the single pass, the whole forward's (1,282
+    # CTAs) the two passes; the rows must still agree bit for bit
+    (41000, 4, 2,   128, 12,   40999),
+    (41000, 4, 2,   128, 12,   40700),
 ]
 
 
