@@ -6,7 +6,7 @@
 // to the lower block index.
 //
 // The score matrix is a GEMM: 128 query rows (group-rows rr = t*G + hl of
-// one kv head g) against 64 past blocks at a time. The block means are fp32;
+// one kv head g) against 32 or 64 past blocks at a time (a chunk). The block means are fp32;
 // they are split into two bf16 parts, hi = bf16(m) and lo = bf16(m - hi),
 // and S = Q.hi^T + Q.lo^T is accumulated in fp32 in TMEM. Q is exactly bf16,
 // so the only rounding beyond fp32 accumulation is |m - hi - lo| <= 2^-18 |m|
