@@ -710,18 +710,18 @@ __global__ void __launch_bounds__(kDkdvThreads, 1)
     }
   } else {
     // ------------------------------------------------ row gather (64 threads)
+    // slice m+1's row and per-row values are loaded while slice m's copies
+    // go out, and slice m+2's list entry one step earlier still, so a step
+    // does not wait on a global load before it can hand its slice over
     const int r = threadIdx.x - 9 * 32;  // row of the slice
     auto list_entry = [&](int m) -> int {
       return (m < n_rs && m * kSlice + r < nr) ? __ldg(d.list + lbase + m * kSlice + r) : -1;
     };
-    int lst_next = list_entry(0);
-    for (int m = 0; m < ns; ++m) {
-      const int st = m % kDkdvStages;
-      const int lst = lst_next;
-      lst_next = list_entry(m + 1);
-      if (!mbar_wait(&sh->q_empty[st], ((m / kDkdvStages) & 1) ^ 1, ab)) goto gather_done;
-      int64_t t = -1;
-      int h = 0;
+    // (t, h) of this thread's row in slice m (t = -1: no row)
+    auto row_of = [&](int m, int lst, int64_t& t, int& h) {
+      t = -1;
+      h = 0;
+      if (m >= ns) return;
       if (m < n_rs) {
         if (lst >= 0) {
           t = p.w0 + lst / p.G;
@@ -735,20 +735,40 @@ __global__ void __launch_bounds__(kDkdvThreads, 1)
           h = g * p.G + (int)(rr % p.G);
         }
       }
-      const int64_t off = t >= 0 ? (t * p.Hq + h) * kHeadDim : -1;
+    };
+    int64_t t_cur;
+    int h_cur;
+    row_of(0, list_entry(0), t_cur, h_cur);
+    float l2_cur = t_cur >= 0 ? __ldg(p.lse2 + (int64_t)h_cur * p.S + t_cur) : INFINITY;
+    float dd_cur = t_cur >= 0 ? __ldg(p.dd + (int64_t)h_cur * p.S + t_cur) : 0.f;
+    int lst_next = list_entry(1);
+    for (int m = 0; m < ns; ++m) {
+      const int st = m % kDkdvStages;
+      int64_t t_nx;
+      int h_nx;
+      row_of(m + 1, lst_next, t_nx, h_nx);
+      const float l2_nx = t_nx >= 0 ? __ldg(p.lse2 + (int64_t)h_nx * p.S + t_nx) : INFINITY;
+      const float dd_nx = t_nx >= 0 ? __ldg(p.dd + (int64_t)h_nx * p.S + t_nx) : 0.f;
+      lst_next = list_entry(m + 2);
+      if (!mbar_wait(&sh->q_empty[st], ((m / kDkdvStages) & 1) ^ 1, ab)) goto gather_done;
+      const int64_t off = t_cur >= 0 ? (t_cur * p.Hq + h_cur) * kHeadDim : -1;
       gather_slice_row(smem_u32(sQ + st * kSliceBytes), p.q, off, r);
       gather_slice_row(smem_u32(sdO + st * kSliceBytes), p.dout, off, r);
       cp_async_commit();
-      sh->lse2[st][r] = t >= 0 ? __ldg(p.lse2 + (int64_t)h * p.S + t) : INFINITY;
-      sh->dd[st][r] = t >= 0 ? __ldg(p.dd + (int64_t)h * p.S + t) : 0.f;
+      sh->lse2[st][r] = l2_cur;
+      sh->dd[st][r] = dd_cur;
       // routed rows lie past the block: no key of it is masked for them
-      sh->tok[st][r] = (t < 0 || m < n_rs) ? 0x7fffffff : (int)t;
+      sh->tok[st][r] = (t_cur < 0 || m < n_rs) ? 0x7fffffff : (int)t_cur;
       if (m > 0) {
         // the previous slice's copies have landed
         cp_async_wait_group<1>();
         fence_proxy_async_smem();
         mbar_arrive(&sh->q_full[(m - 1) % kDkdvStages]);
       }
+      t_cur = t_nx;
+      h_cur = h_nx;
+      l2_cur = l2_nx;
+      dd_cur = dd_nx;
     }
     cp_async_wait_group<0>();
     fence_proxy_async_smem();
