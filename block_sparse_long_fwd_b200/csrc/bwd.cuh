@@ -459,15 +459,21 @@ struct DkdvShared {
   alignas(16) int tok[kDkdvStages][kSlice];
 };
 
-// Row (t, h) of q / dO into row r of a 64-row slice (two 8 KB halves,
-// 128-byte swizzle); a missing row (off < 0) is zero-filled.
-__device__ __forceinline__ void gather_slice_row(uint32_t dst0, const __nv_bfloat16* base, int64_t off, int r) {
-  const bool valid = off >= 0;
-  const __nv_bfloat16* src = valid ? base + off : base;
+// The 32 rows rbase .. rbase+31 of a 64-row slice (two 8 KB halves, 128-byte
+// swizzle), one warp: lane l holds the element offset of row rbase + l
+// (-1: a missing row, zero-filled). Each copy instruction moves two whole
+// rows, 16 lanes per 256-byte row, so a warp instruction touches 4 cache
+// lines instead of one line in each of 32 rows.
+__device__ __forceinline__ void gather_slice_rows(uint32_t dst0, const __nv_bfloat16* base, int64_t off_mine,
+                                                  int rbase, int lane) {
+  const int c16 = lane & 15, half = c16 >> 3, c = c16 & 7;
 #pragma unroll
-  for (int c16 = 0; c16 < 16; ++c16) {
-    const int half = c16 >> 3, c = c16 & 7;
-    cp_async_16(dst0 + half * kSliceHalf + r * 128 + ((c ^ (r & 7)) << 4), src + (valid ? c16 * 8 : 0),
+  for (int i = 0; i < 16; ++i) {
+    const int rl = 2 * i + (lane >> 4);
+    const int64_t off = __shfl_sync(0xffffffffu, off_mine, rl);
+    const int r = rbase + rl;
+    const bool valid = off >= 0;
+    cp_async_16(dst0 + half * kSliceHalf + r * 128 + ((c ^ (r & 7)) << 4), valid ? base + off + c16 * 8 : base,
                 valid ? 16u : 0u);
   }
 }
@@ -750,10 +756,12 @@ __global__ void __launch_bounds__(kDkdvThreads, 1)
       const float l2_nx = t_nx >= 0 ? __ldg(p.lse2 + (int64_t)h_nx * p.S + t_nx) : INFINITY;
       const float dd_nx = t_nx >= 0 ? __ldg(p.dd + (int64_t)h_nx * p.S + t_nx) : 0.f;
       lst_next = list_entry(m + 2);
-      if (!mbar_wait(&sh->q_empty[st], ((m / kDkdvStages) & 1) ^ 1, ab)) goto gather_done;
+      // the copies below are warp-collective: a timeout sends the whole warp out
+      const bool ok = mbar_wait(&sh->q_empty[st], ((m / kDkdvStages) & 1) ^ 1, ab);
+      if (__any_sync(0xffffffffu, !ok)) goto gather_done;
       const int64_t off = t_cur >= 0 ? (t_cur * p.Hq + h_cur) * kHeadDim : -1;
-      gather_slice_row(smem_u32(sQ + st * kSliceBytes), p.q, off, r);
-      gather_slice_row(smem_u32(sdO + st * kSliceBytes), p.dout, off, r);
+      gather_slice_rows(smem_u32(sQ + st * kSliceBytes), p.q, off, r & ~31, r & 31);
+      gather_slice_rows(smem_u32(sdO + st * kSliceBytes), p.dout, off, r & ~31, r & 31);
       cp_async_commit();
       sh->lse2[st][r] = l2_cur;
       sh->dd[st][r] = dd_cur;
